@@ -1,0 +1,200 @@
+/*
+ * vq_moe.h -- C ABI of the VQ-MoE expert-path library (libvqmoe.so).
+ *
+ * The library computes the hot path of vector-quantised (VQ) MoE checkpoints
+ * on one NVIDIA B200 (sm_100a): expert weights are stored as packed
+ * log2(K)-bit indices into a per-module codebook of K fp16 centroids of
+ * d weights each, with one fp16 scale per (row, 64 weights), and dead
+ * "skipzero" rows dropped. The kernels reconstruct the weights on the fly and
+ * contract them with the activations of the tokens routed to each expert.
+ *
+ * Format (VQ model cards):
+ *   - Qwen3.5-397B-A17B-VQ-2.6bpw card, "Methodology": one index per
+ *     d-weight subvector into a per-tensor fp16 codebook, fp16 scale per
+ *     (row, 64 weights).
+ *   - Qwen3.5-397B-A17B-VQ-2.4bpw card, "Methodology": codes packed into
+ *     uint32 words, row-local, 32-code blocks. The bit order inside a block
+ *     is not printed; this library reads it as: code j of a row occupies
+ *     bits [j*b, j*b+b) of the row's bit string, bit i of the string being
+ *     bit (i % 32) of word i / 32 (least significant bit first).
+ *   - same card, "Changelog 2026-10-01 (vq-skipzero)": dead output rows
+ *     carry no codes or scales and output exact zeros.
+ *
+ * Conventions for every call:
+ *   - Pointers marked "device" are CUDA device pointers the caller owns; the
+ *     library never allocates, frees or retains them after the call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Device calls are asynchronous on that stream and never
+ *     synchronise the host; their results are valid once the stream has run.
+ *   - The return value reports argument errors and launch failures
+ *     synchronously. Nothing is launched when a call returns an error.
+ *   - fp16 and bf16 values are passed as their uint16 bit patterns.
+ */
+#ifndef VQ_MOE_H
+#define VQ_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum vq_status {
+    VQ_OK = 0,
+    VQ_ERR_ARG = 1,           /* NULL where a pointer is required, bad size or shape */
+    VQ_ERR_ALIGN = 2,         /* a pointer is not aligned as documented */
+    VQ_ERR_UNSUPPORTED = 3,   /* geometry (d, bits) or size the kernels do not implement */
+    VQ_ERR_WORKSPACE = 4,     /* workspace NULL, misaligned or smaller than required */
+    VQ_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
+    VQ_ERR_DEVICE_CHECK = 6   /* the device reported an inconsistency (see vq_moe_check) */
+} vq_status;
+
+/* Output element types. */
+enum { VQ_F32 = 0, VQ_BF16 = 1 };
+
+/*
+ * One VQ module: the weights of one (layer, projection) for E experts that
+ * share one codebook (reading of "per-tensor codebook": one codebook per
+ * projection of a layer, shared by all of that layer's experts).
+ *
+ * Expert e's weight matrix is W_e [rows, cols] with
+ *   W_e[r, c] = fp32(codebook[code_e(r, c / d)][c % d]) * fp32(scale_e[r, c / 64])
+ * where code_e(r, j) is the j-th b-bit code of row r.
+ *
+ * Requirements: d in {1, 2, 4, 8}; cols a multiple of 64 and of 32*d (whole
+ * 32-code blocks and whole scale groups); (d, bits) one of the implemented
+ * geometries (vq_geometry_supported).
+ */
+typedef struct vq_module {
+    int32_t E;        /* experts */
+    int32_t rows;     /* output features of each expert */
+    int32_t cols;     /* input features of each expert */
+    int32_t d;        /* weights per code (subvector length) */
+    int32_t bits;     /* code width b; the codebook has K = 2^bits entries */
+    /* device, 16-byte aligned: packed codes of the live rows, expert-major,
+     * live rows of one expert in increasing row order; each row is
+     * vq_packed_words(1, cols / d, bits) uint32 words. */
+    const uint32_t *codes;
+    /* device, 2-byte aligned: fp16 scales [live rows, cols / 64], same row order. */
+    const uint16_t *scales;
+    /* device, 16-byte aligned: fp16 codebook [2^bits, d]. */
+    const uint16_t *codebook;
+    /* device or NULL: live-row bitmap [E, ceil(rows / 32)]; bit (r % 32) of
+     * word r / 32 is 1 when row r of the expert is live. NULL: every row of
+     * every expert is live and expert e's row r is packed row e*rows + r. */
+    const uint32_t *live_bitmap;
+    /* device, required when live_bitmap is set: [E, ceil(rows / 32)], the
+     * packed-row index of the first live row at or after row 32*w of expert
+     * e (vq_live_rank builds it). */
+    const uint32_t *live_rank;
+} vq_module;
+
+/* A SwiGLU MoE layer: y = sum_j w_j * down_e( silu(gate_e x) * up_e x ).
+ * gate and up: rows = inter, cols = hidden; down: rows = hidden, cols = inter;
+ * all three with the same E. Each has its own codebook and geometry. */
+typedef struct vq_moe_layer {
+    vq_module gate;
+    vq_module up;
+    vq_module down;
+} vq_moe_layer;
+
+/* Human-readable name of a status. Never NULL. */
+const char *vq_status_str(vq_status s);
+
+/* 1 when the kernels implement geometry (d, bits), else 0. */
+int vq_geometry_supported(int32_t d, int32_t bits);
+
+/* ------------------------------------------------------------ host packing */
+
+/* uint32 words of `rows` packed rows of `ncode` codes of `bits` bits:
+ * rows * (ncode / 32) * bits (a 32-code block is exactly `bits` words).
+ * Returns 0 when ncode is not a positive multiple of 32 or bits not in 1..16. */
+size_t vq_packed_words(int64_t rows, int32_t ncode, int32_t bits);
+
+/* Host. Packs codes [E, rows, ncode] (uint16, values < 2^bits) into the
+ * row-local LSB-first layout, keeping only live rows when live_bitmap (host,
+ * [E, ceil(rows/32)]) is given (skipzero: live rows are byte-identical to a
+ * full packing). out: host, out_words >= vq_packed_words(live rows, ncode,
+ * bits). *rows_written receives the number of packed rows.
+ * Errors: VQ_ERR_ARG (NULL, bad sizes, a code >= 2^bits, out too small). */
+vq_status vq_pack(const uint16_t *codes, int32_t E, int32_t rows, int32_t ncode, int32_t bits,
+                  const uint32_t *live_bitmap, uint32_t *out, size_t out_words, size_t *rows_written);
+
+/* Host. Keeps the live rows of per-row fp16 scales [E, rows, ngroups]
+ * (ngroups = cols / 64) in the same order as vq_pack. */
+vq_status vq_pack_scales(const uint16_t *scales, int32_t E, int32_t rows, int32_t ngroups,
+                         const uint32_t *live_bitmap, uint16_t *out, size_t out_elems,
+                         size_t *rows_written);
+
+/* Host. Builds live_rank [E, ceil(rows/32)] from a live bitmap (both host).
+ * Bits at or beyond `rows` in the last word of an expert must be 0. */
+vq_status vq_live_rank(const uint32_t *live_bitmap, int32_t E, int32_t rows, uint32_t *rank_out);
+
+/* ------------------------------------------------------------ device calls */
+
+/* Diagnostic. codes_out: device uint16 [rows, cols/d]: the codes of expert
+ * `expert`'s rows; dead rows are filled with 0xFFFF. */
+vq_status vq_unpack(const vq_module *m, int32_t expert, uint16_t *codes_out, void *stream);
+
+/* Diagnostic. w_out: device fp32 [rows, cols]: the dequantised weights of
+ * `expert` (exact: the fp16 x fp16 product is exact in fp32); dead rows +0. */
+vq_status vq_dequant(const vq_module *m, int32_t expert, float *w_out, void *stream);
+
+/* y[t, r] = sum_c W_expert[r, c] * x[t, c] for t < T, accumulated in fp32.
+ * x: device bf16 [T, cols], 16-byte aligned. y: device [T, rows] of y_dtype
+ * (VQ_F32 or VQ_BF16, round to nearest even). Dead rows give +0.
+ * The contraction runs on tensor cores with the codebook entries and the
+ * activations in fp16 (bf16 -> fp16 is exact for |x| in [2^-14, 65504]) and
+ * the group scale applied in fp32 to each 64-column partial sum. */
+vq_status vq_gemv(const vq_module *m, int32_t expert, const uint16_t *x, int32_t T, void *y,
+                  int32_t y_dtype, void *stream);
+
+/* Top-k routing and expert bucketing of T tokens.
+ * logits: device fp32 [T, E]. Per token the top_k experts are taken in order
+ * of larger logit first, ties to the smaller expert index, NaN last.
+ * weights: renorm != 0 -> softmax over the selected logits; renorm == 0 ->
+ * the full softmax over all E experts, evaluated at the selected ones.
+ * Outputs (device): ids int32 [T, top_k]; weights fp32 [T, top_k];
+ * offsets int32 [E + 1] (exclusive prefix sums of per-expert pair counts);
+ * perm int32 [T * top_k]: pair indices p = t*top_k + j grouped by expert,
+ * increasing p inside each expert's bucket.
+ * Requires 1 <= top_k <= min(E, 32), E <= 4096, T * top_k < 2^31. */
+vq_status vq_route(const float *logits, int32_t T, int32_t E, int32_t top_k, int32_t renorm,
+                   int32_t *ids, float *weights, int32_t *offsets, int32_t *perm, void *stream);
+
+/* Which MoE path a workspace is sized for. */
+enum { VQ_MODE_DECODE = 0, VQ_MODE_PREFILL = 1 };
+
+/* Bytes of workspace vq_moe_decode (mode VQ_MODE_DECODE) or vq_moe_prefill
+ * (VQ_MODE_PREFILL) need for T tokens and top_k. 0 on invalid arguments. */
+size_t vq_moe_workspace_size(const vq_moe_layer *L, int32_t T, int32_t top_k, int32_t mode);
+
+/* MoE SwiGLU layer for decode-sized batches (a few tokens per expert):
+ *   y[t] = sum_j w[t, j] * W_down,e_j ( silu(W_gate,e_j x[t]) * (W_up,e_j x[t]) )
+ * with (e_j, w[t, j]) from vq_route on `logits` (device fp32 [T, E]).
+ * x: device bf16 [T, hidden], 16-byte aligned. y: device [T, hidden] of
+ * y_dtype. workspace: device, 256-byte aligned, at least
+ * vq_moe_workspace_size(L, T, top_k, VQ_MODE_DECODE) bytes; it holds the
+ * routing tables and the intermediate activations and may be reused by the
+ * next call once this one has run. Sums over experts run in slot order j,
+ * so results are deterministic. */
+vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, const float *logits,
+                        int32_t top_k, int32_t renorm, void *y, int32_t y_dtype, void *workspace,
+                        size_t ws_bytes, void *stream);
+
+/* The same layer for prefill-sized batches (many tokens per expert): per
+ * expert bucket a grouped GEMM on the tcgen05 tensor cores with the weight
+ * tiles decoded on chip. Same arguments and result definition as
+ * vq_moe_decode; workspace sized with VQ_MODE_PREFILL. Additionally requires
+ * every module's packed row to be a multiple of 16 bytes
+ * ((cols / d / 32) * bits divisible by 4). */
+vq_status vq_moe_prefill(const vq_moe_layer *L, const uint16_t *x, int32_t T, const float *logits,
+                         int32_t top_k, int32_t renorm, void *y, int32_t y_dtype, void *workspace,
+                         size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VQ_MOE_H */

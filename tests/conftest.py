@@ -13,6 +13,14 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "slow: long-running case")
 
 
+def pytest_sessionstart(session):
+    # build the oracle (gcc) and the library (nvcc, sm_100a) in-tree if they are stale
+    import oracle
+    oracle.build()
+    from vector_quantized_moe_b200 import build as libbuild
+    libbuild.build()
+
+
 @pytest.fixture(scope="session")
 def oracle_lib():
     import oracle

@@ -1,0 +1,105 @@
+"""CPU tests of the C ABI: the library loads, exports every symbol the header
+declares, and its host-side packing matches the oracle bit for bit. No call
+here launches GPU work."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+import vector_quantized_moe_b200 as vq
+
+
+def test_header_symbols_exported():
+    names = vq.header_functions()
+    assert len(names) >= 13
+    lib = ctypes.CDLL(vq.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    for s in range(7):
+        assert vq.status_str(s)
+    assert vq.status_str(1).startswith("VQ_ERR_ARG")
+
+
+def test_geometries():
+    for d, b in ((2, 8), (2, 10), (4, 9), (4, 11), (8, 12), (1, 3)):
+        assert vq.geometry_supported(d, b)
+    assert not vq.geometry_supported(3, 8)
+    assert not vq.geometry_supported(2, 16)
+
+
+@pytest.mark.parametrize("ncode,bits", [(32, 3), (64, 8), (96, 9), (128, 10), (64, 11), (32, 12), (64, 13), (32, 16)])
+def test_packed_words_closed_form(ncode, bits):
+    assert vq.packed_words(7, ncode, bits) == 7 * (ncode // 32) * bits
+    assert vq.packed_words(1, 33, bits) == 0
+
+
+@pytest.mark.parametrize("bits", [1, 3, 4, 8, 9, 10, 11, 12, 13, 16])
+def test_pack_matches_oracle(bits):
+    g = synth.rng(60, bits)
+    E, rows, ncode = 3, 37, 96
+    codes = synth.raw_codes((E, rows, ncode), bits, g)
+    bm = synth.live_bitmap(E, rows, 5, g)
+    for b in (None, bm):
+        assert np.array_equal(vq.pack(codes, bits, b), oracle.pack(codes, bits, b))
+
+
+def test_pack_scales_and_rank():
+    g = synth.rng(61)
+    E, rows, ng = 4, 70, 3
+    sc = synth.scales(E * rows, ng, g).reshape(E, rows, ng)
+    bm = synth.live_bitmap(E, rows, 11, g)
+    assert np.array_equal(vq.pack_scales(sc, bm), oracle.compact_rows(sc, bm))
+    rank = vq.live_rank(bm, rows)
+    # rank[e, w] = live rows before (e, 32*w), counted by brute force
+    live = [[(bm[e, r // 32] >> (r % 32)) & 1 for r in range(rows)] for e in range(E)]
+    for e in range(E):
+        for w in range(bm.shape[1]):
+            assert rank[e, w] == sum(sum(live[x]) for x in range(e)) + sum(live[e][: 32 * w])
+
+
+def test_pack_rejects_out_of_range_code():
+    codes = np.zeros((1, 1, 32), dtype=np.uint16)
+    codes[0, 0, 5] = 8
+    with pytest.raises(vq.VQError):
+        vq.pack(codes, 3)
+
+
+def test_live_rank_rejects_bits_beyond_rows():
+    bm = np.array([[0xFFFFFFFF]], dtype=np.uint32)
+    with pytest.raises(vq.VQError):
+        vq.live_rank(bm, 20)
+
+
+def _null_module(**kw):
+    m = dict(E=2, rows=64, cols=128, d=2, bits=8, codes=256, scales=512, codebook=1024, live_bitmap=None,
+             live_rank=None)
+    m.update(kw)
+    return vq.vq_module(m["E"], m["rows"], m["cols"], m["d"], m["bits"], m["codes"], m["scales"], m["codebook"],
+                        m["live_bitmap"], m["live_rank"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(codes=None), 1), (dict(cols=100), 1), (dict(d=3), 1), (dict(bits=7), 3), (dict(codes=264), 2),
+    (dict(live_bitmap=4096), 1), (dict(E=0), 1),
+])
+def test_argument_errors_before_launch(kw, status):
+    # fake (never dereferenced) pointers: validation fails before any CUDA call
+    m = _null_module(**kw)
+    rc = vq._L().vq_gemv(ctypes.byref(m), 0, 4096, 1, 8192, 0, None)
+    assert rc == status
+
+
+def test_workspace_size_monotone():
+    m = _null_module()
+    down = _null_module(rows=128, cols=64)
+    L = vq.vq_moe_layer(m, m, down)
+    a = vq._L().vq_moe_workspace_size(ctypes.byref(L), 4, 1, 0)
+    b = vq._L().vq_moe_workspace_size(ctypes.byref(L), 64, 1, 0)
+    assert 0 < a < b
+    assert vq._L().vq_moe_workspace_size(ctypes.byref(L), 4, 3, 0) == 0   # top_k > E

@@ -1,0 +1,454 @@
+// C ABI of the VQ-MoE library: argument validation, host-side packing,
+// workspace layout and kernel dispatch. See include/vq_moe.h.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+
+#include "vq_internal.h"
+
+namespace vq {
+
+int num_sms()
+{
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            sms = 148;
+    }
+    return sms;
+}
+
+namespace {
+
+constexpr size_t CODEBOOK_SMEM_BUDGET = 100 * 1024;   // replicated codebook per CTA
+
+bool geometry_ok(int d, int bits)
+{
+#define VQ_GEO_OK(D_, B_) \
+    if (d == D_ && bits == B_) return true;
+    VQ_GEOMETRIES(VQ_GEO_OK)
+#undef VQ_GEO_OK
+    return false;
+}
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+vq_status check_module(const vq_module *m)
+{
+    if (!m || !m->codes || !m->scales || !m->codebook)
+        return VQ_ERR_ARG;
+    if (m->E < 1 || m->rows < 1 || m->cols < 64 || m->cols % 64 != 0)
+        return VQ_ERR_ARG;
+    if (m->d != 1 && m->d != 2 && m->d != 4 && m->d != 8)
+        return VQ_ERR_ARG;
+    if (m->cols % (32 * m->d) != 0 || m->bits < 1 || m->bits > 16)
+        return VQ_ERR_ARG;
+    if (m->live_bitmap && !m->live_rank)
+        return VQ_ERR_ARG;
+    if (!geometry_ok(m->d, m->bits))
+        return VQ_ERR_UNSUPPORTED;
+    if (!aligned(m->codes, 16) || !aligned(m->codebook, 16) || !aligned(m->scales, 2))
+        return VQ_ERR_ALIGN;
+    if ((m->live_bitmap && !aligned(m->live_bitmap, 4)) || (m->live_rank && !aligned(m->live_rank, 4)))
+        return VQ_ERR_ALIGN;
+    return VQ_OK;
+}
+
+vq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? VQ_OK : VQ_ERR_CUDA; }
+
+// Split of the 64-column groups so that enough warps have work.
+int choose_slices(long n_act_est, int rows, int ngroups, int nmod, long target_items)
+{
+    const long items1 = n_act_est * ((rows + 31) / 32) * nmod;
+    int s = 1;
+    while (ngroups % (2 * s) == 0 && ngroups / (2 * s) >= 2 && items1 * s < target_items)
+        s *= 2;
+    return s;
+}
+
+struct DecodePlan {
+    int T, k, E, H, I;
+    int sa, sb;                  // slices of the gate/up and down passes
+    RoutingLayout r;
+    size_t off_G, off_U, off_h, off_D;
+    size_t total;
+};
+
+vq_status check_layer(const vq_moe_layer *L)
+{
+    if (!L)
+        return VQ_ERR_ARG;
+    vq_status st;
+    if ((st = check_module(&L->gate)) != VQ_OK || (st = check_module(&L->up)) != VQ_OK ||
+        (st = check_module(&L->down)) != VQ_OK)
+        return st;
+    const int E = L->gate.E, H = L->gate.cols, I = L->gate.rows;
+    if (L->up.E != E || L->down.E != E || L->up.cols != H || L->up.rows != I || L->down.rows != H ||
+        L->down.cols != I)
+        return VQ_ERR_ARG;
+    return VQ_OK;
+}
+
+long target_items() { return (long)num_sms() * 16 * 2; }
+
+DecodePlan plan_decode(const vq_moe_layer *L, int T, int k)
+{
+    DecodePlan p{};
+    p.T = T;
+    p.k = k;
+    p.E = L->gate.E;
+    p.H = L->gate.cols;
+    p.I = L->gate.rows;
+    const long n_act = std::min<long>(p.E, (long)T * k);
+    p.sa = choose_slices(n_act, p.I, p.H / 64, 2, target_items());
+    p.sb = choose_slices(n_act, p.H, p.I / 64, 1, target_items());
+    size_t o = 0;
+    p.r = plan_routing(o, T, k, p.E);
+    const size_t tk = (size_t)T * k;
+    p.off_G = o; o = align_up(o + (size_t)p.sa * tk * p.I * 4, 256);
+    p.off_U = o; o = align_up(o + (size_t)p.sa * tk * p.I * 4, 256);
+    p.off_h = o; o = align_up(o + tk * p.I * 2, 256);
+    p.off_D = o; o = align_up(o + (size_t)p.sb * tk * p.H * 4, 256);
+    p.total = o;
+    return p;
+}
+
+}  // namespace
+
+ModDev make_moddev(const vq_module &m)
+{
+    ModDev d{};
+    d.codes = m.codes;
+    d.scales = m.scales;
+    d.codebook = m.codebook;
+    d.bitmap = m.live_bitmap;
+    d.rank = m.live_rank;
+    d.E = m.E;
+    d.rows = m.rows;
+    d.cols = m.cols;
+    d.d = m.d;
+    d.bits = m.bits;
+    d.row_words = (m.cols / m.d / 32) * m.bits;
+    d.ngroups = m.cols / 64;
+    d.bm_words = (m.rows + 31) / 32;
+    const size_t entry = std::max(4, 2 * m.d);
+    const int full = (int)(128 / entry);
+    int rep = full;
+    while (rep > 1 && ((size_t)1 << m.bits) * entry * rep > CODEBOOK_SMEM_BUDGET)
+        rep /= 2;
+    d.rep = rep;
+    d.log_rep = 0;
+    while ((1 << d.log_rep) < rep)
+        ++d.log_rep;
+    return d;
+}
+
+}  // namespace vq
+
+using namespace vq;
+
+extern "C" {
+
+const char *vq_status_str(vq_status s)
+{
+    switch (s) {
+    case VQ_OK: return "VQ_OK";
+    case VQ_ERR_ARG: return "VQ_ERR_ARG: invalid argument";
+    case VQ_ERR_ALIGN: return "VQ_ERR_ALIGN: misaligned pointer";
+    case VQ_ERR_UNSUPPORTED: return "VQ_ERR_UNSUPPORTED: geometry or size not implemented";
+    case VQ_ERR_WORKSPACE: return "VQ_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case VQ_ERR_CUDA: return "VQ_ERR_CUDA: CUDA runtime error";
+    case VQ_ERR_DEVICE_CHECK: return "VQ_ERR_DEVICE_CHECK: device-side check failed";
+    }
+    return "unknown vq_status";
+}
+
+int vq_geometry_supported(int32_t d, int32_t bits) { return geometry_ok(d, bits) ? 1 : 0; }
+
+size_t vq_packed_words(int64_t rows, int32_t ncode, int32_t bits)
+{
+    if (rows < 0 || ncode <= 0 || ncode % 32 != 0 || bits < 1 || bits > 16)
+        return 0;
+    return (size_t)rows * (size_t)(ncode / 32) * (size_t)bits;
+}
+
+static int bm_live(const uint32_t *bm, int rows, int e, int r)
+{
+    if (!bm)
+        return 1;
+    const int nw = (rows + 31) / 32;
+    return (bm[(size_t)e * nw + r / 32] >> (r % 32)) & 1;
+}
+
+vq_status vq_pack(const uint16_t *codes, int32_t E, int32_t rows, int32_t ncode, int32_t bits,
+                  const uint32_t *live_bitmap, uint32_t *out, size_t out_words, size_t *rows_written)
+{
+    if (!codes || !out || E < 1 || rows < 1 || ncode <= 0 || ncode % 32 != 0 || bits < 1 || bits > 16)
+        return VQ_ERR_ARG;
+    const size_t rw = vq_packed_words(1, ncode, bits);
+    size_t n = 0;
+    for (int e = 0; e < E; ++e)
+        for (int r = 0; r < rows; ++r)
+            if (bm_live(live_bitmap, rows, e, r))
+                ++n;
+    if (out_words < n * rw)
+        return VQ_ERR_ARG;
+    const uint32_t lim = 1u << bits;
+    size_t row = 0;
+    for (int e = 0; e < E; ++e)
+        for (int r = 0; r < rows; ++r) {
+            if (!bm_live(live_bitmap, rows, e, r))
+                continue;
+            const uint16_t *src = codes + ((size_t)e * rows + r) * ncode;
+            uint32_t *dst = out + row * rw;
+            std::memset(dst, 0, rw * sizeof(uint32_t));
+            for (int j = 0; j < ncode; ++j) {
+                const uint32_t v = src[j];
+                if (v >= lim)
+                    return VQ_ERR_ARG;
+                const size_t bit = (size_t)j * bits;
+                const size_t w = bit >> 5;
+                const unsigned sh = bit & 31;
+                dst[w] |= v << sh;
+                if (sh + bits > 32)
+                    dst[w + 1] |= v >> (32 - sh);
+            }
+            ++row;
+        }
+    if (rows_written)
+        *rows_written = n;
+    return VQ_OK;
+}
+
+vq_status vq_pack_scales(const uint16_t *scales, int32_t E, int32_t rows, int32_t ngroups,
+                         const uint32_t *live_bitmap, uint16_t *out, size_t out_elems, size_t *rows_written)
+{
+    if (!scales || !out || E < 1 || rows < 1 || ngroups < 1)
+        return VQ_ERR_ARG;
+    size_t n = 0;
+    for (int e = 0; e < E; ++e)
+        for (int r = 0; r < rows; ++r)
+            n += bm_live(live_bitmap, rows, e, r);
+    if (out_elems < n * (size_t)ngroups)
+        return VQ_ERR_ARG;
+    size_t row = 0;
+    for (int e = 0; e < E; ++e)
+        for (int r = 0; r < rows; ++r)
+            if (bm_live(live_bitmap, rows, e, r)) {
+                std::memcpy(out + row * ngroups, scales + ((size_t)e * rows + r) * ngroups,
+                            (size_t)ngroups * sizeof(uint16_t));
+                ++row;
+            }
+    if (rows_written)
+        *rows_written = n;
+    return VQ_OK;
+}
+
+vq_status vq_live_rank(const uint32_t *live_bitmap, int32_t E, int32_t rows, uint32_t *rank_out)
+{
+    if (!live_bitmap || !rank_out || E < 1 || rows < 1)
+        return VQ_ERR_ARG;
+    const int nw = (rows + 31) / 32;
+    uint64_t run = 0;
+    for (int e = 0; e < E; ++e)
+        for (int w = 0; w < nw; ++w) {
+            rank_out[(size_t)e * nw + w] = (uint32_t)run;
+            uint32_t word = live_bitmap[(size_t)e * nw + w];
+            if (w == nw - 1 && rows % 32 != 0 && (word >> (rows % 32)) != 0)
+                return VQ_ERR_ARG;
+            run += (uint64_t)__builtin_popcount(word);
+        }
+    if (run > 0xFFFFFFFFull)
+        return VQ_ERR_ARG;
+    return VQ_OK;
+}
+
+vq_status vq_unpack(const vq_module *m, int32_t expert, uint16_t *codes_out, void *stream)
+{
+    vq_status st = check_module(m);
+    if (st != VQ_OK)
+        return st;
+    if (!codes_out || expert < 0 || expert >= m->E)
+        return VQ_ERR_ARG;
+    return cuda_status(launch_unpack(make_moddev(*m), expert, codes_out, (cudaStream_t)stream));
+}
+
+vq_status vq_dequant(const vq_module *m, int32_t expert, float *w_out, void *stream)
+{
+    vq_status st = check_module(m);
+    if (st != VQ_OK)
+        return st;
+    if (!w_out || expert < 0 || expert >= m->E)
+        return VQ_ERR_ARG;
+    return cuda_status(launch_dequant(make_moddev(*m), expert, w_out, (cudaStream_t)stream));
+}
+
+vq_status vq_gemv(const vq_module *m, int32_t expert, const uint16_t *x, int32_t T, void *y, int32_t y_dtype,
+                  void *stream)
+{
+    vq_status st = check_module(m);
+    if (st != VQ_OK)
+        return st;
+    if (!x || !y || T < 0 || expert < 0 || expert >= m->E || (y_dtype != VQ_F32 && y_dtype != VQ_BF16))
+        return VQ_ERR_ARG;
+    if (!aligned(x, 16))
+        return VQ_ERR_ALIGN;
+    if (T == 0)
+        return VQ_OK;
+    GemvArgs a{};
+    a.mod[0] = make_moddev(*m);
+    a.mod[1] = a.mod[0];
+    a.nmod = 1;
+    a.act = x;
+    a.act_bf16 = 1;
+    a.expert = expert;
+    a.T = T;
+    a.slices = 1;
+    a.out[0] = y;
+    a.out[1] = y;
+    a.out_dtype = y_dtype;
+    a.out_slice_stride = 0;
+    const int occ = gemv_ctas_per_sm(m->d, m->bits, gemv_smem_bytes(a.mod[0]));
+    const long items = (long)((m->rows + 31) / 32);
+    const int ctas = (int)std::max<long>(1, std::min<long>((long)num_sms() * occ, (items + 7) / 8));
+    return cuda_status(launch_gemv(a, ctas, (cudaStream_t)stream, false));
+}
+
+vq_status vq_route(const float *logits, int32_t T, int32_t E, int32_t top_k, int32_t renorm, int32_t *ids,
+                   float *weights, int32_t *offsets, int32_t *perm, void *stream)
+{
+    if (!logits || !ids || !weights || !offsets || !perm || T < 0 || E < 1 || E > 4096 || top_k < 1 ||
+        top_k > std::min(E, 32) || (long)T * top_k >= (1L << 31))
+        return VQ_ERR_ARG;
+    return cuda_status(launch_route(logits, T, E, top_k, renorm, ids, weights, offsets, perm, nullptr, nullptr,
+                                    nullptr, (cudaStream_t)stream, false));
+}
+
+size_t vq_moe_workspace_size(const vq_moe_layer *L, int32_t T, int32_t top_k, int32_t mode)
+{
+    if (check_layer(L) != VQ_OK || T < 0 || top_k < 1 || top_k > std::min(L->gate.E, 32))
+        return 0;
+    if (mode == VQ_MODE_DECODE)
+        return plan_decode(L, T, top_k).total;
+    if (mode == VQ_MODE_PREFILL)
+        return prefill_workspace_size(L, T, top_k);
+    return 0;
+}
+
+static vq_status check_moe_args(const vq_moe_layer *L, const uint16_t *x, int32_t T, const float *logits,
+                                int32_t top_k, void *y, int32_t y_dtype, void *workspace)
+{
+    vq_status st = check_layer(L);
+    if (st != VQ_OK)
+        return st;
+    if (!x || !logits || !y || T < 0 || top_k < 1 || top_k > std::min(L->gate.E, 32) || L->gate.E > 4096 ||
+        (y_dtype != VQ_F32 && y_dtype != VQ_BF16) || (long)T * top_k >= (1L << 31))
+        return VQ_ERR_ARG;
+    if (!aligned(x, 16))
+        return VQ_ERR_ALIGN;
+    if (!workspace || !aligned(workspace, 256))
+        return VQ_ERR_WORKSPACE;
+    return VQ_OK;
+}
+
+vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, const float *logits, int32_t top_k,
+                        int32_t renorm, void *y, int32_t y_dtype, void *workspace, size_t ws_bytes, void *stream)
+{
+    vq_status st = check_moe_args(L, x, T, logits, top_k, y, y_dtype, workspace);
+    if (st != VQ_OK)
+        return st;
+    if (T == 0)
+        return VQ_OK;
+    const DecodePlan p = plan_decode(L, T, top_k);
+    if (ws_bytes < p.total)
+        return VQ_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    int32_t *ids = ws_at<int32_t>(workspace, p.r.ids);
+    float *w = ws_at<float>(workspace, p.r.w);
+    int32_t *offsets = ws_at<int32_t>(workspace, p.r.offsets);
+    int32_t *perm = ws_at<int32_t>(workspace, p.r.perm);
+    int32_t *pos = ws_at<int32_t>(workspace, p.r.pos);
+    int32_t *active = ws_at<int32_t>(workspace, p.r.active);
+    int32_t *nact = ws_at<int32_t>(workspace, p.r.nact);
+    float *G = ws_at<float>(workspace, p.off_G);
+    float *U = ws_at<float>(workspace, p.off_U);
+    __half *h = ws_at<__half>(workspace, p.off_h);
+    float *D = ws_at<float>(workspace, p.off_D);
+    const long tk = (long)T * top_k;
+
+    cudaError_t err = launch_route(logits, T, p.E, top_k, renorm, ids, w, offsets, perm, pos, active, nact, s, true);
+    if (err != cudaSuccess)
+        return VQ_ERR_CUDA;
+
+    // gate and up: one launch when they share a geometry
+    GemvArgs a{};
+    a.act = x;
+    a.act_bf16 = 1;
+    a.offsets = offsets;
+    a.perm = perm;
+    a.top_k = top_k;
+    a.active = active;
+    a.n_active = nact;
+    a.slices = p.sa;
+    a.out_dtype = VQ_F32;
+    a.out_slice_stride = tk * p.I;
+    const ModDev mg = make_moddev(L->gate), mu = make_moddev(L->up);
+    const bool same = mg.d == mu.d && mg.bits == mu.bits && mg.rep == mu.rep;
+    const int sms = num_sms();
+    if (same) {
+        a.mod[0] = mg;
+        a.mod[1] = mu;
+        a.nmod = 2;
+        a.out[0] = G;
+        a.out[1] = U;
+        const int occ = gemv_ctas_per_sm(mg.d, mg.bits, gemv_smem_bytes(mg));
+        err = launch_gemv(a, std::max(1, sms * occ / 2), s, true);
+    } else {
+        a.nmod = 1;
+        a.mod[0] = a.mod[1] = mg;
+        a.out[0] = a.out[1] = G;
+        err = launch_gemv(a, sms * gemv_ctas_per_sm(mg.d, mg.bits, gemv_smem_bytes(mg)), s, true);
+        if (err == cudaSuccess) {
+            a.mod[0] = a.mod[1] = mu;
+            a.out[0] = a.out[1] = U;
+            err = launch_gemv(a, sms * gemv_ctas_per_sm(mu.d, mu.bits, gemv_smem_bytes(mu)), s, true);
+        }
+    }
+    if (err != cudaSuccess)
+        return VQ_ERR_CUDA;
+
+    err = launch_swiglu(G, U, p.sa, tk * p.I, (int)tk, p.I, h, s, true);
+    if (err != cudaSuccess)
+        return VQ_ERR_CUDA;
+
+    GemvArgs b = a;
+    const ModDev md = make_moddev(L->down);
+    b.mod[0] = b.mod[1] = md;
+    b.nmod = 1;
+    b.act = h;
+    b.act_bf16 = 0;
+    b.slices = p.sb;
+    b.out[0] = b.out[1] = D;
+    b.out_slice_stride = tk * p.H;
+    err = launch_gemv(b, sms * gemv_ctas_per_sm(md.d, md.bits, gemv_smem_bytes(md)), s, true);
+    if (err != cudaSuccess)
+        return VQ_ERR_CUDA;
+
+    err = launch_combine(D, p.sb, tk * p.H, w, pos, T, top_k, p.H, y, y_dtype, s, true);
+    return cuda_status(err);
+}
+
+vq_status vq_moe_prefill(const vq_moe_layer *L, const uint16_t *x, int32_t T, const float *logits, int32_t top_k,
+                         int32_t renorm, void *y, int32_t y_dtype, void *workspace, size_t ws_bytes, void *stream)
+{
+    vq_status st = check_moe_args(L, x, T, logits, top_k, y, y_dtype, workspace);
+    if (st != VQ_OK)
+        return st;
+    return run_prefill(L, x, T, logits, top_k, renorm, y, y_dtype, workspace, ws_bytes, (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,104 @@
+// Internal interface between the C ABI (vq_api.cpp) and the kernel launchers.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/vq_moe.h"
+
+// The geometries (d, bits) the kernels are instantiated for.
+#define VQ_GEOMETRIES(X) \
+    X(1, 3) X(1, 4) X(2, 8) X(2, 10) X(2, 11) X(4, 8) X(4, 9) X(4, 11) X(4, 13) X(8, 12)
+
+namespace vq {
+
+// A module as the kernels see it.
+struct ModDev {
+    const uint32_t *codes;
+    const uint16_t *scales;
+    const uint16_t *codebook;
+    const uint32_t *bitmap;
+    const uint32_t *rank;
+    int E, rows, cols, d, bits;
+    int row_words;   // uint32 words per packed row
+    int ngroups;     // cols / 64
+    int bm_words;    // ceil(rows / 32)
+    int rep;         // codebook replicas in shared memory (power of two)
+    int log_rep;
+};
+
+ModDev make_moddev(const vq_module &m);
+
+// Grouped GEMV over the experts that received tokens (tensor-core m16n8k16).
+// One launch covers nmod modules that share the same activation and geometry.
+struct GemvArgs {
+    ModDev mod[2];
+    int nmod;
+    const void *act;        // activation rows: bf16 [T, cols] (act_bf16) or fp16 [slots, cols]
+    int act_bf16;
+    const int32_t *offsets; // [E + 1] bucket offsets; NULL -> single expert over T tokens
+    const int32_t *perm;    // [T*k] pair ids in bucket order (bf16 act: token = perm[q] / top_k)
+    int top_k;
+    const int32_t *active;  // experts with tokens, ascending
+    const int32_t *n_active;
+    int expert;             // single-expert mode
+    int T;                  // single-expert mode: tokens
+    int slices;             // split of the 64-column groups (partial sums per slice)
+    void *out[2];           // per module: [slices][slots][rows]
+    int out_dtype;          // VQ_F32 or VQ_BF16
+    long out_slice_stride;  // elements between slices
+};
+
+cudaError_t launch_gemv(const GemvArgs &a, int ctas_per_mod, cudaStream_t s, bool pdl);
+int gemv_ctas_per_sm(int d, int bits, size_t smem);
+size_t gemv_smem_bytes(const ModDev &m);
+
+// Routing + bucketing in one CTA. pos = inverse of perm; active/n_active as above.
+cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int32_t *ids, float *w,
+                         int32_t *offsets, int32_t *perm, int32_t *pos, int32_t *active, int32_t *n_active,
+                         cudaStream_t s, bool pdl);
+
+// h[q, c] = fp16( silu(sum_s G[s, q, c]) * sum_s U[s, q, c] )
+cudaError_t launch_swiglu(const float *G, const float *U, int slices, long slice_stride, int slots, int inter,
+                          __half *h, cudaStream_t s, bool pdl);
+
+// y[t, r] = sum_j w[t*k + j] * sum_s D[s, pos[t*k + j], r]
+cudaError_t launch_combine(const float *D, int slices, long slice_stride, const float *w, const int32_t *pos,
+                           int T, int k, int hidden, void *y, int y_dtype, cudaStream_t s, bool pdl);
+
+cudaError_t launch_unpack(const ModDev &m, int expert, uint16_t *out, cudaStream_t s);
+cudaError_t launch_dequant(const ModDev &m, int expert, float *out, cudaStream_t s);
+
+int num_sms();
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Routing tables at the front of a MoE workspace (each section 256-byte aligned).
+struct RoutingLayout {
+    size_t ids, w, offsets, perm, pos, active, nact;
+};
+inline RoutingLayout plan_routing(size_t &o, int T, int k, int E)
+{
+    RoutingLayout r;
+    const size_t tk = (size_t)T * k;
+    r.ids = o;     o = align_up(o + tk * 4, 256);
+    r.w = o;       o = align_up(o + tk * 4, 256);
+    r.offsets = o; o = align_up(o + (size_t)(E + 1) * 4, 256);
+    r.perm = o;    o = align_up(o + tk * 4, 256);
+    r.pos = o;     o = align_up(o + tk * 4, 256);
+    r.active = o;  o = align_up(o + (size_t)E * 4, 256);
+    r.nact = o;    o = align_up(o + 4, 256);
+    return r;
+}
+
+template <typename T>
+T *ws_at(void *ws, size_t off) { return reinterpret_cast<T *>(reinterpret_cast<char *>(ws) + off); }
+
+// Prefill path (vq_prefill.cu).
+size_t prefill_workspace_size(const vq_moe_layer *L, int T, int k);
+vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const float *logits, int k, int renorm,
+                      void *y, int y_dtype, void *ws, size_t ws_bytes, cudaStream_t s);
+
+}  // namespace vq

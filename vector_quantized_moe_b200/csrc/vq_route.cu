@@ -1,0 +1,293 @@
+// Top-k router and expert bucketing for the VQ-MoE layer (sm_100a).
+//
+// Routing follows the MoE layers of the VQ model cards (Qwen3.8-Flash-Next:
+// 10-of-512 experts; gemma-4-26b-a4b: 128 experts, top-8). Order of the
+// top-k: larger logit first, ties to the smaller expert index, NaN last.
+// Weights: softmax of the selected logits (renorm) or the full softmax over
+// all experts evaluated at the selected ones.
+//
+// Bucketing: counts per expert, exclusive prefix sums (offsets), and a stable
+// permutation of the pairs p = t*k + j grouped by expert (increasing p inside
+// a bucket), its inverse (pos), and the ascending list of experts with
+// tokens. Every step is integer work or a fixed-order reduction, so the
+// tables are bit-identical from run to run.
+#include "vq_device.cuh"
+#include "vq_internal.h"
+
+namespace vq {
+namespace {
+
+constexpr int ROUTE_THREADS = 1024;
+constexpr int BUCKET_MAX_E_PARALLEL = 1024;   // per-warp histograms fit shared memory up to here
+
+// Monotone map of a float to uint32: NaN -> 0 (lowest), -0 -> +0.
+__device__ __forceinline__ uint32_t order_key(float v)
+{
+    if (v != v)
+        return 0u;
+    uint32_t u = __float_as_uint(v);
+    if (u == 0x80000000u)
+        u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// 64-bit key: value first, then the smaller index wins. Always >= 1.
+__device__ __forceinline__ uint64_t expert_key(float v, int e)
+{
+    return ((uint64_t)order_key(v) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)e);
+}
+
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o; o >>= 1)
+        v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+
+// One warp routes one token. Lane j < k ends with the j-th selection.
+template <int PER_LANE>
+__device__ __forceinline__ void route_token(const float *__restrict__ l, int E, int k, int renorm, int lane,
+                                            int32_t *ids, float *w)
+{
+    uint64_t keys[PER_LANE > 0 ? PER_LANE : 1];
+    if constexpr (PER_LANE > 0) {
+#pragma unroll
+        for (int i = 0; i < PER_LANE; ++i) {
+            const int e = lane + 32 * i;
+            keys[i] = e < E ? expert_key(l[e], e) : 0ull;
+        }
+    }
+    uint64_t prev = ~0ull;
+    int my_id = 0;
+    float my_l = 0.f;
+    for (int j = 0; j < k; ++j) {
+        uint64_t best = 0ull;
+        if constexpr (PER_LANE > 0) {
+#pragma unroll
+            for (int i = 0; i < PER_LANE; ++i)
+                if (keys[i] < prev && keys[i] > best)
+                    best = keys[i];
+        } else {
+            for (int e = lane; e < E; e += 32) {
+                const uint64_t key = expert_key(l[e], e);
+                if (key < prev && key > best)
+                    best = key;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            const uint64_t other = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+            best = other > best ? other : best;
+        }
+        prev = best;
+        if (lane == j) {
+            my_id = (int)(0xFFFFFFFFu - (uint32_t)best);
+            my_l = l[my_id];
+        }
+    }
+    const float top = __shfl_sync(0xFFFFFFFFu, my_l, 0);
+    const float num = lane < k ? expf(my_l - top) : 0.f;
+    float den;
+    if (renorm) {
+        den = warp_sum(num);
+    } else {
+        float s = 0.f;
+        for (int e = lane; e < E; e += 32)
+            s += expf(l[e] - top);
+        den = warp_sum(s);
+    }
+    if (lane < k) {
+        ids[lane] = my_id;
+        w[lane] = num / den;
+    }
+}
+
+template <int PER_LANE>
+__device__ void route_tokens(const float *logits, int t_begin, int t_end, int E, int k, int renorm, int32_t *ids,
+                             float *w)
+{
+    const int lane = threadIdx.x & 31;
+    const int nw = blockDim.x >> 5;
+    for (int t = t_begin + (threadIdx.x >> 5); t < t_end; t += nw)
+        route_token<PER_LANE>(logits + (long)t * E, E, k, renorm, lane, ids + (long)t * k, w + (long)t * k);
+}
+
+__device__ void route_range(const float *logits, int t_begin, int t_end, int E, int k, int renorm, int32_t *ids,
+                            float *w)
+{
+    if (E <= 128)
+        route_tokens<4>(logits, t_begin, t_end, E, k, renorm, ids, w);
+    else if (E <= 512)
+        route_tokens<16>(logits, t_begin, t_end, E, k, renorm, ids, w);
+    else
+        route_tokens<0>(logits, t_begin, t_end, E, k, renorm, ids, w);
+}
+
+// Bucketing by one CTA (pos, active and n_active may be NULL). Warp c of `chunks` handles pairs [c*P, (c+1)*P) with
+// its own histogram row, so the stable scatter runs in parallel.
+// Shared memory: hist [chunks][E] int32.
+__device__ void bucket(const int32_t *ids, int npairs, int E, int32_t *offsets, int32_t *perm, int32_t *pos,
+                       int32_t *active, int32_t *n_active, int32_t *hist, int chunks)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < chunks * E; i += blockDim.x)
+        hist[i] = 0;
+    __syncthreads();
+    const int per = (npairs + chunks - 1) / chunks;
+    if (warp < chunks) {
+        const int p0 = warp * per, p1 = min(npairs, p0 + per);
+        for (int p = p0 + lane; p < p1; p += 32)
+            atomicAdd(&hist[warp * E + ids[p]], 1);
+    }
+    __syncthreads();
+    // per expert: totals and per-chunk exclusive bases (relative to the bucket)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = 0;
+        for (int c = 0; c < chunks; ++c) {
+            const int v = hist[c * E + e];
+            hist[c * E + e] = run;
+            run += v;
+        }
+        offsets[e] = run;   // count for now
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int run = 0, act = 0;
+        const unsigned lt = (1u << lane) - 1u;
+        for (int base = 0; base < E; base += 32) {
+            const int e = base + lane;
+            const int c = e < E ? offsets[e] : 0;
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o)
+                    incl += v;
+            }
+            if (e < E)
+                offsets[e] = run + incl - c;
+            const unsigned ball = __ballot_sync(0xFFFFFFFFu, c > 0);
+            if (c > 0 && active)
+                active[act + __popc(ball & lt)] = e;
+            act += __popc(ball);
+            run += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
+        if (lane == 0) {
+            offsets[E] = run;
+            if (n_active)
+                *n_active = act;
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < chunks * E; i += blockDim.x)
+        hist[i] += offsets[i % E];
+    __syncthreads();
+    if (warp < chunks) {
+        int32_t *cur = hist + warp * E;
+        const int p0 = warp * per, p1 = min(npairs, p0 + per);
+        const unsigned lt = (1u << lane) - 1u;
+        for (int base = p0; base < p1; base += 32) {
+            const int p = base + lane;
+            const bool v = p < p1;
+            const int e = v ? ids[p] : -1;
+            const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+            if (v) {
+                const int slot = cur[e] + __popc(peers & lt);
+                perm[slot] = p;
+                if (pos)
+                    pos[p] = slot;
+            }
+            __syncwarp();
+            if (v && (31 - __clz(peers)) == lane)
+                cur[e] += __popc(peers);
+            __syncwarp();
+        }
+    }
+}
+
+__device__ __forceinline__ int bucket_chunks(int E)
+{
+    return E <= BUCKET_MAX_E_PARALLEL ? ROUTE_THREADS / 32 : 1;
+}
+
+// Small T: one CTA routes every token and buckets the pairs.
+__global__ void __launch_bounds__(ROUTE_THREADS) vq_route_fused_kernel(const float *logits, int T, int E, int k,
+                                                                      int renorm, int32_t *ids, float *w,
+                                                                      int32_t *offsets, int32_t *perm, int32_t *pos,
+                                                                      int32_t *active, int32_t *n_active)
+{
+    extern __shared__ int32_t hist[];
+    grid_dep_wait();
+    route_range(logits, 0, T, E, k, renorm, ids, w);
+    __syncthreads();
+    bucket(ids, T * k, E, offsets, perm, pos, active, n_active, hist, bucket_chunks(E));
+}
+
+// Large T: many CTAs route, then one CTA buckets.
+constexpr int ROUTE_TOKENS_PER_CTA = 256;
+
+__global__ void __launch_bounds__(ROUTE_THREADS) vq_route_topk_kernel(const float *logits, int T, int E, int k,
+                                                                     int renorm, int32_t *ids, float *w)
+{
+    grid_dep_wait();
+    const int t0 = blockIdx.x * ROUTE_TOKENS_PER_CTA;
+    route_range(logits, t0, min(T, t0 + ROUTE_TOKENS_PER_CTA), E, k, renorm, ids, w);
+}
+
+__global__ void __launch_bounds__(ROUTE_THREADS) vq_bucket_kernel(const int32_t *ids, int npairs, int E,
+                                                                 int32_t *offsets, int32_t *perm, int32_t *pos,
+                                                                 int32_t *active, int32_t *n_active)
+{
+    extern __shared__ int32_t hist[];
+    grid_dep_wait();
+    bucket(ids, npairs, E, offsets, perm, pos, active, n_active, hist, bucket_chunks(E));
+}
+
+template <typename K, typename... Args>
+cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+}  // namespace
+
+cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int32_t *ids, float *w,
+                         int32_t *offsets, int32_t *perm, int32_t *pos, int32_t *active, int32_t *n_active,
+                         cudaStream_t s, bool pdl)
+{
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t err = cudaFuncSetAttribute(vq_route_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               227 * 1024);
+        if (err == cudaSuccess)
+            err = cudaFuncSetAttribute(vq_bucket_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (err != cudaSuccess)
+            return err;
+        attr_set = true;
+    }
+    const int chunks = E <= BUCKET_MAX_E_PARALLEL ? ROUTE_THREADS / 32 : 1;
+    const size_t smem = (size_t)chunks * E * sizeof(int32_t);
+    if (T <= ROUTE_TOKENS_PER_CTA)
+        return launch_ex(vq_route_fused_kernel, dim3(1), dim3(ROUTE_THREADS), smem, s, pdl, logits, T, E, k, renorm,
+                         ids, w, offsets, perm, pos, active, n_active);
+    const int ctas = (T + ROUTE_TOKENS_PER_CTA - 1) / ROUTE_TOKENS_PER_CTA;
+    cudaError_t err = launch_ex(vq_route_topk_kernel, dim3(ctas), dim3(ROUTE_THREADS), 0, s, pdl, logits, T, E, k,
+                                renorm, ids, w);
+    if (err != cudaSuccess)
+        return err;
+    return launch_ex(vq_bucket_kernel, dim3(1), dim3(ROUTE_THREADS), smem, s, pdl, (const int32_t *)ids, T * k, E,
+                     offsets, perm, pos, active, n_active);
+}
+
+}  // namespace vq
