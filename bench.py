@@ -1,0 +1,393 @@
+"""Benchmark of the VQ-MoE hot path on B200 (one JSON line on rank 0).
+
+Default workload: the MoE decode layer with d=2/K=256 experts (512 experts,
+top-10, hidden 4096, inter 1024, 8 tokens per step). A step is one
+vq_moe_decode call: routing, bucketing, the gate/up grouped VQ GEMV, SwiGLU,
+the down grouped VQ GEMV and the weighted combine, over one batch of seeded
+synthetic inputs rotated among 16 routing draws (3.4 GB of expert weights, far
+beyond L2, so a step's experts are not L2-resident from the previous step).
+
+metric: decode HBM GB/s = algorithmic bytes of a step (live codes and group
+scales of the experts the step touches, codebooks, activations, logits and
+outputs) / step time. The roofline object reports the gate/up grouped GEMV
+(the dominant kernel) against the measured HBM copy bandwidth.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: the path does not shard (one GPU per layer); N ranks run N
+independent replicas and value sums their bytes over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import workloads as wl  # noqa: E402
+
+METRIC = "VQ expert decode HBM GB/s"
+UNIT = "GB/s"
+N_DRAWS = 16
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _module_bytes(md):
+    """Bytes of one expert's live codes + scales, per expert, for a module."""
+    import vector_quantized_moe_b200 as vq
+    rw = vq.packed_words(1, md.cols // md.d, md.bits)
+    per_row = rw * 4 + (md.cols // 64) * 2
+    if md.bitmap is None:
+        live = np.full(md.E, md.rows)
+    else:
+        live = np.array([sum(bin(int(w)).count("1") for w in md.bitmap[e]) for e in range(md.E)])
+    return live * per_row
+
+
+def _kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("vq_decode.cu", "vq_device.cuh"):
+        with open(os.path.join(ROOT, "vector_quantized_moe_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic_per_launch(kernel_tag):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary,
+    or None when the summary is missing or the kernel source changed since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f).get(kernel_tag)
+        if t and t.get("source_hash") == _kernel_source_hash():
+            return float(t["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while a window of GPU work runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def run_reference(args):
+    """The oracle (CPU, float64) on bounded samples of the same workload."""
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    spec = wl.DECODE_D2K256
+    T = spec.batches[1]
+    import vector_quantized_moe_b200 as vq
+    mds = wl.layer_modules(spec, raw=False, row_words=lambda c, g: vq.packed_words(1, c // g.d, g.bits))
+    from tests.helpers import oracle_module
+    oms = [oracle_module(m) for m in mds]
+    per_expert = sum(_module_bytes(m) for m in mds)
+    cb_bytes = sum(m.codebook.nbytes for m in mds)
+    draws = [wl.layer_inputs(spec, T, i) for i in range(N_DRAWS)]
+    total_b, total_t = 0.0, 0.0
+    for step in range(args.warmup + args.steps):
+        x, lg = draws[step % N_DRAWS]
+        tok = np.array([step % T])
+        ids, *_ = oracle.route(lg[tok], spec.top_k)
+        nbytes = float(per_expert[np.unique(ids)].sum() + cb_bytes + spec.hidden * 2 + spec.E * 4 + spec.hidden * 4)
+        t0 = time.perf_counter()
+        oracle.moe(*oms, x, lg, spec.top_k, tokens=tok)
+        dt = time.perf_counter() - t0
+        if step >= args.warmup:
+            total_b += nbytes
+            total_t += dt
+    value = total_b / total_t / 1e9
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_t / args.steps * 1e3,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": spec.name, "T": T, "sample": "1 token of the batch per step"},
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                            "sample": "one token per step (its 10 experts), float64 oracle"},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def run_ours(args):
+    import torch
+    import vector_quantized_moe_b200 as vq
+    from tests.helpers import lib_module
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    spec = wl.DECODE_D2K256
+    if args.small:
+        # same per-expert shapes with 64 experts (430 MB of weights): the case for full ncu captures
+        import dataclasses
+        spec = dataclasses.replace(spec, E=64, name=spec.name.replace("e512", "e64"))
+    T = spec.batches[1]
+    k = spec.top_k
+    mds = wl.layer_modules(spec, raw=False, row_words=lambda c, g: vq.packed_words(1, c // g.d, g.bits))
+    mods = [lib_module(m, device=dev) for m in mds]
+    layer = vq.MoELayer(*mods)
+    per_expert = [_module_bytes(m) for m in mds]
+    cb_bytes = sum(m.codebook.nbytes for m in mds)
+
+    draws = [wl.layer_inputs(spec, T, i) for i in range(N_DRAWS)]
+    xs = [torch.from_numpy(x.view(np.int16)).to(dev) for x, _ in draws]
+    lgs = [torch.from_numpy(lg).to(dev) for _, lg in draws]
+    y = torch.empty((T, spec.hidden), dtype=torch.float32, device=dev)
+    wsp = layer.workspace(T, k, vq.VQ_MODE_DECODE, dev)
+
+    # algorithmic bytes of each draw from its routing (untimed)
+    step_bytes, gu_bytes = [], []
+    io = T * spec.hidden * 2 + T * spec.E * 4 + T * spec.hidden * 4
+    for lg in lgs:
+        _, _, off, _ = vq.route(lg, k)
+        touched = np.nonzero(np.diff(off.cpu().numpy()) > 0)[0]
+        g, u, d = (float(p[touched].sum()) for p in per_expert)
+        step_bytes.append(g + u + d + cb_bytes + io)
+        gu_bytes.append(g + u + mds[0].codebook.nbytes + mds[1].codebook.nbytes + T * spec.hidden * 2)
+
+    def step(i):
+        layer.decode(xs[i % N_DRAWS], lgs[i % N_DRAWS], k, out=y, workspace=wsp)
+
+    def barrier():
+        if ws > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(v):
+        if ws == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum_over_ranks(v):
+        if ws == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t)
+        return float(t.item())
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    if args.ncu:
+        # minimal launch sequence for profiler captures: 16 route calls above,
+        # warmup * 5 launches, then steps * 5 launches
+        for i in range(args.steps):
+            step(i)
+        torch.cuda.synchronize()
+        return
+
+    # main timed region, with clocks sampled over a window that contains it
+    clk = ClockSampler(local)
+    clk.start()
+    t_end = time.perf_counter() + 1.0
+    i = 0
+    while time.perf_counter() < t_end:       # pre-roll so the sampler sees the loaded clock
+        for _ in range(50):
+            step(i)
+            i += 1
+        torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = clk.stop()
+    ms_total = max_over_ranks(e0.elapsed_time(e1))
+    ms_step = ms_total / args.steps
+    my_bytes = sum(step_bytes[i % N_DRAWS] for i in range(args.steps))
+    value = sum_over_ranks(my_bytes) / (ms_total * 1e-3) / 1e9
+
+    # trace pass: per-stage durations from events recorded at stage boundaries
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        vq.set_trace_events(evs[i])
+        step(i)
+    vq.set_trace_events(None)
+    torch.cuda.synchronize()
+    stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(5)] for i in range(args.steps)])
+    stage_ms = stage.mean(axis=0)
+    gu_ms = float(stage_ms[1])
+    gu_avg_bytes = float(np.mean([gu_bytes[i % N_DRAWS] for i in range(args.steps)]))
+    hbm, tf_burst, tf_sust, src = _peaks()
+    achieved = gu_avg_bytes / (gu_ms * 1e-3) / 1e9
+
+    # end-to-end: host buffers in pinned memory, copies inside the timed region
+    hx = [torch.from_numpy(x.view(np.int16)).pin_memory() for x, _ in draws]
+    hl = [torch.from_numpy(lg).pin_memory() for _, lg in draws]
+    hy = torch.empty((T, spec.hidden), dtype=torch.float32).pin_memory()
+    dx = torch.empty_like(xs[0])
+    dl = torch.empty_like(lgs[0])
+    torch.cuda.synchronize()
+    barrier()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for i in range(args.steps):
+        dx.copy_(hx[i % N_DRAWS], non_blocking=True)
+        dl.copy_(hl[i % N_DRAWS], non_blocking=True)
+        layer.decode(dx, dl, k, out=y, workspace=wsp)
+        hy.copy_(y, non_blocking=True)
+    f1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1))
+    e2e_value = sum_over_ranks(my_bytes) / (e2e_ms * 1e-3) / 1e9
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(mds, draws, spec, T, per_expert, cb_bytes)
+
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16xf16->f32", "data": "synthetic",
+        "config": {"workload": spec.name, "T": T, "top_k": k, "E": spec.E, "hidden": spec.hidden,
+                   "inter": spec.inter, "geometry": "d2K256 (8-bit codes) x3",
+                   "l2": f"inputs larger than L2: {N_DRAWS} rotating routing draws over "
+                         f"{sum(float(p.sum()) for p in per_expert) / 1e9:.2f} GB of expert weights",
+                   "parallelism": "replicas" if ws > 1 else "single-gpu",
+                   "tokens_per_s": T * args.steps * ws / (ms_total * 1e-3)},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": _traffic_per_launch("grouped_gemv_gate_up"),
+                     "kernel": "vq_grouped_gemv_kernel<2,8> (gate+up)", "peak_source": f"{src} hbm_gbs",
+                     "bytes_per_launch": gu_avg_bytes, "ms_per_launch": gu_ms},
+        "stage_ms": {"route": float(stage_ms[0]), "gate_up_gemv": gu_ms, "swiglu": float(stage_ms[2]),
+                     "down_gemv": float(stage_ms[3]), "combine": float(stage_ms[4])},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(xs[0].numel() * 2 + lgs[0].numel() * 4),
+                "d2h_bytes_per_step": int(y.numel() * 4)},
+        "gpu_launches": 5 * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+def cpu_baseline(mds, draws, spec, T, per_expert, cb_bytes, budget_s=10.0):
+    """The oracle as it stands on a bounded sample: tokens of the first draw
+    until about budget_s seconds of CPU work."""
+    import oracle
+    from tests.helpers import oracle_module
+    oracle.build()
+    oms = [oracle_module(m) for m in mds]
+    x, lg = draws[0]
+    done, nbytes, t_used = 0, 0.0, 0.0
+    while done < T and t_used < budget_s:
+        tok = np.array([done])
+        ids, *_ = oracle.route(lg[tok], spec.top_k)
+        t0 = time.perf_counter()
+        oracle.moe(*oms, x, lg, spec.top_k, tokens=tok)
+        t_used += time.perf_counter() - t0
+        nbytes += float(sum(p[np.unique(ids)].sum() for p in per_expert) + cb_bytes + spec.hidden * 10 + spec.E * 4)
+        done += 1
+    return {"value": nbytes / t_used / 1e9, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{done} token(s) of the 8-token batch ({done * spec.top_k} expert passes), float64",
+            "seconds": t_used}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ncu", action="store_true", help="only warmup + timed steps, for profiler captures")
+    ap.add_argument("--small", action="store_true", help="64-expert variant of the workload (profiling)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

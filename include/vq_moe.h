@@ -193,6 +193,17 @@ vq_status vq_moe_prefill(const vq_moe_layer *L, const uint16_t *x, int32_t T, co
                          int32_t top_k, int32_t renorm, void *y, int32_t y_dtype, void *workspace,
                          size_t ws_bytes, void *stream);
 
+/* Tracing (no counterpart on the pages; an observability hook for timing
+ * each kernel stage with the caller's CUDA events). events: host array of
+ * n_events cudaEvent_t handles (as void*) created by the caller, or NULL to
+ * switch tracing off. While set, the calling thread's vq_moe_decode and
+ * vq_moe_prefill record events[i] on their stream at stage boundary i:
+ *   decode:  0 | route | 1 | gate/up GEMV | 2 | SwiGLU | 3 | down GEMV | 4 | combine | 5
+ *   prefill: 0 | route | 1 | gather | 2 | gate/up GEMM | 3 | down GEMM | 4 | combine | 5
+ * Boundaries beyond n_events are not recorded. The library does not own
+ * the events. Errors: VQ_ERR_ARG when n_events < 0. */
+vq_status vq_set_trace_events(void *const *events, int32_t n_events);
+
 #ifdef __cplusplus
 }
 #endif

@@ -5,12 +5,11 @@ from __future__ import annotations
 
 import numpy as np
 
-import oracle
-import synth
 from synth.workloads import Geometry, ModuleData, module_data
 
 
-def oracle_module(md: ModuleData) -> "oracle.Module":
+def oracle_module(md: ModuleData):
+    import oracle   # imported here so that the library-side helpers never load the oracle
     if md.codes is not None:
         words = oracle.pack(md.codes, md.bits, md.bitmap)
         sc = oracle.compact_rows(md.scales, md.bitmap)

@@ -63,6 +63,7 @@ def _load():
         "vq_moe_workspace_size": (SZ, [LP, I32, I32, I32]),
         "vq_moe_decode": (ctypes.c_int, [LP, P, I32, P, I32, I32, P, I32, P, SZ, P]),
         "vq_moe_prefill": (ctypes.c_int, [LP, P, I32, P, I32, I32, P, I32, P, SZ, P]),
+        "vq_set_trace_events": (ctypes.c_int, [P, I32]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -234,6 +235,25 @@ def route(logits, top_k: int, renorm: bool = True, stream=None):
     _check(_L().vq_route(logits.data_ptr(), T, E, top_k, int(bool(renorm)), ids.data_ptr(), w.data_ptr(),
                          offsets.data_ptr(), perm.data_ptr(), _stream(stream)), "vq_route")
     return ids, w, offsets, perm
+
+
+def set_trace_events(events) -> None:
+    """Record the given torch.cuda.Event objects at the stage boundaries of the
+    next MoE calls on this thread (vq_set_trace_events); None switches it off."""
+    global _trace_keep
+    if events is None:
+        _trace_keep = None
+        _check(_L().vq_set_trace_events(None, 0), "vq_set_trace_events")
+        return
+    for e in events:
+        if e.cuda_event == 0:
+            e.record()
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    _trace_keep = arr
+    _check(_L().vq_set_trace_events(arr, len(events)), "vq_set_trace_events")
+
+
+_trace_keep = None
 
 
 class MoELayer:

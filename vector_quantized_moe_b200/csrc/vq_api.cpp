@@ -74,7 +74,7 @@ struct DecodePlan {
     int T, k, E, H, I;
     int sa, sb;                  // slices of the gate/up and down passes
     RoutingLayout r;
-    size_t off_G, off_U, off_h, off_D;
+    size_t off_x16, off_G, off_U, off_h, off_D;
     size_t total;
 };
 
@@ -109,6 +109,7 @@ DecodePlan plan_decode(const vq_moe_layer *L, int T, int k)
     size_t o = 0;
     p.r = plan_routing(o, T, k, p.E);
     const size_t tk = (size_t)T * k;
+    p.off_x16 = o; o = align_up(o + (size_t)T * p.H * 2, 256);
     p.off_G = o; o = align_up(o + (size_t)p.sa * tk * p.I * 4, 256);
     p.off_U = o; o = align_up(o + (size_t)p.sa * tk * p.I * 4, 256);
     p.off_h = o; o = align_up(o + tk * p.I * 2, 256);
@@ -147,6 +148,17 @@ ModDev make_moddev(const vq_module &m)
     return d;
 }
 
+namespace {
+thread_local cudaEvent_t *g_trace = nullptr;
+thread_local int g_trace_n = 0;
+}  // namespace
+
+void trace_point(int i, cudaStream_t s)
+{
+    if (g_trace && i < g_trace_n)
+        cudaEventRecord(g_trace[i], s);
+}
+
 }  // namespace vq
 
 using namespace vq;
@@ -168,6 +180,15 @@ const char *vq_status_str(vq_status s)
 }
 
 int vq_geometry_supported(int32_t d, int32_t bits) { return geometry_ok(d, bits) ? 1 : 0; }
+
+vq_status vq_set_trace_events(void *const *events, int32_t n_events)
+{
+    if (n_events < 0)
+        return VQ_ERR_ARG;
+    g_trace = events ? (cudaEvent_t *)events : nullptr;
+    g_trace_n = events ? n_events : 0;
+    return VQ_OK;
+}
 
 size_t vq_packed_words(int64_t rows, int32_t ncode, int32_t bits)
 {
@@ -305,6 +326,7 @@ vq_status vq_gemv(const vq_module *m, int32_t expert, const uint16_t *x, int32_t
     a.nmod = 1;
     a.act = x;
     a.act_bf16 = 1;
+    a.act_by_slot = 0;
     a.expert = expert;
     a.T = T;
     a.slices = 1;
@@ -325,7 +347,7 @@ vq_status vq_route(const float *logits, int32_t T, int32_t E, int32_t top_k, int
         top_k > std::min(E, 32) || (long)T * top_k >= (1L << 31))
         return VQ_ERR_ARG;
     return cuda_status(launch_route(logits, T, E, top_k, renorm, ids, weights, offsets, perm, nullptr, nullptr,
-                                    nullptr, (cudaStream_t)stream, false));
+                                    nullptr, nullptr, nullptr, 0, (cudaStream_t)stream, false));
 }
 
 size_t vq_moe_workspace_size(const vq_moe_layer *L, int32_t T, int32_t top_k, int32_t mode)
@@ -374,20 +396,25 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     int32_t *pos = ws_at<int32_t>(workspace, p.r.pos);
     int32_t *active = ws_at<int32_t>(workspace, p.r.active);
     int32_t *nact = ws_at<int32_t>(workspace, p.r.nact);
+    __half *x16 = ws_at<__half>(workspace, p.off_x16);
     float *G = ws_at<float>(workspace, p.off_G);
     float *U = ws_at<float>(workspace, p.off_U);
     __half *h = ws_at<__half>(workspace, p.off_h);
     float *D = ws_at<float>(workspace, p.off_D);
     const long tk = (long)T * top_k;
 
-    cudaError_t err = launch_route(logits, T, p.E, top_k, renorm, ids, w, offsets, perm, pos, active, nact, s, true);
+    trace_point(0, s);
+    cudaError_t err = launch_route(logits, T, p.E, top_k, renorm, ids, w, offsets, perm, pos, active, nact, x, x16,
+                                   p.H, s, true);
     if (err != cudaSuccess)
         return VQ_ERR_CUDA;
+    trace_point(1, s);
 
     // gate and up: one launch when they share a geometry
     GemvArgs a{};
-    a.act = x;
-    a.act_bf16 = 1;
+    a.act = x16;
+    a.act_bf16 = 0;
+    a.act_by_slot = 0;
     a.offsets = offsets;
     a.perm = perm;
     a.top_k = top_k;
@@ -406,7 +433,8 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
         a.out[0] = G;
         a.out[1] = U;
         const int occ = gemv_ctas_per_sm(mg.d, mg.bits, gemv_smem_bytes(mg));
-        err = launch_gemv(a, std::max(1, sms * occ / 2), s, true);
+        const int per_y = gemv_both_modules_per_cta(mg.d, mg.bits) ? sms * occ : std::max(1, sms * occ / 2);
+        err = launch_gemv(a, per_y, s, true);
     } else {
         a.nmod = 1;
         a.mod[0] = a.mod[1] = mg;
@@ -421,9 +449,11 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     if (err != cudaSuccess)
         return VQ_ERR_CUDA;
 
+    trace_point(2, s);
     err = launch_swiglu(G, U, p.sa, tk * p.I, (int)tk, p.I, h, s, true);
     if (err != cudaSuccess)
         return VQ_ERR_CUDA;
+    trace_point(3, s);
 
     GemvArgs b = a;
     const ModDev md = make_moddev(L->down);
@@ -431,6 +461,7 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     b.nmod = 1;
     b.act = h;
     b.act_bf16 = 0;
+    b.act_by_slot = 1;
     b.slices = p.sb;
     b.out[0] = b.out[1] = D;
     b.out_slice_stride = tk * p.H;
@@ -438,7 +469,9 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     if (err != cudaSuccess)
         return VQ_ERR_CUDA;
 
+    trace_point(4, s);
     err = launch_combine(D, p.sb, tk * p.H, w, pos, T, top_k, p.H, y, y_dtype, s, true);
+    trace_point(5, s);
     return cuda_status(err);
 }
 

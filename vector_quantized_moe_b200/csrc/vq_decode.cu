@@ -140,54 +140,92 @@ __device__ __forceinline__ void store_out(void *out, int dtype, long idx, float 
 }
 
 constexpr int GEMV_THREADS = 256;
+constexpr int GEMV_PD = 3;   // groups of loads in flight per warp
+
+// d=2 with 8-bit codes: each codebook entry owns a 256-byte line holding 32
+// per-lane replicas of module 0 (bytes 0..127) and of module 1 (128..255).
+// A code byte then turns into its lane's smem address with one byte permute:
+// offset = code * 256 + module * 128 + lane * 4, and a warp's 32 lookups hit
+// 32 distinct banks.
+template <int D, int BITS>
+struct FastByteCodes {
+    static constexpr bool value = (D == 2 && BITS == 8);
+};
 
 template <int D, int BITS>
-__global__ void __launch_bounds__(GEMV_THREADS, 1) vq_grouped_gemv_kernel(const __grid_constant__ GemvArgs a)
+__device__ __forceinline__ void fill_codebook_lines(uint32_t *cbs, const uint16_t *cb0, const uint16_t *cb1, int nmod)
+{
+    const int n = 256 * 64;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int c = i >> 6, m = (i >> 5) & 1;
+        const uint16_t *cb = m ? cb1 : cb0;
+        cbs[i] = (m < nmod) ? reinterpret_cast<const uint32_t *>(cb)[c] : 0u;
+    }
+}
+
+// Loads of one 64-column group for one lane: the code words of its four rows
+// and their fp16 scales (the activations, L1-resident, are read when used).
+template <int D, int BITS>
+struct GroupLoads {
+    uint32_t cw[4][Geo<D, BITS>::LW];
+    int co[4];
+    uint16_t sv[4];
+};
+
+template <int D, int BITS, int PD>
+__global__ void __launch_bounds__(GEMV_THREADS, 2) vq_grouped_gemv_kernel(const __grid_constant__ GemvArgs a)
 {
     using G = Geo<D, BITS>;
+    constexpr bool FAST = FastByteCodes<D, BITS>::value;
     extern __shared__ __align__(16) uint32_t cbs[];
-    const ModDev m = blockIdx.y == 0 ? a.mod[0] : a.mod[1];
-    void *const out = blockIdx.y == 0 ? a.out[0] : a.out[1];
 
-    fill_codebook<D, BITS>(cbs, m.codebook, m.log_rep);
+    // modules per CTA: the fast layout holds both codebooks; otherwise blockIdx.y picks one
+    const int cta_mods = FAST ? a.nmod : 1;
+    if constexpr (FAST)
+        fill_codebook_lines<D, BITS>(cbs, a.mod[0].codebook, a.mod[1].codebook, a.nmod);
+    else
+        fill_codebook<D, BITS>(cbs, (blockIdx.y == 0 ? a.mod[0] : a.mod[1]).codebook,
+                               (blockIdx.y == 0 ? a.mod[0] : a.mod[1]).log_rep);
     __syncthreads();
     grid_dep_wait();
 
     const int lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int rep = lane & (m.rep - 1);
     const int wpc = blockDim.x >> 5;
     const long gwarp = (long)blockIdx.x * wpc + (threadIdx.x >> 5);
     const long nwarps = (long)gridDim.x * wpc;
 
     const int n_act = a.offsets ? *a.n_active : 1;
-    const int nblk = (m.rows + 31) >> 5;
+    const ModDev m0 = FAST ? a.mod[0] : (blockIdx.y == 0 ? a.mod[0] : a.mod[1]);
+    const int nblk = (m0.rows + 31) >> 5;
     const int S = a.slices;
-    const int gps = m.ngroups / S;
-    const long n_items = (long)n_act * nblk * S;
+    const int gps = m0.ngroups / S;
+    const long n_items = (long)n_act * nblk * S * cta_mods;
 
     for (long it = gwarp; it < n_items; it += nwarps) {
-        const int slice = (int)(it % S);
-        const long rest = it / S;
+        long rest = it;
+        const int slice = (int)(rest % S);
+        rest /= S;
         const int blk = (int)(rest % nblk);
-        const int ai = (int)(rest / nblk);
+        rest /= nblk;
+        const int mi = FAST ? (int)(rest % cta_mods) : (int)blockIdx.y;
+        const int ai = FAST ? (int)(rest / cta_mods) : (int)rest;
+        const ModDev &m = (mi == 0) ? a.mod[0] : a.mod[1];
+        void *const out = (mi == 0) ? a.out[0] : a.out[1];
+        const int rep = lane & (m.rep - 1);
+        const uint32_t lane_sel = (uint32_t)(mi * 128 + lane * 4);
+
         const int e = a.offsets ? a.active[ai] : a.expert;
         const int q0 = a.offsets ? a.offsets[e] : 0;
         const int n = a.offsets ? a.offsets[e + 1] - q0 : a.T;
 
-        // rows of this lane: i = 0,1 -> tile 0 rows g, g+8; i = 2,3 -> tile 1
-        const uint32_t *rowp[4];
-        const uint16_t *scp[4];
-        bool live[4];
+        // rows of this lane: i = 0,1 -> tile 0 rows g, g+8; i = 2,3 -> tile 1.
+        // prow[i] = packed-row index, -1 for a dead row or a row past the end.
+        int prow[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int r = blk * 32 + 8 * i + g;
-            long pr = -1;
-            if (r < m.rows)
-                pr = live_row(m.bitmap, m.rank, m.bm_words, m.rows, e, r);
-            live[i] = pr >= 0;
-            rowp[i] = m.codes + (live[i] ? pr : 0) * (long)m.row_words;
-            scp[i] = m.scales + (live[i] ? pr : 0) * (long)m.ngroups;
+            prow[i] = r < m.rows ? (int)live_row(m.bitmap, m.rank, m.bm_words, m.rows, e, r) : -1;
         }
         const int gbeg = slice * gps, gend = gbeg + gps;
 
@@ -196,12 +234,8 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1) vq_grouped_gemv_kernel(const 
             const uint16_t *arow = nullptr;
             if (has_tok) {
                 const int q = q0 + tok0 + g;
-                long arow_idx;
-                if (a.act_bf16)
-                    arow_idx = a.perm ? (long)(a.perm[q] / a.top_k) : (long)(tok0 + g);
-                else
-                    arow_idx = q;
-                arow = reinterpret_cast<const uint16_t *>(a.act) + arow_idx * (long)m.cols + 16 * t;
+                const long ar = a.act_by_slot ? (long)q : (a.perm ? (long)(a.perm[q] / a.top_k) : (long)(tok0 + g));
+                arow = reinterpret_cast<const uint16_t *>(a.act) + ar * (long)m.cols + 16 * t;
             }
             float acc[2][4];
 #pragma unroll
@@ -210,58 +244,70 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1) vq_grouped_gemv_kernel(const 
                 for (int j = 0; j < 4; ++j)
                     acc[i][j] = 0.f;
 
-            // one-group-deep software pipeline: loads of group G+1 are in flight
-            // while group G is decoded and multiplied
-            uint32_t cw[2][4][G::LW];
-            int co[2][4];
-            uint4 av[2][2];
-            uint16_t sv[2][4];
-            auto issue = [&](int buf, int grp) {
+            GroupLoads<D, BITS> st[PD];
+            auto issue = [&](GroupLoads<D, BITS> &L, int grp) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    load_quarter<D, BITS>(rowp[i], 4L * grp + t, live[i], cw[buf][i], co[buf][i]);
-                    sv[buf][i] = live[i] ? ldg_u16(scp[i] + grp) : (uint16_t)0;
-                }
-                if (has_tok) {
-                    av[buf][0] = ldg_u128(arow + (long)grp * 64);
-                    av[buf][1] = ldg_u128(arow + (long)grp * 64 + 8);
-                } else {
-                    av[buf][0] = make_uint4(0u, 0u, 0u, 0u);
-                    av[buf][1] = make_uint4(0u, 0u, 0u, 0u);
+                    const bool lv = prow[i] >= 0;
+                    load_quarter<D, BITS>(m.codes + (long)prow[i] * m.row_words, 4L * grp + t, lv, L.cw[i], L.co[i]);
+                    L.sv[i] = lv ? ldg_u16(m.scales + (long)prow[i] * m.ngroups + grp) : (uint16_t)0;
                 }
             };
-            auto compute = [&](int buf) {
-                uint32_t bw[8] = {av[buf][0].x, av[buf][0].y, av[buf][0].z, av[buf][0].w,
-                                  av[buf][1].x, av[buf][1].y, av[buf][1].z, av[buf][1].w};
+            auto compute = [&](const GroupLoads<D, BITS> &L, int grp) {
+                uint4 av0 = make_uint4(0u, 0u, 0u, 0u), av1 = av0;
+                if (has_tok) {
+                    av0 = ldg_u128(arow + (long)grp * 64);
+                    av1 = ldg_u128(arow + (long)grp * 64 + 8);
+                }
+                uint32_t bw[8] = {av0.x, av0.y, av0.z, av0.w, av1.x, av1.y, av1.z, av1.w};
                 if (a.act_bf16) {
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
                         bw[i] = bf16x2_to_f16x2(bw[i]);
                 }
-                uint32_t c[4][G::CODES];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    extract_codes<D, BITS>(cw[buf][i], co[buf][i], c[i]);
                 float tmp[2][4];
 #pragma unroll
                 for (int i = 0; i < 2; ++i)
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
                         tmp[i][j] = 0.f;
+                if constexpr (FAST) {
+                    const char *cbb = reinterpret_cast<const char *>(cbs);
 #pragma unroll
-                for (int s = 0; s < 4; ++s) {
+                    for (int s = 0; s < 4; ++s) {
 #pragma unroll
-                    for (int rt = 0; rt < 2; ++rt) {
-                        uint32_t A[4];
-                        a_words<D>(cbs, m.log_rep, rep, c[2 * rt], s, A[0], A[2]);
-                        a_words<D>(cbs, m.log_rep, rep, c[2 * rt + 1], s, A[1], A[3]);
-                        mma_16816(tmp[rt], A, bw[2 * s], bw[2 * s + 1]);
+                        for (int rt = 0; rt < 2; ++rt) {
+                            uint32_t A[4];
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const uint32_t sel = 0x5504u | ((uint32_t)(2 * (s & 1) + h) << 4);
+                                const uint32_t wlo = L.cw[2 * rt][s >> 1], whi = L.cw[2 * rt + 1][s >> 1];
+                                A[2 * h] = *reinterpret_cast<const uint32_t *>(cbb + __byte_perm(wlo, lane_sel, sel));
+                                A[2 * h + 1] = *reinterpret_cast<const uint32_t *>(cbb + __byte_perm(whi, lane_sel, sel));
+                            }
+                            mma_16816(tmp[rt], A, bw[2 * s], bw[2 * s + 1]);
+                        }
+                    }
+                } else {
+                    uint32_t c[4][G::CODES];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        extract_codes<D, BITS>(L.cw[i], L.co[i], c[i]);
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) {
+#pragma unroll
+                        for (int rt = 0; rt < 2; ++rt) {
+                            uint32_t A[4];
+                            a_words<D>(cbs, m.log_rep, rep, c[2 * rt], s, A[0], A[2]);
+                            a_words<D>(cbs, m.log_rep, rep, c[2 * rt + 1], s, A[1], A[3]);
+                            mma_16816(tmp[rt], A, bw[2 * s], bw[2 * s + 1]);
+                        }
                     }
                 }
 #pragma unroll
                 for (int rt = 0; rt < 2; ++rt) {
-                    const float slo = f16_to_f32(sv[buf][2 * rt]);
-                    const float shi = f16_to_f32(sv[buf][2 * rt + 1]);
+                    const float slo = f16_to_f32(L.sv[2 * rt]);
+                    const float shi = f16_to_f32(L.sv[2 * rt + 1]);
                     acc[rt][0] = fmaf(tmp[rt][0], slo, acc[rt][0]);
                     acc[rt][1] = fmaf(tmp[rt][1], slo, acc[rt][1]);
                     acc[rt][2] = fmaf(tmp[rt][2], shi, acc[rt][2]);
@@ -269,17 +315,21 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1) vq_grouped_gemv_kernel(const 
                 }
             };
 
-            issue(0, gbeg);
-            int grp = gbeg;
-            for (; grp + 1 < gend; grp += 2) {
-                issue(1, grp + 1);
-                compute(0);
-                if (grp + 2 < gend)
-                    issue(0, grp + 2);
-                compute(1);
+            // ring of PD groups: loads of the next PD-1 groups are in flight
+            // while one group is decoded and multiplied
+#pragma unroll
+            for (int s = 0; s < PD - 1; ++s)
+                if (gbeg + s < gend)
+                    issue(st[s], gbeg + s);
+            for (int grp = gbeg; grp < gend; grp += PD) {
+#pragma unroll
+                for (int s = 0; s < PD; ++s) {
+                    if (grp + s + PD - 1 < gend)
+                        issue(st[(s + PD - 1) % PD], grp + s + PD - 1);
+                    if (grp + s < gend)
+                        compute(st[s], grp + s);
+                }
             }
-            if (grp < gend)
-                compute(0);
 
             // lane holds rows (g, g+8) of each tile for bucket tokens tok0 + 2t + {0, 1}
 #pragma unroll
@@ -294,7 +344,7 @@ __global__ void __launch_bounds__(GEMV_THREADS, 1) vq_grouped_gemv_kernel(const 
                         const int tk = tok0 + 2 * t + cc;
                         if (tk >= n)
                             continue;
-                        const float v = live[2 * rt + hf] ? acc[rt][2 * hf + cc] : 0.f;
+                        const float v = prow[2 * rt + hf] >= 0 ? acc[rt][2 * hf + cc] : 0.f;
                         store_out(out, a.out_dtype, (long)slice * a.out_slice_stride + (long)(q0 + tk) * m.rows + r, v);
                     }
                 }
@@ -403,7 +453,7 @@ cudaError_t launch(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
 template <int D, int BITS>
 cudaError_t gemv_dispatch(const GemvArgs &a, int ctas, size_t smem, cudaStream_t s, bool pdl)
 {
-    auto k = vq_grouped_gemv_kernel<D, BITS>;
+    auto k = vq_grouped_gemv_kernel<D, BITS, GEMV_PD>;
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
@@ -411,13 +461,14 @@ cudaError_t gemv_dispatch(const GemvArgs &a, int ctas, size_t smem, cudaStream_t
             return err;
         attr_set = true;
     }
-    return launch(k, dim3(ctas, a.nmod), dim3(GEMV_THREADS), smem, s, pdl, a);
+    const int gy = FastByteCodes<D, BITS>::value ? 1 : a.nmod;
+    return launch(k, dim3(ctas, gy), dim3(GEMV_THREADS), smem, s, pdl, a);
 }
 
 template <int D, int BITS>
 int gemv_occupancy(size_t smem)
 {
-    auto k = vq_grouped_gemv_kernel<D, BITS>;
+    auto k = vq_grouped_gemv_kernel<D, BITS, GEMV_PD>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, GEMV_THREADS, smem) != cudaSuccess)
@@ -429,9 +480,13 @@ int gemv_occupancy(size_t smem)
 
 size_t gemv_smem_bytes(const ModDev &m)
 {
+    if (m.d == 2 && m.bits == 8)
+        return 256 * 256;   // 256-byte line per entry, both modules
     const int ew = m.d <= 2 ? 1 : m.d / 2;
     return ((size_t)1 << m.bits) * (size_t)m.rep * ew * 4;
 }
+
+bool gemv_both_modules_per_cta(int d, int bits) { return d == 2 && bits == 8; }
 
 int gemv_ctas_per_sm(int d, int bits, size_t smem)
 {

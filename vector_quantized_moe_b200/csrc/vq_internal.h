@@ -36,8 +36,9 @@ ModDev make_moddev(const vq_module &m);
 struct GemvArgs {
     ModDev mod[2];
     int nmod;
-    const void *act;        // activation rows: bf16 [T, cols] (act_bf16) or fp16 [slots, cols]
+    const void *act;        // activation rows: fp16 (or bf16 when act_bf16) [tokens or slots, cols]
     int act_bf16;
+    int act_by_slot;        // 1: activation row = bucket slot q; 0: token (perm[q] / top_k, or t)
     const int32_t *offsets; // [E + 1] bucket offsets; NULL -> single expert over T tokens
     const int32_t *perm;    // [T*k] pair ids in bucket order (bf16 act: token = perm[q] / top_k)
     int top_k;
@@ -53,12 +54,14 @@ struct GemvArgs {
 
 cudaError_t launch_gemv(const GemvArgs &a, int ctas_per_mod, cudaStream_t s, bool pdl);
 int gemv_ctas_per_sm(int d, int bits, size_t smem);
+bool gemv_both_modules_per_cta(int d, int bits);
 size_t gemv_smem_bytes(const ModDev &m);
 
-// Routing + bucketing in one CTA. pos = inverse of perm; active/n_active as above.
+// Routing + bucketing. pos = inverse of perm; active/n_active as above (may be NULL).
+// When x is not NULL the same launch also writes x16 = fp16(x) [T, H].
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int32_t *ids, float *w,
                          int32_t *offsets, int32_t *perm, int32_t *pos, int32_t *active, int32_t *n_active,
-                         cudaStream_t s, bool pdl);
+                         const uint16_t *x, __half *x16, int H, cudaStream_t s, bool pdl);
 
 // h[q, c] = fp16( silu(sum_s G[s, q, c]) * sum_s U[s, q, c] )
 cudaError_t launch_swiglu(const float *G, const float *U, int slices, long slice_stride, int slots, int inter,
@@ -95,6 +98,9 @@ inline RoutingLayout plan_routing(size_t &o, int T, int k, int E)
 
 template <typename T>
 T *ws_at(void *ws, size_t off) { return reinterpret_cast<T *>(reinterpret_cast<char *>(ws) + off); }
+
+// Stage-boundary tracing (vq_set_trace_events): records event i on stream s if set.
+void trace_point(int i, cudaStream_t s);
 
 // Prefill path (vq_prefill.cu).
 size_t prefill_workspace_size(const vq_moe_layer *L, int T, int k);

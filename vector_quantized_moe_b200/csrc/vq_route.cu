@@ -206,6 +206,19 @@ __device__ void bucket(const int32_t *ids, int npairs, int E, int32_t *offsets, 
     }
 }
 
+// x16[t, c] = fp16(x[t, c]) for the tokens [t0, t1) (the tensor-core kernels
+// read fp16 activations; bf16 -> fp16 is exact for magnitudes in [2^-14, 65504]).
+__device__ void convert_rows(const uint16_t *x, __half *x16, int t0, int t1, int H)
+{
+    if (!x)
+        return;
+    const long n = (long)(t1 - t0) * H / 2;
+    const uint32_t *src = reinterpret_cast<const uint32_t *>(x + (long)t0 * H);
+    uint32_t *dst = reinterpret_cast<uint32_t *>(x16 + (long)t0 * H);
+    for (long i = threadIdx.x; i < n; i += blockDim.x)
+        dst[i] = bf16x2_to_f16x2(src[i]);
+}
+
 __device__ __forceinline__ int bucket_chunks(int E)
 {
     return E <= BUCKET_MAX_E_PARALLEL ? ROUTE_THREADS / 32 : 1;
@@ -215,10 +228,12 @@ __device__ __forceinline__ int bucket_chunks(int E)
 __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_fused_kernel(const float *logits, int T, int E, int k,
                                                                       int renorm, int32_t *ids, float *w,
                                                                       int32_t *offsets, int32_t *perm, int32_t *pos,
-                                                                      int32_t *active, int32_t *n_active)
+                                                                      int32_t *active, int32_t *n_active,
+                                                                      const uint16_t *x, __half *x16, int H)
 {
     extern __shared__ int32_t hist[];
     grid_dep_wait();
+    convert_rows(x, x16, 0, T, H);
     route_range(logits, 0, T, E, k, renorm, ids, w);
     __syncthreads();
     bucket(ids, T * k, E, offsets, perm, pos, active, n_active, hist, bucket_chunks(E));
@@ -228,10 +243,12 @@ __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_fused_kernel(const flo
 constexpr int ROUTE_TOKENS_PER_CTA = 256;
 
 __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_topk_kernel(const float *logits, int T, int E, int k,
-                                                                     int renorm, int32_t *ids, float *w)
+                                                                     int renorm, int32_t *ids, float *w,
+                                                                     const uint16_t *x, __half *x16, int H)
 {
     grid_dep_wait();
     const int t0 = blockIdx.x * ROUTE_TOKENS_PER_CTA;
+    convert_rows(x, x16, t0, min(T, t0 + ROUTE_TOKENS_PER_CTA), H);
     route_range(logits, t0, min(T, t0 + ROUTE_TOKENS_PER_CTA), E, k, renorm, ids, w);
 }
 
@@ -264,7 +281,7 @@ cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
 
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int32_t *ids, float *w,
                          int32_t *offsets, int32_t *perm, int32_t *pos, int32_t *active, int32_t *n_active,
-                         cudaStream_t s, bool pdl)
+                         const uint16_t *x, __half *x16, int H, cudaStream_t s, bool pdl)
 {
     static bool attr_set = false;
     if (!attr_set) {
@@ -280,10 +297,10 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
     const size_t smem = (size_t)chunks * E * sizeof(int32_t);
     if (T <= ROUTE_TOKENS_PER_CTA)
         return launch_ex(vq_route_fused_kernel, dim3(1), dim3(ROUTE_THREADS), smem, s, pdl, logits, T, E, k, renorm,
-                         ids, w, offsets, perm, pos, active, n_active);
+                         ids, w, offsets, perm, pos, active, n_active, x, x16, H);
     const int ctas = (T + ROUTE_TOKENS_PER_CTA - 1) / ROUTE_TOKENS_PER_CTA;
     cudaError_t err = launch_ex(vq_route_topk_kernel, dim3(ctas), dim3(ROUTE_THREADS), 0, s, pdl, logits, T, E, k,
-                                renorm, ids, w);
+                                renorm, ids, w, x, x16, H);
     if (err != cudaSuccess)
         return err;
     return launch_ex(vq_bucket_kernel, dim3(1), dim3(ROUTE_THREADS), smem, s, pdl, (const int32_t *)ids, T * k, E,
