@@ -193,6 +193,27 @@ vq_status vq_moe_prefill(const vq_moe_layer *L, const uint16_t *x, int32_t T, co
                          int32_t top_k, int32_t renorm, void *y, int32_t y_dtype, void *workspace,
                          size_t ws_bytes, void *stream);
 
+/* vq_moe_decode without a workspace argument, for callers that cannot
+ * allocate device memory: code running inside a host framework that owns
+ * every device allocation and allows no new ones on its serving path, or a
+ * program that reaches this library through a thin C FFI without a CUDA
+ * memory API. The paper has no counterpart; the layer computed is exactly
+ * vq_moe_decode's, with the same arguments minus the workspace.
+ *
+ * Scratch: one 16 MiB file-scope device array inside the library. Every GPU
+ * that loads the library holds it until the process exits. Calls whose
+ * vq_moe_workspace_size(L, T, top_k, VQ_MODE_DECODE) exceeds 16 MiB return
+ * VQ_ERR_WORKSPACE and launch nothing.
+ * Set-up: the first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.
+ * Sharing: all calls on a device use the same array and it keeps the last
+ * call's contents (no call needs it zeroed: each writes what it reads).
+ * Calls that overlap on the GPU (other streams, other host threads) race on
+ * it; serialise them. The library allocates nothing for this call. */
+vq_status vq_moe_decode_noalloc(const vq_moe_layer *L, const uint16_t *x, int32_t T, const float *logits,
+                                int32_t top_k, int32_t renorm, void *y, int32_t y_dtype, void *stream);
+
 /* Tracing (no counterpart on the pages; an observability hook for timing
  * each kernel stage with the caller's CUDA events). events: host array of
  * n_events cudaEvent_t handles (as void*) created by the caller, or NULL to

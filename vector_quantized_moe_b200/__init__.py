@@ -64,6 +64,7 @@ def _load():
         "vq_moe_decode": (ctypes.c_int, [LP, P, I32, P, I32, I32, P, I32, P, SZ, P]),
         "vq_moe_prefill": (ctypes.c_int, [LP, P, I32, P, I32, I32, P, I32, P, SZ, P]),
         "vq_set_trace_events": (ctypes.c_int, [P, I32]),
+        "vq_moe_decode_noalloc": (ctypes.c_int, [LP, P, I32, P, I32, I32, P, I32, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
