@@ -88,6 +88,10 @@ typedef struct vq_module {
      * packed-row index of the first live row at or after row 32*w of expert
      * e (vq_live_rank builds it). */
     const uint32_t *live_rank;
+    /* number of packed rows in `codes` and `scales` (the extent the kernels
+     * may read); required when live_bitmap is set, ignored (E * rows)
+     * otherwise. */
+    int64_t live_rows;
 } vq_module;
 
 /* A SwiGLU MoE layer: y = sum_j w_j * down_e( silu(gate_e x) * up_e x ).
@@ -186,9 +190,11 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
 /* The same layer for prefill-sized batches (many tokens per expert): per
  * expert bucket a grouped GEMM on the tcgen05 tensor cores with the weight
  * tiles decoded on chip. Same arguments and result definition as
- * vq_moe_decode; workspace sized with VQ_MODE_PREFILL. Additionally requires
- * every module's packed row to be a multiple of 16 bytes
- * ((cols / d / 32) * bits divisible by 4). */
+ * vq_moe_decode; workspace sized with VQ_MODE_PREFILL. Additionally requires,
+ * for every module, a packed row that is a multiple of 16 bytes
+ * ((cols / d / 32) * bits divisible by 4) and cols a multiple of 64 * CH,
+ * CH being the smallest number of 64-column steps whose codes fill a whole
+ * number of 16-byte units (VQ_ERR_UNSUPPORTED otherwise). */
 vq_status vq_moe_prefill(const vq_moe_layer *L, const uint16_t *x, int32_t T, const float *logits,
                          int32_t top_k, int32_t renorm, void *y, int32_t y_dtype, void *workspace,
                          size_t ws_bytes, void *stream);

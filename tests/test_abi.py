@@ -81,7 +81,7 @@ def _null_module(**kw):
              live_rank=None)
     m.update(kw)
     return vq.vq_module(m["E"], m["rows"], m["cols"], m["d"], m["bits"], m["codes"], m["scales"], m["codebook"],
-                        m["live_bitmap"], m["live_rank"])
+                        m["live_bitmap"], m["live_rank"], m.get("live_rows", 0))
 
 
 @pytest.mark.parametrize("kw,status", [

@@ -35,7 +35,7 @@ class vq_module(ctypes.Structure):
     _fields_ = [("E", ctypes.c_int32), ("rows", ctypes.c_int32), ("cols", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("bits", ctypes.c_int32),
                 ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("codebook", ctypes.c_void_p),
-                ("live_bitmap", ctypes.c_void_p), ("live_rank", ctypes.c_void_p)]
+                ("live_bitmap", ctypes.c_void_p), ("live_rank", ctypes.c_void_p), ("live_rows", ctypes.c_int64)]
 
 
 class vq_moe_layer(ctypes.Structure):
@@ -185,7 +185,8 @@ class Module:
 
     def struct(self) -> vq_module:
         return vq_module(self.E, self.rows, self.cols, self.d, self.bits, _ptr(self.codes), _ptr(self.scales),
-                         _ptr(self.codebook), _ptr(self.live_bitmap), _ptr(self.live_rank))
+                         _ptr(self.codebook), _ptr(self.live_bitmap), _ptr(self.live_rank),
+                         int(self.scales.shape[0]))
 
 
 def unpack(m: Module, expert: int, stream=None):

@@ -47,7 +47,7 @@ vq_status check_module(const vq_module *m)
         return VQ_ERR_ARG;
     if (m->cols % (32 * m->d) != 0 || m->bits < 1 || m->bits > 16)
         return VQ_ERR_ARG;
-    if (m->live_bitmap && !m->live_rank)
+    if (m->live_bitmap && (!m->live_rank || m->live_rows < 1 || m->live_rows > (int64_t)m->E * m->rows))
         return VQ_ERR_ARG;
     if (!geometry_ok(m->d, m->bits))
         return VQ_ERR_UNSUPPORTED;
@@ -136,6 +136,7 @@ ModDev make_moddev(const vq_module &m)
     d.row_words = (m.cols / m.d / 32) * m.bits;
     d.ngroups = m.cols / 64;
     d.bm_words = (m.rows + 31) / 32;
+    d.live_rows = m.live_bitmap ? m.live_rows : (int64_t)m.E * m.rows;
     const size_t entry = std::max(4, 2 * m.d);
     const int full = (int)(128 / entry);
     int rep = full;

@@ -25,6 +25,7 @@ struct ModDev {
     int row_words;   // uint32 words per packed row
     int ngroups;     // cols / 64
     int bm_words;    // ceil(rows / 32)
+    int64_t live_rows;  // packed rows in codes / scales
     int rep;         // codebook replicas in shared memory (power of two)
     int log_rep;
 };

@@ -1,19 +1,822 @@
-// Prefill path of the VQ-MoE layer (tcgen05 grouped GEMM): not built yet.
+// Prefill path of the VQ-MoE layer on sm_100a: per expert bucket a grouped
+// GEMM on the 5th-generation tensor cores (tcgen05.mma, fp32 accumulators in
+// tensor memory) with the weight tiles decoded on chip.
+//
+// Format (VQ model cards): Qwen3.5-397B-A17B-VQ-2.6bpw "Methodology" (one
+// index per d-weight subvector into an fp16 codebook, fp16 scale per
+// (row, 64 weights)); Qwen3.5-397B-A17B-VQ-2.4bpw "Methodology" (uint32
+// words, row-local 32-code blocks) and "Changelog 2026-10-01" (skipzero).
+// The gemma-4 card ("Faster prefill") describes its Apple-GPU prefill only as
+// decoding weights in chunks before the matmul; this kernel is a new design.
+//
+// One CTA per SM, persistent over (expert, 128-row weight tile, 128-token
+// tile) work items. Warp roles:
+//   warp 0     TMA: activation tiles (fp16, 128B-swizzled, one 64-column
+//              k-step per stage) and packed-code tiles (a chunk of CH k-steps)
+//   warp 1     owns the tensor memory; one thread issues tcgen05.mma
+//   warps 2-5  thread i decodes row i of the weight tile for each k-step
+//              (unpack, codebook lookup, x fp16 scale) into the swizzled
+//              K-major shared-memory layout the tensor core reads, then runs
+//              the epilogue from tensor memory (lane i = row i)
+// D[row, token] = sum_k W[row, k] X[token, k]: the weight tile is the
+// M=128 operand, the tokens of the bucket the N operand (16..128), so small
+// buckets waste no M rows. Every mbarrier wait is bounded; on a timeout the
+// CTA records an error word, stops, and frees its tensor memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <utility>
+
+#include "vq_device.cuh"
 #include "vq_internal.h"
 
 namespace vq {
+namespace {
+
+constexpr int BM = 128;             // weight rows per tile = TMEM lanes
+constexpr int BN = 128;             // tokens per tile
+constexpr int NTHREADS = 192;       // 6 warps
+constexpr uint32_t WAIT_LIMIT = 1u << 22;
+constexpr int A_TILE = BM * 128;    // bytes of one 128 x 64 fp16 tile
+constexpr int B_TILE = BN * 128;
+
+__host__ __device__ constexpr int chunk_steps(int kb)
+{
+    int ch = 1;
+    while ((ch * kb) % 128)
+        ++ch;
+    return ch;
+}
+
+template <int D, int BITS>
+struct PG {
+    static constexpr int KB = (64 / D) * BITS;       // code bits of one row per 64-column step
+    static constexpr int CH = chunk_steps(KB);       // steps per code chunk (whole 16-byte units)
+    static constexpr int CHW = CH * KB / 32;         // words per row per chunk
+    static constexpr uint32_t MASK = (1u << BITS) - 1u;
+};
+
+struct PrefillArgs {
+    CUtensorMap tmap_b;       // activations fp16 [slots, K], box {64, BN}, 128B swizzle
+    CUtensorMap tmap_c[2];    // packed codes u32 [live rows, row_words], box {CHW, BM}
+    ModDev mod[2];
+    int nmod;
+    const int32_t *offsets;
+    const int32_t *active;
+    const int32_t *n_active;
+    int K;                    // contraction length
+    int rows;                 // weight rows (M)
+    int sa, sc;               // operand stages, code stages
+    uint32_t off_a, off_b, off_c, off_cb, off_tiles, off_bar;
+    void *out;                // SwiGLU: fp16 [slots, rows]; else fp32 [slots, rows]
+    int swiglu;
+    int *err;
+};
+
+// ------------------------------------------------------------------ PTX
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait on a phase; false when it gave up (limit reached or the CTA aborted).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *err,
+                                          int code)
+{
+    for (uint32_t i = 0; i < WAIT_LIMIT; ++i) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if ((i & 63) == 63 && *abort_flag)
+            return false;
+    }
+    *abort_flag = 1;
+    atomicExch(err, code);
+    return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// K-major operand in the 128-byte swizzled canonical layout: rows of 128 B,
+// 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
+{
+    uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)1 << 16;              // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;    // stride byte offset: 8 rows x 128 B
+    d |= (uint64_t)1 << 46;              // descriptor version (sm_100)
+    d |= (uint64_t)2 << 61;              // 128-byte swizzle
+    return d;
+}
+
+// fp16 x fp16 -> fp32, A and B K-major, M = 128, N = n.
+__device__ __forceinline__ uint32_t idesc_f16(int n)
+{
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b)
+{
+    __half2 r = __hmul2(*reinterpret_cast<__half2 *>(&a), *reinterpret_cast<__half2 *>(&b));
+    return *reinterpret_cast<uint32_t *>(&r);
+}
+
+// ------------------------------------------------------------------ dequant
+
+template <int BITS, int NW>
+__device__ __forceinline__ uint32_t code_at(const uint32_t (&w)[NW], int pos)
+{
+    const int wi = pos >> 5, sh = pos & 31;
+    if (sh + BITS <= 32)
+        return (w[wi] >> sh) & ((1u << BITS) - 1u);
+    return __funnelshift_r(w[wi], w[wi + 1], sh) & ((1u << BITS) - 1u);
+}
+
+// Row `row` of the 128 x 64 fp16 weight tile for k-step JJ of the chunk held
+// in w: 64 weights = 64/D codes, each a codebook entry times the row's scale
+// (fp16 product, rounded to nearest), stored as eight 16-byte chunks at
+// swizzled positions (chunk q of row r at q ^ (r & 7)).
+template <int D, int BITS, int JJ>
+__device__ __forceinline__ void dequant_step(const uint32_t (&w)[PG<D, BITS>::CHW], const char *cb, uint32_t s2,
+                                             bool live, char *arow, int rsw)
+{
+    constexpr int NC = 64 / D;
+    constexpr int KB = PG<D, BITS>::KB;
+    uint32_t o[32];
+    if constexpr (D == 1) {
+#pragma unroll
+        for (int c = 0; c < NC; c += 2) {
+            const uint32_t c0 = code_at<BITS>(w, JJ * KB + c * BITS);
+            const uint32_t c1 = code_at<BITS>(w, JJ * KB + (c + 1) * BITS);
+            const uint32_t v = (uint32_t)*reinterpret_cast<const uint16_t *>(cb + 2 * c0) |
+                               ((uint32_t)*reinterpret_cast<const uint16_t *>(cb + 2 * c1) << 16);
+            o[c >> 1] = hmul2(v, s2);
+        }
+    } else if constexpr (D == 2) {
+#pragma unroll
+        for (int c = 0; c < NC; ++c)
+            o[c] = hmul2(*reinterpret_cast<const uint32_t *>(cb + 4 * code_at<BITS>(w, JJ * KB + c * BITS)), s2);
+    } else if constexpr (D == 4) {
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(cb + 8 * code_at<BITS>(w, JJ * KB + c * BITS));
+            o[2 * c] = hmul2(v.x, s2);
+            o[2 * c + 1] = hmul2(v.y, s2);
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(cb + 16 * code_at<BITS>(w, JJ * KB + c * BITS));
+            o[4 * c] = hmul2(v.x, s2);
+            o[4 * c + 1] = hmul2(v.y, s2);
+            o[4 * c + 2] = hmul2(v.z, s2);
+            o[4 * c + 3] = hmul2(v.w, s2);
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        uint4 v = live ? make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]) : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4 *>(arow + ((q ^ rsw) << 4)) = v;
+    }
+}
+
+template <int D, int BITS, int JJ>
+__device__ __forceinline__ void dequant_chunk_steps(const uint32_t (&w)[2][PG<D, BITS>::CHW], const char *cb0,
+                                                    const char *cb1, const uint32_t (&s2)[2][PG<D, BITS>::CH],
+                                                    bool live0, bool live1, int nmod, char *a_stage, int rowi)
+{
+    char *arow = a_stage + rowi * 128;
+    dequant_step<D, BITS, JJ>(w[0], cb0, s2[0][JJ], live0, arow, rowi & 7);
+    if (nmod == 2)
+        dequant_step<D, BITS, JJ>(w[1], cb1, s2[1][JJ], live1, arow + A_TILE, rowi & 7);
+}
+
+// ------------------------------------------------------------------ kernel
+
+struct Item {
+    int e, m0, q0, n;
+};
+
+__device__ __forceinline__ Item item_of(long it, int MT, const int *tiles, int n_act, const int32_t *active,
+                                        const int32_t *offsets)
+{
+    const int mt = (int)(it % MT);
+    const int ntg = (int)(it / MT);
+    int lo = 0, hi = n_act;   // last ai with tiles[ai] <= ntg
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (tiles[mid] <= ntg)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    Item r;
+    r.e = active[lo];
+    const int nt = ntg - tiles[lo];
+    r.m0 = mt * BM;
+    r.q0 = offsets[r.e] + nt * BN;
+    r.n = min(BN, offsets[r.e + 1] - r.q0);
+    return r;
+}
+
+// packed row of the first row of an m-tile (m0 is a multiple of 128)
+__device__ __forceinline__ int tile_prow0(const ModDev &m, int e, int m0)
+{
+    if (!m.bitmap)
+        return e * m.rows + m0;
+    return (int)m.rank[(long)e * m.bm_words + (m0 >> 5)];
+}
+
+template <int D, int BITS>
+__global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __grid_constant__ PrefillArgs a)
+{
+    using P = PG<D, BITS>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *sm_a = smem + a.off_a;
+    uint8_t *sm_b = smem + a.off_b;
+    uint8_t *sm_c = smem + a.off_c;
+    char *sm_cb = reinterpret_cast<char *>(smem + a.off_cb);
+    int *tiles = reinterpret_cast<int *>(smem + a.off_tiles);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + a.off_bar);
+    uint64_t *full_a = bars, *full_b = bars + a.sa, *empty = bars + 2 * a.sa;
+    uint64_t *full_c = bars + 3 * a.sa, *empty_c = full_c + a.sc, *acc_full = empty_c + a.sc;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(acc_full + 1);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nmod = a.nmod;
+    const int cb_bytes = (1 << BITS) * D * 2;
+
+    // codebooks (fp16 [K, d] per module) into shared memory
+    for (int i = threadIdx.x; i < nmod * cb_bytes / 16; i += NTHREADS) {
+        const int m = i / (cb_bytes / 16), j = i % (cb_bytes / 16);
+        reinterpret_cast<uint4 *>(sm_cb + m * cb_bytes)[j] =
+            reinterpret_cast<const uint4 *>(m == 0 ? a.mod[0].codebook : a.mod[1].codebook)[j];
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < a.sa; ++s) {
+            mbar_init(&full_a[s], 128);
+            mbar_init(&full_b[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int s = 0; s < a.sc; ++s) {
+            mbar_init(&full_c[s], 1);
+            mbar_init(&empty_c[s], 128);
+        }
+        mbar_init(acc_full, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    const uint32_t tmem_cols = nmod == 2 ? 2 * BN : BN;
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(tmem_cols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    grid_dep_wait();
+
+    // tile prefix over the active experts: tiles[ai] = first global n-tile of expert active[ai]
+    const int n_act = *a.n_active;
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int ai = 0; ai < n_act; ++ai) {
+            tiles[ai] = run;
+            const int e = a.active[ai];
+            run += (a.offsets[e + 1] - a.offsets[e] + BN - 1) / BN;
+        }
+        tiles[n_act] = run;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int MT = (a.rows + BM - 1) / BM;
+    const long n_items = (long)tiles[n_act] * MT;
+    const int ksteps = a.K / 64;
+    const int nchunks = ksteps / P::CH;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            uint32_t ks = 0, cs = 0;
+            bool ok = true;
+            for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+                const Item itm = item_of(it, MT, tiles, n_act, a.active, a.offsets);
+                int prow0[2];
+                for (int m = 0; m < nmod; ++m)
+                    prow0[m] = tile_prow0(a.mod[m], itm.e, itm.m0);
+                for (int c = 0; c < nchunks && ok; ++c) {
+                    const uint32_t cst = cs % a.sc, cph = (cs / a.sc) & 1;
+                    if (!(ok = mbar_wait(&empty_c[cst], cph ^ 1, abort_flag, a.err, 1)))
+                        break;
+                    mbar_expect_tx(&full_c[cst], (uint32_t)(nmod * BM * P::CHW * 4));
+                    for (int m = 0; m < nmod; ++m)
+                        tma_load_2d(sm_c + ((size_t)cst * nmod + m) * BM * P::CHW * 4, &a.tmap_c[m], c * P::CHW,
+                                    prow0[m], &full_c[cst]);
+                    ++cs;
+                    for (int j = 0; j < P::CH; ++j) {
+                        const uint32_t st = ks % a.sa, ph = (ks / a.sa) & 1;
+                        if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag, a.err, 2)))
+                            break;
+                        mbar_expect_tx(&full_b[st], (uint32_t)B_TILE);
+                        tma_load_2d(sm_b + (size_t)st * B_TILE, &a.tmap_b, (c * P::CH + j) * 64, itm.q0, &full_b[st]);
+                        ++ks;
+                    }
+                }
+            }
+            if (!ok) {
+                // let the loads already issued land before the CTA leaves
+                for (uint32_t s = 0; s < (uint32_t)a.sa; ++s)
+                    if (ks > s)
+                        mbar_wait(&full_b[(ks - 1 - s) % a.sa], ((ks - 1 - s) / a.sa) & 1, abort_flag, a.err, 3);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            uint32_t ks = 0;
+            bool ok = true;
+            for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+                const Item itm = item_of(it, MT, tiles, n_act, a.active, a.offsets);
+                const int n16 = (itm.n + 15) & ~15;
+                const uint32_t idesc = idesc_f16(n16);
+                for (int k = 0; k < ksteps; ++k) {
+                    const uint32_t st = ks % a.sa, ph = (ks / a.sa) & 1;
+                    if (!(ok = mbar_wait(&full_a[st], ph, abort_flag, a.err, 4)))
+                        break;
+                    if (!(ok = mbar_wait(&full_b[st], ph, abort_flag, a.err, 5)))
+                        break;
+                    tc_fence_after();
+                    const uint64_t bdesc = sw128_desc(smem_u32(sm_b + (size_t)st * B_TILE));
+                    for (int m = 0; m < nmod; ++m) {
+                        const uint64_t adesc = sw128_desc(smem_u32(sm_a + ((size_t)st * nmod + m) * A_TILE));
+#pragma unroll
+                        for (int k16 = 0; k16 < 4; ++k16)
+                            umma(tmem + m * BN, adesc + 2 * k16, bdesc + 2 * k16, idesc, (k | k16) != 0);
+                    }
+                    umma_commit(&empty[st]);
+                    ++ks;
+                }
+                if (ok)
+                    umma_commit(acc_full);
+            }
+        }
+    } else {
+        // ---------------------------------------------------------- dequant + epilogue
+        const int rowi = 32 * (warp & 3) + lane;
+        const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
+        uint32_t ks = 0, cs = 0, nit = 0;
+        bool ok = true;
+        for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+            const Item itm = item_of(it, MT, tiles, n_act, a.active, a.offsets);
+            const int r = itm.m0 + rowi;
+            int lrow[2] = {-1, -1};
+            long prow[2] = {-1, -1};
+            for (int m = 0; m < nmod; ++m) {
+                const ModDev &md = a.mod[m];
+                prow[m] = r < a.rows ? live_row(md.bitmap, md.rank, md.bm_words, md.rows, itm.e, r) : -1;
+                lrow[m] = prow[m] >= 0 ? (int)(prow[m] - tile_prow0(md, itm.e, itm.m0)) : -1;
+            }
+            for (int c = 0; c < nchunks && ok; ++c) {
+                // scales of this chunk's k-steps, then the chunk's code words
+                uint32_t s2[2][P::CH];
+#pragma unroll
+                for (int m = 0; m < 2; ++m)
+#pragma unroll
+                    for (int j = 0; j < P::CH; ++j) {
+                        uint32_t s = 0;
+                        if (m < nmod && prow[m] >= 0)
+                            s = ldg_u16(a.mod[m].scales + prow[m] * a.mod[m].ngroups + c * P::CH + j);
+                        s2[m][j] = s | (s << 16);
+                    }
+                const uint32_t cst = cs % a.sc, cph = (cs / a.sc) & 1;
+                if (!(ok = mbar_wait(&full_c[cst], cph, abort_flag, a.err, 6)))
+                    break;
+                uint32_t w[2][P::CHW];
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(
+                        sm_c + ((size_t)cst * nmod + (m < nmod ? m : 0)) * BM * P::CHW * 4 +
+                        (size_t)(lrow[m] >= 0 ? lrow[m] : 0) * P::CHW * 4);
+#pragma unroll
+                    for (int q = 0; q < P::CHW / 4; ++q) {
+                        const uint4 v = (m < nmod) ? src[q] : make_uint4(0u, 0u, 0u, 0u);
+                        w[m][4 * q] = v.x;
+                        w[m][4 * q + 1] = v.y;
+                        w[m][4 * q + 2] = v.z;
+                        w[m][4 * q + 3] = v.w;
+                    }
+                }
+                mbar_arrive(&empty_c[cst]);
+                ++cs;
+                auto step = [&](auto jj_c) {
+                    constexpr int JJ = decltype(jj_c)::value;
+                    if (!ok)
+                        return;
+                    const uint32_t st = ks % a.sa, ph = (ks / a.sa) & 1;
+                    if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag, a.err, 7)))
+                        return;
+                    dequant_chunk_steps<D, BITS, JJ>(w, sm_cb, sm_cb + cb_bytes, s2, lrow[0] >= 0, lrow[1] >= 0,
+                                                     nmod, reinterpret_cast<char *>(sm_a) + (size_t)st * nmod * A_TILE,
+                                                     rowi);
+                    fence_async_smem();
+                    mbar_arrive(&full_a[st]);
+                    ++ks;
+                };
+                [&]<int... J>(std::integer_sequence<int, J...>) {
+                    (step(std::integral_constant<int, J>{}), ...);
+                }(std::make_integer_sequence<int, P::CH>{});
+            }
+            if (!ok)
+                break;
+            // epilogue: accumulators of this tile are complete
+            if (!(ok = mbar_wait(acc_full, nit & 1, abort_flag, a.err, 8)))
+                break;
+            ++nit;
+            tc_fence_after();
+            for (int cb0 = 0; cb0 < itm.n; cb0 += 32) {
+                uint32_t g[32], u[32];
+                tmem_ld32(tmem + lane_addr + cb0, g);
+                if (nmod == 2)
+                    tmem_ld32(tmem + lane_addr + BN + cb0, u);
+                tmem_wait_ld();
+                if (r < a.rows) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = cb0 + j;
+                        if (n >= itm.n)
+                            break;
+                        const long o = (long)(itm.q0 + n) * a.rows + r;
+                        if (a.swiglu) {
+                            const float gv = __uint_as_float(g[j]), uv = __uint_as_float(u[j]);
+                            reinterpret_cast<__half *>(a.out)[o] = __float2half_rn(gv / (1.f + __expf(-gv)) * uv);
+                        } else {
+                            reinterpret_cast<float *>(a.out)[o] = __uint_as_float(g[j]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tmem_cols));
+    }
+}
+
+// gathered activations: Xg[q, :] = fp16(x[perm[q] / k, :])
+__global__ void vq_gather_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ perm, int k, long slots,
+                                 int H, __half *__restrict__ xg)
+{
+    grid_dep_wait();
+    const int per_row = H / 8;
+    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < slots * per_row; i += (long)gridDim.x * blockDim.x) {
+        const long q = i / per_row;
+        const int c = (int)(i % per_row) * 8;
+        const long t = perm[q] / k;
+        const uint4 v = ldg_u128(x + t * H + c);
+        uint4 o;
+        o.x = bf16x2_to_f16x2(v.x);
+        o.y = bf16x2_to_f16x2(v.y);
+        o.z = bf16x2_to_f16x2(v.z);
+        o.w = bf16x2_to_f16x2(v.w);
+        *reinterpret_cast<uint4 *>(xg + q * H + c) = o;
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+bool make_map_f16(CUtensorMap *map, const void *base, long rows, int cols)
+{
+    auto enc = encode_fn();
+    if (!enc)
+        return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {64, BN};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_codes(CUtensorMap *map, const ModDev &m, int chw)
+{
+    auto enc = encode_fn();
+    if (!enc)
+        return false;
+    cuuint64_t dims[2] = {(cuuint64_t)m.row_words, (cuuint64_t)m.live_rows};
+    cuuint64_t strides[1] = {(cuuint64_t)m.row_words * 4};
+    cuuint32_t box[2] = {(cuuint32_t)chw, BM};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(m.codes), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int chw_of(int d, int bits)
+{
+    const int kb = (64 / d) * bits;
+    return chunk_steps(kb) * kb / 32;
+}
+
+int ch_of(int d, int bits) { return chunk_steps((64 / d) * bits); }
+
+struct SmemPlan {
+    int sa, sc;
+    uint32_t off_a, off_b, off_c, off_cb, off_tiles, off_bar, total;
+};
+
+SmemPlan smem_plan(int nmod, int d, int bits, int E)
+{
+    const uint32_t limit = 227 * 1024 - 1024;   // minus the alignment slack
+    const uint32_t code_stage = (uint32_t)nmod * BM * chw_of(d, bits) * 4;
+    const uint32_t cb = (uint32_t)align_up((size_t)nmod * ((size_t)1 << bits) * d * 2, 128);
+    const uint32_t tiles = (uint32_t)align_up((size_t)(E + 1) * 4, 128);
+    SmemPlan p{};
+    for (int sa = 4; sa >= 2; --sa) {
+        p.sa = sa;
+        p.sc = 2;
+        p.off_a = 0;
+        p.off_b = p.off_a + (uint32_t)sa * nmod * A_TILE;
+        p.off_c = p.off_b + (uint32_t)sa * B_TILE;
+        p.off_cb = p.off_c + p.sc * code_stage;
+        p.off_tiles = p.off_cb + cb;
+        p.off_bar = (uint32_t)align_up(p.off_tiles + tiles, 8);
+        p.total = p.off_bar + (3 * sa + 2 * p.sc + 1) * 8 + 16 + 1024;
+        if (p.total <= limit + 1024)
+            return p;
+    }
+    p.total = 0;
+    return p;
+}
+
+template <int D, int BITS>
+cudaError_t launch_gemm(const PrefillArgs &a, int ctas, uint32_t smem, cudaStream_t s)
+{
+    auto k = vq_prefill_gemm_kernel<D, BITS>;
+    cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess)
+        return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ctas);
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, a);
+}
+
+cudaError_t dispatch_gemm(const PrefillArgs &a, int d, int bits, int ctas, uint32_t smem, cudaStream_t s)
+{
+#define VQ_PGEMM(D_, B_) \
+    if (d == D_ && bits == B_) return launch_gemm<D_, B_>(a, ctas, smem, s);
+    VQ_GEOMETRIES(VQ_PGEMM)
+#undef VQ_PGEMM
+    return cudaErrorInvalidValue;
+}
+
+struct PrefillPlan {
+    RoutingLayout r;
+    size_t err, xg, h, dp, total;
+};
+
+PrefillPlan plan_prefill(const vq_moe_layer *L, int T, int k)
+{
+    PrefillPlan p{};
+    size_t o = 0;
+    p.r = plan_routing(o, T, k, L->gate.E);
+    const size_t tk = (size_t)T * k;
+    p.err = o; o = align_up(o + 16, 256);
+    p.xg = o; o = align_up(o + tk * L->gate.cols * 2, 256);
+    p.h = o; o = align_up(o + tk * L->gate.rows * 2, 256);
+    p.dp = o; o = align_up(o + tk * L->down.rows * 4, 256);
+    p.total = o;
+    return p;
+}
+
+bool module_prefill_ok(const vq_module &m)
+{
+    const int row_words = (m.cols / m.d / 32) * m.bits;
+    return row_words % 4 == 0 && m.cols % (64 * ch_of(m.d, m.bits)) == 0;
+}
+
+}  // namespace
 
 size_t prefill_workspace_size(const vq_moe_layer *L, int T, int k)
 {
-    size_t o = 0;
-    plan_routing(o, T, k, L->gate.E);
-    return o;
+    return plan_prefill(L, T, k).total;
 }
 
-vq_status run_prefill(const vq_moe_layer *, const uint16_t *, int, const float *, int, int, void *, int, void *,
-                      size_t, cudaStream_t)
+vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const float *logits, int k, int renorm, void *y,
+                      int y_dtype, void *ws, size_t ws_bytes, cudaStream_t s)
 {
-    return VQ_ERR_UNSUPPORTED;
+    if (!module_prefill_ok(L->gate) || !module_prefill_ok(L->up) || !module_prefill_ok(L->down))
+        return VQ_ERR_UNSUPPORTED;
+    if (L->gate.d != L->up.d || L->gate.bits != L->up.bits)
+        return VQ_ERR_UNSUPPORTED;   // gate and up share one fused tile
+    if (!encode_fn())
+        return VQ_ERR_CUDA;
+    const int E = L->gate.E, H = L->gate.cols, I = L->gate.rows;
+    if (T == 0)
+        return VQ_OK;
+    const PrefillPlan p = plan_prefill(L, T, k);
+    if (ws_bytes < p.total)
+        return VQ_ERR_WORKSPACE;
+    int32_t *ids = ws_at<int32_t>(ws, p.r.ids);
+    float *w = ws_at<float>(ws, p.r.w);
+    int32_t *offsets = ws_at<int32_t>(ws, p.r.offsets);
+    int32_t *perm = ws_at<int32_t>(ws, p.r.perm);
+    int32_t *pos = ws_at<int32_t>(ws, p.r.pos);
+    int32_t *active = ws_at<int32_t>(ws, p.r.active);
+    int32_t *nact = ws_at<int32_t>(ws, p.r.nact);
+    int *err = ws_at<int>(ws, p.err);
+    __half *xg = ws_at<__half>(ws, p.xg);
+    __half *hh = ws_at<__half>(ws, p.h);
+    float *dp = ws_at<float>(ws, p.dp);
+    const long tk = (long)T * k;
+
+    trace_point(0, s);
+    cudaError_t e = launch_route(logits, T, E, k, renorm, ids, w, offsets, perm, pos, active, nact, nullptr, nullptr, 0,
+                                 s, true);
+    if (e != cudaSuccess)
+        return VQ_ERR_CUDA;
+    if (cudaMemsetAsync(err, 0, 4, s) != cudaSuccess)
+        return VQ_ERR_CUDA;
+    trace_point(1, s);
+    {
+        cudaLaunchConfig_t cfg = {};
+        const long n = tk * (H / 8);
+        cfg.gridDim = dim3((unsigned)std::min<long>((n + 255) / 256, 8192));
+        cfg.blockDim = dim3(256);
+        cfg.stream = s;
+        e = cudaLaunchKernelEx(&cfg, vq_gather_kernel, x, (const int32_t *)perm, k, tk, H, xg);
+        if (e != cudaSuccess)
+            return VQ_ERR_CUDA;
+    }
+    trace_point(2, s);
+
+    const int sms = num_sms();
+    // gate/up with the SwiGLU epilogue -> h fp16 [slots, inter]
+    {
+        PrefillArgs a{};
+        a.mod[0] = make_moddev(L->gate);
+        a.mod[1] = make_moddev(L->up);
+        a.nmod = 2;
+        if (!make_map_f16(&a.tmap_b, xg, tk, H) ||
+            !make_map_codes(&a.tmap_c[0], a.mod[0], chw_of(a.mod[0].d, a.mod[0].bits)) ||
+            !make_map_codes(&a.tmap_c[1], a.mod[1], chw_of(a.mod[1].d, a.mod[1].bits)))
+            return VQ_ERR_CUDA;
+        a.offsets = offsets;
+        a.active = active;
+        a.n_active = nact;
+        a.K = H;
+        a.rows = I;
+        const SmemPlan sp = smem_plan(2, a.mod[0].d, a.mod[0].bits, E);
+        if (sp.total == 0)
+            return VQ_ERR_UNSUPPORTED;
+        a.sa = sp.sa;
+        a.sc = sp.sc;
+        a.off_a = sp.off_a;
+        a.off_b = sp.off_b;
+        a.off_c = sp.off_c;
+        a.off_cb = sp.off_cb;
+        a.off_tiles = sp.off_tiles;
+        a.off_bar = sp.off_bar;
+        a.out = hh;
+        a.swiglu = 1;
+        a.err = err;
+        e = dispatch_gemm(a, a.mod[0].d, a.mod[0].bits, sms, sp.total, s);
+        if (e != cudaSuccess)
+            return VQ_ERR_CUDA;
+    }
+    trace_point(3, s);
+    // down -> fp32 per-slot outputs [slots, hidden]
+    {
+        PrefillArgs a{};
+        a.mod[0] = make_moddev(L->down);
+        a.mod[1] = a.mod[0];
+        a.nmod = 1;
+        if (!make_map_f16(&a.tmap_b, hh, tk, I) ||
+            !make_map_codes(&a.tmap_c[0], a.mod[0], chw_of(a.mod[0].d, a.mod[0].bits)))
+            return VQ_ERR_CUDA;
+        a.tmap_c[1] = a.tmap_c[0];
+        a.offsets = offsets;
+        a.active = active;
+        a.n_active = nact;
+        a.K = I;
+        a.rows = H;
+        const SmemPlan sp = smem_plan(1, a.mod[0].d, a.mod[0].bits, E);
+        if (sp.total == 0)
+            return VQ_ERR_UNSUPPORTED;
+        a.sa = sp.sa;
+        a.sc = sp.sc;
+        a.off_a = sp.off_a;
+        a.off_b = sp.off_b;
+        a.off_c = sp.off_c;
+        a.off_cb = sp.off_cb;
+        a.off_tiles = sp.off_tiles;
+        a.off_bar = sp.off_bar;
+        a.out = dp;
+        a.swiglu = 0;
+        a.err = err;
+        e = dispatch_gemm(a, a.mod[0].d, a.mod[0].bits, sms, sp.total, s);
+        if (e != cudaSuccess)
+            return VQ_ERR_CUDA;
+    }
+    trace_point(4, s);
+    e = launch_combine(dp, 1, 0, w, pos, T, k, H, y, y_dtype, s, true);
+    trace_point(5, s);
+    return e == cudaSuccess ? VQ_OK : VQ_ERR_CUDA;
 }
 
 }  // namespace vq
