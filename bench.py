@@ -193,6 +193,13 @@ def run_ours(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
+    if args.only == "prefill":
+        layer_p, fn = measure_prefill(torch, vq, dev, args.steps, args.warmup, small=args.small, ncu_mode=True)
+        for i in range(args.steps):
+            fn(i)
+        torch.cuda.synchronize()
+        return
+
     spec = wl.DECODE_D2K256
     if args.small:
         # same per-expert shapes with 64 experts (430 MB of weights): the case for full ncu captures
@@ -321,6 +328,14 @@ def run_ours(args):
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(mds, draws, spec, T, per_expert, cb_bytes)
 
+    extra = {}
+    if not args.no_extra:
+        extra["decode_T1"] = measure_decode_t1(torch, vq, layer, spec, per_expert, cb_bytes, dev, args.steps,
+                                               args.warmup)
+        del layer, mods
+        torch.cuda.empty_cache()
+        extra["prefill"] = measure_prefill(torch, vq, dev, min(args.steps, 20), args.warmup)
+
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -342,11 +357,100 @@ def run_ours(args):
         "gpu_launches": 5 * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
+        "extra": extra,
     }
     if rank == 0:
         print(json.dumps(out), flush=True)
     if ws > 1:
         torch.distributed.destroy_process_group()
+
+
+def _time_steps(torch, fn, steps):
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for i in range(steps):
+        fn(i)
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def _traced(torch, vq, fn, steps, n_events=6):
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_events)] for _ in range(steps)]
+    for i in range(steps):
+        vq.set_trace_events(evs[i])
+        fn(i)
+    vq.set_trace_events(None)
+    torch.cuda.synchronize()
+    return np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(n_events - 1)] for i in range(steps)])
+
+
+def measure_decode_t1(torch, vq, layer, spec, per_expert, cb_bytes, dev, steps, warmup):
+    """Same layer, one token per step (latency-bound case), 16 rotating routing draws."""
+    draws = [wl.layer_inputs(spec, 1, 100 + i) for i in range(N_DRAWS)]
+    xs = [torch.from_numpy(x.view(np.int16)).to(dev) for x, _ in draws]
+    lgs = [torch.from_numpy(lg).to(dev) for _, lg in draws]
+    y = torch.empty((1, spec.hidden), dtype=torch.float32, device=dev)
+    ws = layer.workspace(1, spec.top_k, vq.VQ_MODE_DECODE, dev)
+    nbytes = []
+    for lg in lgs:
+        _, _, off, _ = vq.route(lg, spec.top_k)
+        touched = np.nonzero(np.diff(off.cpu().numpy()) > 0)[0]
+        nbytes.append(sum(float(p[touched].sum()) for p in per_expert) + cb_bytes + spec.hidden * 6 + spec.E * 4)
+    fn = lambda i: layer.decode(xs[i % N_DRAWS], lgs[i % N_DRAWS], spec.top_k, out=y, workspace=ws)
+    for i in range(warmup):
+        fn(i)
+    ms = _time_steps(torch, fn, steps)
+    tot = sum(nbytes[i % N_DRAWS] for i in range(steps))
+    return {"workload": spec.name, "T": 1, "value": tot / (ms * 1e-3) / 1e9, "unit": UNIT, "ms_per_step": ms / steps,
+            "tokens_per_s": steps / (ms * 1e-3), "launches_per_step": 5}
+
+
+def measure_prefill(torch, vq, dev, steps, warmup, small=False, ncu_mode=False):
+    """MoE prefill layer, d=4/K=512, 4096 tokens, Zipf(1.1) routing: tcgen05 grouped GEMM path."""
+    import dataclasses
+    from tests.helpers import lib_module
+    spec = wl.PREFILL_D4K512
+    T = spec.batches[0]
+    if small:
+        spec = dataclasses.replace(spec, E=64, name=spec.name.replace("e256", "e64"))
+        T = 1024
+    mds = wl.layer_modules(spec, raw=False, row_words=lambda c, g: vq.packed_words(1, c // g.d, g.bits))
+    layer = vq.MoELayer(*[lib_module(m, device=dev) for m in mds])
+    draws = [wl.layer_inputs(spec, T, i) for i in range(2)]
+    xs = [torch.from_numpy(x.view(np.int16)).to(dev) for x, _ in draws]
+    lgs = [torch.from_numpy(lg).to(dev) for _, lg in draws]
+    y = torch.empty((T, spec.hidden), dtype=torch.float32, device=dev)
+    ws = layer.workspace(T, spec.top_k, vq.VQ_MODE_PREFILL, dev)
+    fn = lambda i: layer.prefill(xs[i % 2], lgs[i % 2], spec.top_k, out=y, workspace=ws)
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    pairs = T * spec.top_k
+    flops_gu = 2.0 * pairs * 2 * spec.inter * spec.hidden
+    flops_dn = 2.0 * pairs * spec.hidden * spec.inter
+    if ncu_mode:
+        return layer, fn
+    ms = _time_steps(torch, fn, steps)
+    stage = _traced(torch, vq, fn, steps).mean(axis=0)
+    _, tf_burst, tf_sust, src = _peaks()
+    gu_tflops = flops_gu / (stage[2] * 1e-3) / 1e12
+    out = {"workload": spec.name, "T": T, "metric": "prefill TFLOP/s", "unit": "TFLOP/s",
+           "value": (flops_gu + flops_dn) / (ms / steps * 1e-3) / 1e12, "ms_per_step": ms / steps,
+           "tokens_per_s": T * steps / (ms * 1e-3), "flops_per_step": flops_gu + flops_dn,
+           "stage_ms": {"route": float(stage[0]), "gather": float(stage[1]), "gate_up_gemm": float(stage[2]),
+                        "down_gemm": float(stage[3]), "combine": float(stage[4])},
+           "roofline": {"bound": "tensor", "achieved": gu_tflops, "peak": tf_burst, "unit": "TFLOP/s",
+                        "frac": gu_tflops / tf_burst, "traffic": _traffic_per_launch("prefill_gemm_gate_up"),
+                        "kernel": "vq_prefill_gemm_kernel<4,9> (gate+up, SwiGLU epilogue)",
+                        "peak_source": f"{src} bf16_tflops (fp16 runs at the bf16 rate)",
+                        "flops_per_launch": flops_gu, "ms_per_launch": float(stage[2])},
+           "launches_per_step": 7}
+    del layer
+    torch.cuda.empty_cache()
+    return out
 
 
 def cpu_baseline(mds, draws, spec, T, per_expert, cb_bytes, budget_s=10.0):
@@ -380,6 +484,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ncu", action="store_true", help="only warmup + timed steps, for profiler captures")
     ap.add_argument("--small", action="store_true", help="64-expert variant of the workload (profiling)")
+    ap.add_argument("--only", choices=("decode", "prefill"), default="decode",
+                    help="with --ncu: which path the profiler run exercises")
+    ap.add_argument("--no-extra", action="store_true", help="skip the 1-token decode and prefill lines")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -178,7 +178,7 @@ size_t vq_moe_workspace_size(const vq_moe_layer *L, int32_t T, int32_t top_k, in
  *   y[t] = sum_j w[t, j] * W_down,e_j ( silu(W_gate,e_j x[t]) * (W_up,e_j x[t]) )
  * with (e_j, w[t, j]) from vq_route on `logits` (device fp32 [T, E]).
  * x: device bf16 [T, hidden], 16-byte aligned. y: device [T, hidden] of
- * y_dtype. workspace: device, 256-byte aligned, at least
+ * y_dtype, 16-byte aligned. workspace: device, 256-byte aligned, at least
  * vq_moe_workspace_size(L, T, top_k, VQ_MODE_DECODE) bytes; it holds the
  * routing tables and the intermediate activations and may be reused by the
  * next call once this one has run. Sums over experts run in slot order j,

@@ -155,3 +155,22 @@ def test_moe_decode_full_size(spec, T, sample):
     assert_close(y.cpu().numpy()[tok], ref, what=f"{spec.name} T{T}")
     del layer
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("d,bits", GEOS)
+@pytest.mark.parametrize("T", [1, 9])
+def test_gemv_staged_path(d, bits, T):
+    # 1024 columns (16 groups) and 300 rows with skipzero: the TMA-staged kernel
+    # path (several 256-row items, a ragged last item, compacted live rows)
+    E, rows, cols = 3, 300, 1024
+    md = small_module(E, rows, cols, d, bits, n_dead=37, seed=11 * d + bits)
+    om, lm = oracle_module(md), lib_module(md)
+    x = synth.activations(T, cols, synth.rng(6, T))
+    xt = torch.from_numpy(x.view(np.int16)).cuda()
+    for e in range(E):
+        y = vq.gemv(lm, e, xt)
+        torch.cuda.synchronize()
+        got = y.cpu().numpy()
+        assert_close(got, oracle.gemv(om, e, x), what=f"staged gemv d{d} b{bits} T{T} e{e}")
+        dead = ~_live_mask(md, e)
+        assert np.all(got[:, dead] == 0)

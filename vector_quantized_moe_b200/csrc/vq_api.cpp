@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "vq_internal.h"
@@ -58,23 +60,18 @@ vq_status check_module(const vq_module *m)
     return VQ_OK;
 }
 
-vq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? VQ_OK : VQ_ERR_CUDA; }
-
-// Split of the 64-column groups so that enough warps have work.
-int choose_slices(long n_act_est, int rows, int ngroups, int nmod, long target_items)
+vq_status cuda_status(cudaError_t e)
 {
-    const long items1 = n_act_est * ((rows + 31) / 32) * nmod;
-    int s = 1;
-    while (ngroups % (2 * s) == 0 && ngroups / (2 * s) >= 2 && items1 * s < target_items)
-        s *= 2;
-    return s;
+    if (e != cudaSuccess && std::getenv("VQ_DEBUG"))
+        std::fprintf(stderr, "vq: CUDA error %d: %s\n", (int)e, cudaGetErrorString(e));
+    return e == cudaSuccess ? VQ_OK : VQ_ERR_CUDA;
 }
 
 struct DecodePlan {
     int T, k, E, H, I;
     int sa, sb;                  // slices of the gate/up and down passes
     RoutingLayout r;
-    size_t off_x16, off_G, off_U, off_h, off_D;
+    size_t off_err, off_x16, off_G, off_U, off_h, off_D;
     size_t total;
 };
 
@@ -93,8 +90,6 @@ vq_status check_layer(const vq_moe_layer *L)
     return VQ_OK;
 }
 
-long target_items() { return (long)num_sms() * 16 * 2; }
-
 DecodePlan plan_decode(const vq_moe_layer *L, int T, int k)
 {
     DecodePlan p{};
@@ -104,11 +99,16 @@ DecodePlan plan_decode(const vq_moe_layer *L, int T, int k)
     p.H = L->gate.cols;
     p.I = L->gate.rows;
     const long n_act = std::min<long>(p.E, (long)T * k);
-    p.sa = choose_slices(n_act, p.I, p.H / 64, 2, target_items());
-    p.sb = choose_slices(n_act, p.H, p.I / 64, 1, target_items());
+    const ModDev gu[2] = {make_moddev(L->gate), make_moddev(L->up)};
+    const ModDev dn = make_moddev(L->down);
+    const bool same = gu[0].d == gu[1].d && gu[0].bits == gu[1].bits && gu[0].rep == gu[1].rep;
+    p.sa = same ? gemv_choose_slices(gu, 2, n_act)
+                : std::min(gemv_choose_slices(&gu[0], 1, n_act), gemv_choose_slices(&gu[1], 1, n_act));
+    p.sb = gemv_choose_slices(&dn, 1, n_act);
     size_t o = 0;
     p.r = plan_routing(o, T, k, p.E);
     const size_t tk = (size_t)T * k;
+    p.off_err = o; o = align_up(o + 16, 256);
     p.off_x16 = o; o = align_up(o + (size_t)T * p.H * 2, 256);
     p.off_G = o; o = align_up(o + (size_t)p.sa * tk * p.I * 4, 256);
     p.off_U = o; o = align_up(o + (size_t)p.sa * tk * p.I * 4, 256);
@@ -328,6 +328,7 @@ vq_status vq_gemv(const vq_module *m, int32_t expert, const uint16_t *x, int32_t
     a.act = x;
     a.act_bf16 = 1;
     a.act_by_slot = 0;
+    a.act_rows = T;
     a.expert = expert;
     a.T = T;
     a.slices = 1;
@@ -335,10 +336,8 @@ vq_status vq_gemv(const vq_module *m, int32_t expert, const uint16_t *x, int32_t
     a.out[1] = y;
     a.out_dtype = y_dtype;
     a.out_slice_stride = 0;
-    const int occ = gemv_ctas_per_sm(m->d, m->bits, gemv_smem_bytes(a.mod[0]));
-    const long items = (long)((m->rows + 31) / 32);
-    const int ctas = (int)std::max<long>(1, std::min<long>((long)num_sms() * occ, (items + 7) / 8));
-    return cuda_status(launch_gemv(a, ctas, (cudaStream_t)stream, false));
+    a.err = nullptr;
+    return cuda_status(launch_gemv(a, (cudaStream_t)stream, false));
 }
 
 vq_status vq_route(const float *logits, int32_t T, int32_t E, int32_t top_k, int32_t renorm, int32_t *ids,
@@ -371,7 +370,7 @@ static vq_status check_moe_args(const vq_moe_layer *L, const uint16_t *x, int32_
     if (!x || !logits || !y || T < 0 || top_k < 1 || top_k > std::min(L->gate.E, 32) || L->gate.E > 4096 ||
         (y_dtype != VQ_F32 && y_dtype != VQ_BF16) || (long)T * top_k >= (1L << 31))
         return VQ_ERR_ARG;
-    if (!aligned(x, 16))
+    if (!aligned(x, 16) || !aligned(y, 16))
         return VQ_ERR_ALIGN;
     if (!workspace || !aligned(workspace, 256))
         return VQ_ERR_WORKSPACE;
@@ -397,6 +396,7 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     int32_t *pos = ws_at<int32_t>(workspace, p.r.pos);
     int32_t *active = ws_at<int32_t>(workspace, p.r.active);
     int32_t *nact = ws_at<int32_t>(workspace, p.r.nact);
+    int *errw = ws_at<int>(workspace, p.off_err);
     __half *x16 = ws_at<__half>(workspace, p.off_x16);
     float *G = ws_at<float>(workspace, p.off_G);
     float *U = ws_at<float>(workspace, p.off_U);
@@ -416,6 +416,7 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     a.act = x16;
     a.act_bf16 = 0;
     a.act_by_slot = 0;
+    a.act_rows = T;
     a.offsets = offsets;
     a.perm = perm;
     a.top_k = top_k;
@@ -424,27 +425,25 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     a.slices = p.sa;
     a.out_dtype = VQ_F32;
     a.out_slice_stride = tk * p.I;
+    a.err = errw;
     const ModDev mg = make_moddev(L->gate), mu = make_moddev(L->up);
     const bool same = mg.d == mu.d && mg.bits == mu.bits && mg.rep == mu.rep;
-    const int sms = num_sms();
     if (same) {
         a.mod[0] = mg;
         a.mod[1] = mu;
         a.nmod = 2;
         a.out[0] = G;
         a.out[1] = U;
-        const int occ = gemv_ctas_per_sm(mg.d, mg.bits, gemv_smem_bytes(mg));
-        const int per_y = gemv_both_modules_per_cta(mg.d, mg.bits) ? sms * occ : std::max(1, sms * occ / 2);
-        err = launch_gemv(a, per_y, s, true);
+        err = launch_gemv(a, s, true);
     } else {
         a.nmod = 1;
         a.mod[0] = a.mod[1] = mg;
         a.out[0] = a.out[1] = G;
-        err = launch_gemv(a, sms * gemv_ctas_per_sm(mg.d, mg.bits, gemv_smem_bytes(mg)), s, true);
+        err = launch_gemv(a, s, true);
         if (err == cudaSuccess) {
             a.mod[0] = a.mod[1] = mu;
             a.out[0] = a.out[1] = U;
-            err = launch_gemv(a, sms * gemv_ctas_per_sm(mu.d, mu.bits, gemv_smem_bytes(mu)), s, true);
+            err = launch_gemv(a, s, true);
         }
     }
     if (err != cudaSuccess)
@@ -463,10 +462,11 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     b.act = h;
     b.act_bf16 = 0;
     b.act_by_slot = 1;
+    b.act_rows = tk;
     b.slices = p.sb;
     b.out[0] = b.out[1] = D;
     b.out_slice_stride = tk * p.H;
-    err = launch_gemv(b, sms * gemv_ctas_per_sm(md.d, md.bits, gemv_smem_bytes(md)), s, true);
+    err = launch_gemv(b, s, true);
     if (err != cudaSuccess)
         return VQ_ERR_CUDA;
 

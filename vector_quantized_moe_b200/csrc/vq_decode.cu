@@ -21,6 +21,7 @@
 // fp32 scale is applied once per group to the partial sums.
 #include "vq_device.cuh"
 #include "vq_internal.h"
+#include "vq_sm100.cuh"
 
 namespace vq {
 namespace {
@@ -352,6 +353,379 @@ __global__ void __launch_bounds__(GEMV_THREADS, 2) vq_grouped_gemv_kernel(const 
     }
 }
 
+// ------------------------------------------------------------ TMA-fed grouped GEMV
+//
+// The same decomposition, with the packed codes streamed by TMA through a
+// ring of shared-memory stages instead of per-lane global loads. A CTA has 8
+// consumer warps (32 rows each, 256 rows per work item) and one producer
+// warp whose lane 0 issues one 2D tensor load per stage: 256 rows x CG
+// groups of codes. Consumers read their lane-quarters from shared memory.
+// For d=2/8-bit codes a stage row is 128 bytes loaded with the 128-byte
+// swizzle, and m16 row g of a warp is weight row sigma(g) (even rows in the
+// first half-warp, odd rows in the second), so a warp's 8-byte code reads hit
+// distinct banks. Each wait on a stage barrier is bounded.
+
+constexpr int TG_CONSUMERS = 8;
+constexpr int TG_THREADS = 32 * (TG_CONSUMERS + 1);
+constexpr int TG_ROWS = 32 * TG_CONSUMERS;
+constexpr int TG_NT = 1;   // token tiles of 8 per pass (the kernel body assumes one)
+
+__host__ __device__ constexpr int tg_stage_groups(int d, int bits)
+{
+    if (d == 2 && bits == 8)
+        return 4;
+    const int gb = (64 / d) * bits;   // bits of one row per group
+    int cg = 1;
+    while ((cg * gb) % 128)
+        ++cg;
+    return cg;
+}
+
+template <int D, int BITS>
+struct TGeo {
+    static constexpr bool SWZ = (D == 2 && BITS == 8);
+    static constexpr int CG = tg_stage_groups(D, BITS);
+    static constexpr int GB = (64 / D) * BITS;      // bits per row per group
+    static constexpr int SRB = CG * GB / 8;         // bytes per row per stage
+    static constexpr int ACOLS = CG * 64;           // activation columns per stage
+    static constexpr int ACW = ACOLS < 256 ? ACOLS : 256;   // columns per activation box
+};
+
+struct GemvTmaArgs {
+    CUtensorMap tmap[2];      // codes: u32 [live rows, row_words], box {SRB/4, 256}
+    CUtensorMap tmap_sc[2];   // scales: fp16 [live rows, ngroups], box {8, 256}
+    CUtensorMap tmap_act;     // activations: 16-bit [act rows, cols], box {ACW, 1}
+    GemvArgs g;
+    int ns;
+    uint32_t stage_bytes, off_sc, off_act;   // stage layout: codes | scales | activations
+    uint32_t off_stage, off_bar;
+    int *err;
+};
+
+__device__ __forceinline__ int tg_sigma(int g) { return g < 4 ? 2 * g : 2 * (g - 4) + 1; }
+
+__device__ __forceinline__ int tg_prow0(const ModDev &m, int e, int r0)
+{
+    if (!m.bitmap)
+        return e * m.rows + r0;
+    return (int)m.rank[(long)e * m.bm_words + (r0 >> 5)];
+}
+
+template <int D, int BITS>
+__device__ __forceinline__ void tg_read_quarter(const uint8_t *row, int gq, int t, int br,
+                                                uint32_t (&w)[Geo<D, BITS>::LW], int &o)
+{
+    using G = Geo<D, BITS>;
+    using TG = TGeo<D, BITS>;
+    if constexpr (TG::SWZ) {
+        const int c = 2 * gq + (t >> 1);
+        const uint2 v = *reinterpret_cast<const uint2 *>(row + (((c ^ (br & 7)) << 4) | ((t & 1) << 3)));
+        w[0] = v.x;
+        w[1] = v.y;
+        o = 0;
+    } else {
+        const int off = (4 * gq + t) * G::QB;
+        const uint32_t *p = reinterpret_cast<const uint32_t *>(row) + (off >> 5);
+        o = off & 31;
+        if constexpr (G::ALIGNED) {
+#pragma unroll
+            for (int i = 0; i < G::LW; ++i)
+                w[i] = p[i];
+        } else {
+            const int need = (o + G::QB + 31) >> 5;
+#pragma unroll
+            for (int i = 0; i < G::LW; ++i)
+                w[i] = i < need ? p[i] : 0u;
+        }
+    }
+}
+
+template <int D, int BITS>
+__global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid_constant__ GemvTmaArgs A)
+{
+    using G = Geo<D, BITS>;
+    using TG = TGeo<D, BITS>;
+    constexpr bool FAST = FastByteCodes<D, BITS>::value;
+    const GemvArgs &a = A.g;
+    extern __shared__ __align__(1024) uint8_t tg_smem_raw[];
+    uint8_t *smem = tg_smem_raw;
+    if (smem_u32(smem) & 1023u) {   // the 128-byte swizzle needs 1024-byte aligned stages
+        if (threadIdx.x == 0 && A.err)
+            atomicExch(A.err, 19);
+        return;
+    }
+    uint32_t *cbs = reinterpret_cast<uint32_t *>(smem);
+    uint8_t *stages = smem + A.off_stage;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + A.off_bar);
+    uint64_t *empty = full + A.ns;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + A.ns);
+
+    const int cta_mods = FAST ? a.nmod : 1;
+    if constexpr (FAST)
+        fill_codebook_lines<D, BITS>(cbs, a.mod[0].codebook, a.mod[1].codebook, a.nmod);
+    else
+        fill_codebook<D, BITS>(cbs, (blockIdx.y == 0 ? a.mod[0] : a.mod[1]).codebook,
+                               (blockIdx.y == 0 ? a.mod[0] : a.mod[1]).log_rep);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < A.ns; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], TG_CONSUMERS);
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    grid_dep_wait();
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const ModDev m0 = FAST ? a.mod[0] : (blockIdx.y == 0 ? a.mod[0] : a.mod[1]);
+    const int n_act = a.offsets ? *a.n_active : 1;
+    const int nrb = (m0.rows + TG_ROWS - 1) / TG_ROWS;
+    const int S = a.slices;
+    const int gps = m0.ngroups / S;
+    const int spp = gps / TG::CG;
+    const long n_items = (long)n_act * nrb * S * cta_mods;
+    const uint32_t stage_bytes_codes = (uint32_t)TG_ROWS * TG::SRB;
+
+    auto decode_item = [&](long it, int &slice, int &rb, int &mi, int &e, int &q0, int &n) {
+        long rest = it;
+        slice = (int)(rest % S);
+        rest /= S;
+        rb = (int)(rest % nrb);
+        rest /= nrb;
+        mi = FAST ? (int)(rest % cta_mods) : (int)blockIdx.y;
+        const int ai = FAST ? (int)(rest / cta_mods) : (int)rest;
+        e = a.offsets ? a.active[ai] : a.expert;
+        q0 = a.offsets ? a.offsets[e] : 0;
+        n = a.offsets ? a.offsets[e + 1] - q0 : a.T;
+    };
+
+    if (warp == TG_CONSUMERS) {
+        // ------------------------------------------------ producer: codes, scales and the
+        // activation rows of the pass's tokens for every stage, one barrier per stage
+        if (lane == 0) {
+            uint32_t k = 0, slot = 0, ph = 0;   // stages issued; ring slot and phase of stage k
+            bool ok = true;
+            for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+                int slice, rb, mi, e, q0, n;
+                decode_item(it, slice, rb, mi, e, q0, n);
+                const ModDev &m = mi == 0 ? a.mod[0] : a.mod[1];
+                const int prow0 = tg_prow0(m, e, rb * TG_ROWS);
+                const int passes = (n + 8 * TG_NT - 1) / (8 * TG_NT);
+                for (int p = 0; p < passes && ok; ++p) {
+                    const int tok0 = p * 8 * TG_NT;
+                    const int np = min(8 * TG_NT, n - tok0);
+                    int arow[8 * TG_NT];
+                    for (int i = 0; i < np; ++i) {
+                        const int q = q0 + tok0 + i;
+                        arow[i] = a.act_by_slot ? q : (a.perm ? a.perm[q] / a.top_k : tok0 + i);
+                    }
+                    const uint32_t tx = stage_bytes_codes + (uint32_t)TG_ROWS * 16 + (uint32_t)np * TG::ACOLS * 2;
+                    for (int j = 0; j < spp; ++j) {
+                        if (!(ok = mbar_wait(&empty[slot], ph ^ 1, abort_flag, A.err, 11)))
+                            break;
+                        uint8_t *sb = stages + (size_t)slot * A.stage_bytes;
+                        mbar_expect_tx(&full[slot], tx);
+                        const int g0 = slice * gps + j * TG::CG;
+                        tma_load_2d(sb, &A.tmap[mi], g0 * TG::GB / 32, prow0, &full[slot]);
+                        tma_load_2d(sb + A.off_sc, &A.tmap_sc[mi], g0 & ~7, prow0, &full[slot]);
+                        for (int i = 0; i < np; ++i)
+                            for (int c = 0; c < TG::ACOLS; c += TG::ACW)
+                                tma_load_2d(sb + A.off_act + (size_t)i * TG::ACOLS * 2 + c * 2, &A.tmap_act,
+                                            g0 * 64 + c, arow[i], &full[slot]);
+                        ++k;
+                        if (++slot == (uint32_t)A.ns) {
+                            slot = 0;
+                            ph ^= 1;
+                        }
+                    }
+                }
+            }
+            if (!ok) {
+                for (uint32_t s = 0; s < (uint32_t)A.ns && s < k; ++s) {
+                    const uint32_t kk = k - 1 - s;
+                    mbar_wait(&full[kk % A.ns], (kk / A.ns) & 1, abort_flag, A.err, 12);
+                }
+            }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------- consumers
+    const int g = lane >> 2, t = lane & 3;
+    uint32_t slot = 0, ph = 0;
+    bool ok = true;
+    for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        int slice, rb, mi, e, q0, n;
+        decode_item(it, slice, rb, mi, e, q0, n);
+        const ModDev &m = mi == 0 ? a.mod[0] : a.mod[1];
+        void *const out = mi == 0 ? a.out[0] : a.out[1];
+        const int rep = lane & (m.rep - 1);
+        const uint32_t lane_sel = (uint32_t)(mi * 128 + lane * 4);
+        const int r0 = rb * TG_ROWS;
+        const int prow0 = tg_prow0(m, e, r0);
+        int br[4], prow[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = r0 + 32 * warp + 8 * i + tg_sigma(g);
+            prow[i] = r < m.rows ? (int)live_row(m.bitmap, m.rank, m.bm_words, m.rows, e, r) : -1;
+            br[i] = prow[i] >= 0 ? prow[i] - prow0 : -1;
+        }
+        const int passes = (n + 8 * TG_NT - 1) / (8 * TG_NT);
+        for (int p = 0; p < passes && ok; ++p) {
+            const int tok0 = p * 8 * TG_NT;
+            const int ntiles = min(TG_NT, (n - tok0 + 7) / 8);
+            bool has_tok[TG_NT];
+#pragma unroll
+            for (int nt = 0; nt < TG_NT; ++nt)
+                has_tok[nt] = nt < ntiles && tok0 + 8 * nt + g < n;
+            float acc[TG_NT][2][4];
+#pragma unroll
+            for (int nt = 0; nt < TG_NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        acc[nt][i][j] = 0.f;
+
+            for (int j = 0; j < spp; ++j) {
+                const int g0 = slice * gps + j * TG::CG;
+                if (!(ok = mbar_wait(&full[slot], ph, abort_flag, A.err, 13)))
+                    break;
+                const uint8_t *sbase = stages + (size_t)slot * A.stage_bytes;
+                const uint16_t *ssc = reinterpret_cast<const uint16_t *>(sbase + A.off_sc) + (g0 & 7);
+                const uint8_t *sact = sbase + A.off_act;
+                // groups are taken GP at a time so that a warp has 2 * GP independent
+                // accumulation chains in flight
+                constexpr int GP = TG::CG >= 2 ? 2 : 1;
+#pragma unroll
+                for (int gp = 0; gp < TG::CG; gp += GP) {
+                    uint32_t cw[GP][4][G::LW];
+                    int co[GP][4];
+                    uint32_t bw[GP][8];
+                    float sv[GP][4];
+#pragma unroll
+                    for (int u = 0; u < GP; ++u) {
+                        const int gq = gp + u;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            if (br[i] >= 0) {
+                                tg_read_quarter<D, BITS>(sbase + (size_t)br[i] * TG::SRB, gq, t, br[i], cw[u][i],
+                                                         co[u][i]);
+                                sv[u][i] = f16_to_f32(ssc[(size_t)br[i] * 8 + gq]);
+                            } else {
+#pragma unroll
+                                for (int q = 0; q < G::LW; ++q)
+                                    cw[u][i][q] = 0u;
+                                co[u][i] = 0;
+                                sv[u][i] = 0.f;
+                            }
+                        }
+                        uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+                        if (has_tok[0]) {
+                            const uint4 *ap =
+                                reinterpret_cast<const uint4 *>(sact + (size_t)g * TG::ACOLS * 2 + gq * 128 + t * 32);
+                            v0 = ap[0];
+                            v1 = ap[1];
+                        }
+                        bw[u][0] = v0.x; bw[u][1] = v0.y; bw[u][2] = v0.z; bw[u][3] = v0.w;
+                        bw[u][4] = v1.x; bw[u][5] = v1.y; bw[u][6] = v1.z; bw[u][7] = v1.w;
+                        if (a.act_bf16) {
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                bw[u][q] = bf16x2_to_f16x2(bw[u][q]);
+                        }
+                    }
+                    if (gp + GP >= TG::CG) {   // every code read of this stage is done
+                        __syncwarp();
+                        if (lane == 0)
+                            mbar_arrive(&empty[slot]);
+                    }
+                    uint32_t c[GP][4][G::CODES];
+                    if constexpr (!FAST) {
+#pragma unroll
+                        for (int u = 0; u < GP; ++u)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i)
+                                extract_codes<D, BITS>(cw[u][i], co[u][i], c[u][i]);
+                    }
+                    float tmp[GP][2][4];
+#pragma unroll
+                    for (int u = 0; u < GP; ++u)
+#pragma unroll
+                        for (int i = 0; i < 2; ++i)
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                tmp[u][i][q] = 0.f;
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) {
+#pragma unroll
+                        for (int u = 0; u < GP; ++u) {
+#pragma unroll
+                            for (int rt = 0; rt < 2; ++rt) {
+                                uint32_t Aw[4];
+                                if constexpr (FAST) {
+                                    const char *cbb = reinterpret_cast<const char *>(cbs);
+#pragma unroll
+                                    for (int h = 0; h < 2; ++h) {
+                                        const uint32_t sel = 0x5504u | ((uint32_t)(2 * (s & 1) + h) << 4);
+                                        Aw[2 * h] = *reinterpret_cast<const uint32_t *>(
+                                            cbb + __byte_perm(cw[u][2 * rt][s >> 1], lane_sel, sel));
+                                        Aw[2 * h + 1] = *reinterpret_cast<const uint32_t *>(
+                                            cbb + __byte_perm(cw[u][2 * rt + 1][s >> 1], lane_sel, sel));
+                                    }
+                                } else {
+                                    a_words<D>(cbs, m.log_rep, rep, c[u][2 * rt], s, Aw[0], Aw[2]);
+                                    a_words<D>(cbs, m.log_rep, rep, c[u][2 * rt + 1], s, Aw[1], Aw[3]);
+                                }
+                                if (ntiles > 0)
+                                    mma_16816(tmp[u][rt], Aw, bw[u][2 * s], bw[u][2 * s + 1]);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < GP; ++u)
+#pragma unroll
+                        for (int rt = 0; rt < 2; ++rt) {
+                            const float slo = sv[u][2 * rt], shi = sv[u][2 * rt + 1];
+                            acc[0][rt][0] = fmaf(tmp[u][rt][0], slo, acc[0][rt][0]);
+                            acc[0][rt][1] = fmaf(tmp[u][rt][1], slo, acc[0][rt][1]);
+                            acc[0][rt][2] = fmaf(tmp[u][rt][2], shi, acc[0][rt][2]);
+                            acc[0][rt][3] = fmaf(tmp[u][rt][3], shi, acc[0][rt][3]);
+                        }
+                }
+                if (++slot == (uint32_t)A.ns) {
+                    slot = 0;
+                    ph ^= 1;
+                }
+            }
+            if (!ok)
+                break;
+            // lane holds rows sigma(g) (+8i) for bucket tokens tok0 + 8nt + 2t + {0, 1}
+#pragma unroll
+            for (int nt = 0; nt < TG_NT; ++nt)
+#pragma unroll
+                for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const int i = 2 * rt + hf;
+                        const int r = r0 + 32 * warp + 8 * i + tg_sigma(g);
+                        if (r >= m.rows)
+                            continue;
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc) {
+                            const int tk = tok0 + 8 * nt + 2 * t + cc;
+                            if (nt >= ntiles || tk >= n)
+                                continue;
+                            const float v = prow[i] >= 0 ? acc[nt][rt][2 * hf + cc] : 0.f;
+                            store_out(out, a.out_dtype,
+                                      (long)slice * a.out_slice_stride + (long)(q0 + tk) * m.rows + r, v);
+                        }
+                    }
+        }
+    }
+}
+
 // ------------------------------------------------------------ SwiGLU and combine
 
 __global__ void vq_swiglu_kernel(const float *__restrict__ G, const float *__restrict__ U, int slices, long slice_stride,
@@ -369,22 +743,49 @@ __global__ void vq_swiglu_kernel(const float *__restrict__ G, const float *__res
     }
 }
 
-__global__ void vq_combine_kernel(const float *__restrict__ D, int slices, long slice_stride, const float *__restrict__ w,
-                                  const int32_t *__restrict__ pos, int T, int k, int hidden, void *y, int y_dtype)
+// y[t, :] = sum_j w[t, j] * sum_s D[s, pos[t*k + j], :], slots in order j, one
+// block per token, four columns per thread.
+__global__ void __launch_bounds__(256) vq_combine_kernel(const float *__restrict__ D, int slices, long slice_stride,
+                                                         const float *__restrict__ w, const int32_t *__restrict__ pos,
+                                                         int T, int k, int hidden, void *y, int y_dtype)
 {
+    __shared__ long q_s[32];
+    __shared__ float w_s[32];
     grid_dep_wait();
-    const long n = (long)T * hidden;
-    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
-        const int tok = (int)(i / hidden), r = (int)(i % hidden);
-        float acc = 0.f;
-        for (int j = 0; j < k; ++j) {
-            const long q = pos[(long)tok * k + j];
-            float part = 0.f;
-            for (int s = 0; s < slices; ++s)
-                part += D[s * slice_stride + q * hidden + r];
-            acc = fmaf(w[(long)tok * k + j], part, acc);
+    const int h4 = hidden >> 2;
+    for (int tok = blockIdx.x; tok < T; tok += gridDim.x) {
+        __syncthreads();   // q_s / w_s of the previous token are no longer read
+        if (threadIdx.x < k) {
+            q_s[threadIdx.x] = (long)pos[(long)tok * k + threadIdx.x] * hidden;
+            w_s[threadIdx.x] = w[(long)tok * k + threadIdx.x];
         }
-        store_out(y, y_dtype, i, acc);
+        __syncthreads();
+        for (int c4 = blockIdx.y * blockDim.x + threadIdx.x; c4 < h4; c4 += gridDim.y * blockDim.x) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int j = 0; j < k; ++j) {
+                float4 part = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int s = 0; s < slices; ++s) {
+                    const float4 v = reinterpret_cast<const float4 *>(D + s * slice_stride + q_s[j])[c4];
+                    part.x += v.x;
+                    part.y += v.y;
+                    part.z += v.z;
+                    part.w += v.w;
+                }
+                const float wj = w_s[j];
+                acc.x = fmaf(wj, part.x, acc.x);
+                acc.y = fmaf(wj, part.y, acc.y);
+                acc.z = fmaf(wj, part.z, acc.z);
+                acc.w = fmaf(wj, part.w, acc.w);
+            }
+            const long o = (long)tok * hidden + 4 * c4;
+            if (y_dtype == VQ_F32) {
+                *reinterpret_cast<float4 *>(reinterpret_cast<float *>(y) + o) = acc;
+            } else {
+                const uint2 b = make_uint2((uint32_t)f32_to_bf16_bits(acc.x) | ((uint32_t)f32_to_bf16_bits(acc.y) << 16),
+                                           (uint32_t)f32_to_bf16_bits(acc.z) | ((uint32_t)f32_to_bf16_bits(acc.w) << 16));
+                *reinterpret_cast<uint2 *>(reinterpret_cast<uint16_t *>(y) + o) = b;
+            }
+        }
     }
 }
 
@@ -451,7 +852,7 @@ cudaError_t launch(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t s,
 }
 
 template <int D, int BITS>
-cudaError_t gemv_dispatch(const GemvArgs &a, int ctas, size_t smem, cudaStream_t s, bool pdl)
+cudaError_t gemv_dispatch(const GemvArgs &a, cudaStream_t s, bool pdl)
 {
     auto k = vq_grouped_gemv_kernel<D, BITS, GEMV_PD>;
     static bool attr_set = false;
@@ -461,19 +862,87 @@ cudaError_t gemv_dispatch(const GemvArgs &a, int ctas, size_t smem, cudaStream_t
             return err;
         attr_set = true;
     }
-    const int gy = FastByteCodes<D, BITS>::value ? 1 : a.nmod;
+    const size_t smem = gemv_smem_bytes(a.mod[0]);
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, GEMV_THREADS, smem) != cudaSuccess || occ < 1)
+        occ = 1;
+    const bool both = FastByteCodes<D, BITS>::value;
+    const int gy = both ? 1 : a.nmod;
+    const int ctas = std::max(1, num_sms() * occ / gy);
     return launch(k, dim3(ctas, gy), dim3(GEMV_THREADS), smem, s, pdl, a);
 }
 
-template <int D, int BITS>
-int gemv_occupancy(size_t smem)
+struct TgPlan {
+    int ns;
+    uint32_t stage, off_sc, off_act, off_stage, off_bar, total;
+};
+
+TgPlan tg_plan(const ModDev &m)
 {
-    auto k = vq_grouped_gemv_kernel<D, BITS, GEMV_PD>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, GEMV_THREADS, smem) != cudaSuccess)
-        return 1;
-    return n > 0 ? n : 1;
+    TgPlan p{};
+    const uint32_t cb = (uint32_t)align_up(gemv_smem_bytes(m), 1024);
+    const int cg = tg_stage_groups(m.d, m.bits);
+    const uint32_t codes = (uint32_t)TG_ROWS * (uint32_t)(cg * (64 / m.d) * m.bits / 8);
+    p.off_sc = codes;
+    p.off_act = codes + (uint32_t)TG_ROWS * 16;
+    p.stage = (uint32_t)align_up(p.off_act + 8u * TG_NT * cg * 64 * 2, 1024);
+    const uint32_t limit = 227 * 1024 - 1024 - 256;
+    p.ns = limit > cb ? (int)std::min<uint32_t>(8, (limit - cb) / p.stage) : 0;
+    p.off_stage = cb;
+    p.off_bar = cb + p.ns * p.stage;
+    p.total = p.off_bar + 16 * p.ns + 16 + 1024;
+    return p;
+}
+
+bool tg_ok(const ModDev &m, int slices)
+{
+    const int cg = tg_stage_groups(m.d, m.bits);
+    return tma_available() && m.row_words % 4 == 0 && m.ngroups % 8 == 0 && m.ngroups % slices == 0 &&
+           (m.ngroups / slices) % cg == 0 && tg_plan(m).ns >= 2;
+}
+
+template <int D, int BITS>
+cudaError_t gemv_tma_dispatch(const GemvArgs &a, cudaStream_t s, bool pdl)
+{
+    using TG = TGeo<D, BITS>;
+    GemvTmaArgs A{};
+    A.g = a;
+    for (int i = 0; i < a.nmod; ++i) {
+        const ModDev &m = a.mod[i];
+        if (!tma_map_2d(&A.tmap[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, m.codes, (uint64_t)m.row_words,
+                        (uint64_t)m.live_rows, (uint32_t)(TG::SRB / 4), (uint32_t)TG_ROWS,
+                        TG::SWZ ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+    }
+    for (int i = 0; i < a.nmod; ++i) {
+        const ModDev &m = a.mod[i];
+        if (!tma_map_2d(&A.tmap_sc[i], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, m.scales, (uint64_t)m.ngroups,
+                        (uint64_t)m.live_rows, 8, (uint32_t)TG_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+    }
+    if (!tma_map_2d(&A.tmap_act, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.act, (uint64_t)a.mod[0].cols,
+                    (uint64_t)a.act_rows, (uint32_t)TG::ACW, 1, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    if (a.nmod == 1) {
+        A.tmap[1] = A.tmap[0];
+        A.tmap_sc[1] = A.tmap_sc[0];
+    }
+    const TgPlan p = tg_plan(a.mod[0]);
+    A.ns = p.ns;
+    A.stage_bytes = p.stage;
+    A.off_sc = p.off_sc;
+    A.off_act = p.off_act;
+    A.off_stage = p.off_stage;
+    A.off_bar = p.off_bar;
+    A.err = a.err;
+    auto k = vq_gemv_tma_kernel<D, BITS>;
+    cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.total);
+    if (err != cudaSuccess)
+        return err;
+    const bool both = FastByteCodes<D, BITS>::value;
+    const int gy = both ? 1 : a.nmod;
+    const int ctas = std::max(1, num_sms() / gy);
+    return launch(k, dim3(ctas, gy), dim3(TG_THREADS), p.total, s, pdl, A);
 }
 
 }  // namespace
@@ -486,23 +955,33 @@ size_t gemv_smem_bytes(const ModDev &m)
     return ((size_t)1 << m.bits) * (size_t)m.rep * ew * 4;
 }
 
-bool gemv_both_modules_per_cta(int d, int bits) { return d == 2 && bits == 8; }
-
-int gemv_ctas_per_sm(int d, int bits, size_t smem)
+int gemv_choose_slices(const ModDev *mods, int nmod, long n_act)
 {
-#define VQ_OCC(D_, B_) \
-    if (d == D_ && bits == B_) return gemv_occupancy<D_, B_>(smem);
-    VQ_GEOMETRIES(VQ_OCC)
-#undef VQ_OCC
-    return 1;
+    const ModDev &m = mods[0];
+    bool tma = tg_ok(m, 1);
+    for (int i = 1; i < nmod; ++i)
+        tma = tma && tg_ok(mods[i], 1);
+    const int cg = tma ? tg_stage_groups(m.d, m.bits) : 1;
+    // work items: 256-row CTA items (TMA kernel) or 32-row warp items
+    const long per = tma ? (long)((m.rows + TG_ROWS - 1) / TG_ROWS) : (long)((m.rows + 31) / 32);
+    const long target = tma ? 2L * num_sms() : 32L * num_sms();
+    const long items1 = n_act * per * nmod;
+    int s = 1;
+    while (m.ngroups % (2 * s) == 0 && (m.ngroups / (2 * s)) % cg == 0 && m.ngroups / (2 * s) >= 2 * cg &&
+           items1 * s < target)
+        s *= 2;
+    return s;
 }
 
-cudaError_t launch_gemv(const GemvArgs &a, int ctas_per_mod, cudaStream_t s, bool pdl)
+cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, bool pdl)
 {
     const ModDev &m = a.mod[0];
-    const size_t smem = gemv_smem_bytes(m);
-#define VQ_GEMV(D_, B_) \
-    if (m.d == D_ && m.bits == B_) return gemv_dispatch<D_, B_>(a, ctas_per_mod, smem, s, pdl);
+    bool tma = tg_ok(m, a.slices);
+    for (int i = 1; i < a.nmod; ++i)
+        tma = tma && tg_ok(a.mod[i], a.slices);
+#define VQ_GEMV(D_, B_)                                                        \
+    if (m.d == D_ && m.bits == B_)                                             \
+        return tma ? gemv_tma_dispatch<D_, B_>(a, s, pdl) : gemv_dispatch<D_, B_>(a, s, pdl);
     VQ_GEOMETRIES(VQ_GEMV)
 #undef VQ_GEMV
     return cudaErrorInvalidValue;
@@ -519,10 +998,14 @@ cudaError_t launch_swiglu(const float *G, const float *U, int slices, long slice
 cudaError_t launch_combine(const float *D, int slices, long slice_stride, const float *w, const int32_t *pos, int T, int k,
                            int hidden, void *y, int y_dtype, cudaStream_t s, bool pdl)
 {
-    const long n = (long)T * hidden;
-    const int blocks = (int)((n + 255) / 256 < 8192 ? (n + 255) / 256 : 8192);
-    return launch(vq_combine_kernel, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, s, pdl, D, slices, slice_stride, w, pos,
-                  T, k, hidden, y, y_dtype);
+    const int blocks = T < 8192 ? (T > 0 ? T : 1) : 8192;
+    // few tokens: spread each token's columns over several blocks
+    const int h4 = hidden / 4;
+    int ysplit = 1;
+    while (blocks * ysplit < 2 * num_sms() && ysplit * 256 < h4)
+        ysplit *= 2;
+    return launch(vq_combine_kernel, dim3(blocks, ysplit), dim3(256), 0, s, pdl, D, slices, slice_stride, w, pos, T, k,
+                  hidden, y, y_dtype);
 }
 
 cudaError_t launch_unpack(const ModDev &m, int expert, uint16_t *out, cudaStream_t s)

@@ -1,6 +1,7 @@
 // Internal interface between the C ABI (vq_api.cpp) and the kernel launchers.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -40,6 +41,7 @@ struct GemvArgs {
     const void *act;        // activation rows: fp16 (or bf16 when act_bf16) [tokens or slots, cols]
     int act_bf16;
     int act_by_slot;        // 1: activation row = bucket slot q; 0: token (perm[q] / top_k, or t)
+    long act_rows;          // rows of the activation array
     const int32_t *offsets; // [E + 1] bucket offsets; NULL -> single expert over T tokens
     const int32_t *perm;    // [T*k] pair ids in bucket order (bf16 act: token = perm[q] / top_k)
     int top_k;
@@ -51,11 +53,15 @@ struct GemvArgs {
     void *out[2];           // per module: [slices][slots][rows]
     int out_dtype;          // VQ_F32 or VQ_BF16
     long out_slice_stride;  // elements between slices
+    int *err;               // device error word for bounded waits (may be NULL)
 };
 
-cudaError_t launch_gemv(const GemvArgs &a, int ctas_per_mod, cudaStream_t s, bool pdl);
-int gemv_ctas_per_sm(int d, int bits, size_t smem);
-bool gemv_both_modules_per_cta(int d, int bits);
+// Launches the TMA-fed kernel when the modules allow it (16-byte packed rows,
+// whole stages per slice), else the register-prefetch kernel.
+cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, bool pdl);
+// Slices of the 64-column groups for nmod modules sharing a launch and about
+// n_act experts with tokens (consistent with the kernel launch_gemv picks).
+int gemv_choose_slices(const ModDev *mods, int nmod, long n_act);
 size_t gemv_smem_bytes(const ModDev &m);
 
 // Routing + bucketing. pos = inverse of perm; active/n_active as above (may be NULL).
@@ -76,6 +82,11 @@ cudaError_t launch_unpack(const ModDev &m, int expert, uint16_t *out, cudaStream
 cudaError_t launch_dequant(const ModDev &m, int expert, float *out, cudaStream_t s);
 
 int num_sms();
+
+// 2D tiled TMA tensor map over a row-major [outer, inner] array (vq_tma.cpp).
+bool tma_available();
+bool tma_map_2d(CUtensorMap *map, CUtensorMapDataType dtype, int elem_bytes, const void *base, uint64_t inner,
+                uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 

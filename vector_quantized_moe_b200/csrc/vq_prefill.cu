@@ -14,10 +14,11 @@
 //   warp 0     TMA: activation tiles (fp16, 128B-swizzled, one 64-column
 //              k-step per stage) and packed-code tiles (a chunk of CH k-steps)
 //   warp 1     owns the tensor memory; one thread issues tcgen05.mma
-//   warps 2-5  thread i decodes row i of the weight tile for each k-step
-//              (unpack, codebook lookup, x fp16 scale) into the swizzled
-//              K-major shared-memory layout the tensor core reads, then runs
-//              the epilogue from tensor memory (lane i = row i)
+//   warps 2-9  two warpgroups taking alternate k-steps: thread i of a
+//              warpgroup decodes row i of the weight tile (unpack, codebook
+//              lookup, x fp16 scale) into the swizzled K-major shared-memory
+//              layout the tensor core reads; both then run the epilogue from
+//              tensor memory (lane i = row i), on alternate 32-column blocks
 // D[row, token] = sum_k W[row, k] X[token, k]: the weight tile is the
 // M=128 operand, the tokens of the bucket the N operand (16..128), so small
 // buckets waste no M rows. Every mbarrier wait is bounded; on a timeout the
@@ -30,14 +31,14 @@
 
 #include "vq_device.cuh"
 #include "vq_internal.h"
+#include "vq_sm100.cuh"
 
 namespace vq {
 namespace {
 
 constexpr int BM = 128;             // weight rows per tile = TMEM lanes
 constexpr int BN = 128;             // tokens per tile
-constexpr int NTHREADS = 192;       // 6 warps
-constexpr uint32_t WAIT_LIMIT = 1u << 22;
+constexpr int NTHREADS = 320;       // 10 warps: TMA, MMA, 8 dequant/epilogue
 constexpr int A_TILE = BM * 128;    // bytes of one 128 x 64 fp16 tile
 constexpr int B_TILE = BN * 128;
 
@@ -49,17 +50,32 @@ __host__ __device__ constexpr int chunk_steps(int kb)
     return ch;
 }
 
+// codebook replicas in shared memory (log2): as many as fit 32 KB for two
+// modules, at most 16
+__host__ __device__ constexpr int prefill_log_rep(int d, int bits)
+{
+    int lr = 0;
+    while (lr < 4 && 2L * (1L << bits) * d * 2 * (2L << lr) <= 32768)
+        ++lr;
+    return lr;
+}
+
+__host__ __device__ constexpr int log2i(int v) { return v <= 1 ? 0 : 1 + log2i(v / 2); }
+
 template <int D, int BITS>
 struct PG {
     static constexpr int KB = (64 / D) * BITS;       // code bits of one row per 64-column step
     static constexpr int CH = chunk_steps(KB);       // steps per code chunk (whole 16-byte units)
     static constexpr int CHW = CH * KB / 32;         // words per row per chunk
     static constexpr uint32_t MASK = (1u << BITS) - 1u;
+    static constexpr int LREP = prefill_log_rep(D, BITS);
+    static constexpr int L = LREP + 1 + log2i(D);    // code -> byte offset of its replica row
 };
 
 struct PrefillArgs {
     CUtensorMap tmap_b;       // activations fp16 [slots, K], box {64, BN}, 128B swizzle
     CUtensorMap tmap_c[2];    // packed codes u32 [live rows, row_words], box {CHW, BM}
+    CUtensorMap tmap_s[2];    // scales fp16 [live rows, ngroups], box {8, BM}
     ModDev mod[2];
     int nmod;
     const int32_t *offsets;
@@ -69,117 +85,11 @@ struct PrefillArgs {
     int rows;                 // weight rows (M)
     int sa, sc;               // operand stages, code stages
     uint32_t off_a, off_b, off_c, off_cb, off_tiles, off_bar;
+    int scale_tma;            // scales staged by TMA with the code chunks (else read per thread)
     void *out;                // SwiGLU: fp16 [slots, rows]; else fp32 [slots, rows]
     int swiglu;
     int *err;
 };
-
-// ------------------------------------------------------------------ PTX
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait on a phase; false when it gave up (limit reached or the CTA aborted).
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *err,
-                                          int code)
-{
-    for (uint32_t i = 0; i < WAIT_LIMIT; ++i) {
-        if (mbar_try_wait(bar, parity))
-            return true;
-        if ((i & 63) == 63 && *abort_flag)
-            return false;
-    }
-    *abort_flag = 1;
-    atomicExch(err, code);
-    return false;
-}
-
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-        ::"r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-// K-major operand in the 128-byte swizzled canonical layout: rows of 128 B,
-// 8-row groups 1024 B apart.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
-{
-    uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
-    d |= (uint64_t)1 << 16;              // leading byte offset (unused for swizzled K-major)
-    d |= (uint64_t)(1024 >> 4) << 32;    // stride byte offset: 8 rows x 128 B
-    d |= (uint64_t)1 << 46;              // descriptor version (sm_100)
-    d |= (uint64_t)2 << 61;              // 128-byte swizzle
-    return d;
-}
-
-// fp16 x fp16 -> fp32, A and B K-major, M = 128, N = n.
-__device__ __forceinline__ uint32_t idesc_f16(int n)
-{
-    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc));
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t *bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-                 : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b)
 {
@@ -198,41 +108,83 @@ __device__ __forceinline__ uint32_t code_at(const uint32_t (&w)[NW], int pos)
     return __funnelshift_r(w[wi], w[wi + 1], sh) & ((1u << BITS) - 1u);
 }
 
-// Row `row` of the 128 x 64 fp16 weight tile for k-step JJ of the chunk held
-// in w: 64 weights = 64/D codes, each a codebook entry times the row's scale
-// (fp16 product, rounded to nearest), stored as eight 16-byte chunks at
-// swizzled positions (chunk q of row r at q ^ (r & 7)).
+// The 16-byte-aligned words of a chunk row that hold k-step JJ's code bits.
 template <int D, int BITS, int JJ>
-__device__ __forceinline__ void dequant_step(const uint32_t (&w)[PG<D, BITS>::CHW], const char *cb, uint32_t s2,
+struct Win {
+    static constexpr int KB = PG<D, BITS>::KB;
+    static constexpr int W0 = ((JJ * KB) / 32) & ~3;
+    static constexpr int W1 = (((JJ * KB + KB + 31) / 32) + 3) & ~3;
+    static constexpr int NV = (W1 - W0) / 4;
+    static constexpr int BASE = JJ * KB - 32 * W0;
+};
+
+// Byte offset of the lane's replica of the code at bit `pos` of the window:
+// (code << L) | rep_off, formed with one shift and one mask-or.
+template <int BITS, int L, int NW>
+__device__ __forceinline__ uint32_t entry_off(const uint32_t (&w)[NW], int pos, uint32_t rep_off)
+{
+    const int wi = pos >> 5, sh = pos & 31;
+    uint32_t v;
+    int s;
+    if (sh + BITS <= 32) {
+        v = w[wi];
+        s = sh;
+    } else {
+        v = __funnelshift_r(w[wi], w[wi + 1], sh);
+        s = 0;
+    }
+    const uint32_t x = s >= L ? (v >> (s - L)) : (v << (L - s));
+    return (x & (((1u << BITS) - 1u) << L)) | rep_off;
+}
+
+// Row `row` of the 128 x 64 fp16 weight tile for k-step JJ of a code chunk:
+// 64 weights = 64/D codes read from the chunk row `crow` in shared memory,
+// each a codebook entry (the lane's replica) times the row's scale (fp16
+// product, rounded to nearest), stored as eight 16-byte chunks at swizzled
+// positions (chunk q of row r at q ^ (r & 7)).
+template <int D, int BITS, int JJ>
+__device__ __forceinline__ void dequant_step(const uint8_t *crow, const char *cb, uint32_t rep_off, uint32_t s2,
                                              bool live, char *arow, int rsw)
 {
+    using W = Win<D, BITS, JJ>;
     constexpr int NC = 64 / D;
-    constexpr int KB = PG<D, BITS>::KB;
+    constexpr int L = PG<D, BITS>::L;
+    uint32_t w[4 * W::NV];
+#pragma unroll
+    for (int v = 0; v < W::NV; ++v) {
+        const uint4 q = reinterpret_cast<const uint4 *>(crow)[W::W0 / 4 + v];
+        w[4 * v] = q.x;
+        w[4 * v + 1] = q.y;
+        w[4 * v + 2] = q.z;
+        w[4 * v + 3] = q.w;
+    }
     uint32_t o[32];
     if constexpr (D == 1) {
 #pragma unroll
         for (int c = 0; c < NC; c += 2) {
-            const uint32_t c0 = code_at<BITS>(w, JJ * KB + c * BITS);
-            const uint32_t c1 = code_at<BITS>(w, JJ * KB + (c + 1) * BITS);
-            const uint32_t v = (uint32_t)*reinterpret_cast<const uint16_t *>(cb + 2 * c0) |
-                               ((uint32_t)*reinterpret_cast<const uint16_t *>(cb + 2 * c1) << 16);
+            const uint32_t v = (uint32_t)*reinterpret_cast<const uint16_t *>(
+                                   cb + entry_off<BITS, L>(w, W::BASE + c * BITS, rep_off)) |
+                               ((uint32_t)*reinterpret_cast<const uint16_t *>(
+                                    cb + entry_off<BITS, L>(w, W::BASE + (c + 1) * BITS, rep_off))
+                                << 16);
             o[c >> 1] = hmul2(v, s2);
         }
     } else if constexpr (D == 2) {
 #pragma unroll
         for (int c = 0; c < NC; ++c)
-            o[c] = hmul2(*reinterpret_cast<const uint32_t *>(cb + 4 * code_at<BITS>(w, JJ * KB + c * BITS)), s2);
+            o[c] = hmul2(*reinterpret_cast<const uint32_t *>(cb + entry_off<BITS, L>(w, W::BASE + c * BITS, rep_off)),
+                         s2);
     } else if constexpr (D == 4) {
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
-            const uint2 v = *reinterpret_cast<const uint2 *>(cb + 8 * code_at<BITS>(w, JJ * KB + c * BITS));
+            const uint2 v = *reinterpret_cast<const uint2 *>(cb + entry_off<BITS, L>(w, W::BASE + c * BITS, rep_off));
             o[2 * c] = hmul2(v.x, s2);
             o[2 * c + 1] = hmul2(v.y, s2);
         }
     } else {
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(cb + 16 * code_at<BITS>(w, JJ * KB + c * BITS));
+            const uint4 v = *reinterpret_cast<const uint4 *>(cb + entry_off<BITS, L>(w, W::BASE + c * BITS, rep_off));
             o[4 * c] = hmul2(v.x, s2);
             o[4 * c + 1] = hmul2(v.y, s2);
             o[4 * c + 2] = hmul2(v.z, s2);
@@ -244,17 +196,6 @@ __device__ __forceinline__ void dequant_step(const uint32_t (&w)[PG<D, BITS>::CH
         uint4 v = live ? make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]) : make_uint4(0u, 0u, 0u, 0u);
         *reinterpret_cast<uint4 *>(arow + ((q ^ rsw) << 4)) = v;
     }
-}
-
-template <int D, int BITS, int JJ>
-__device__ __forceinline__ void dequant_chunk_steps(const uint32_t (&w)[2][PG<D, BITS>::CHW], const char *cb0,
-                                                    const char *cb1, const uint32_t (&s2)[2][PG<D, BITS>::CH],
-                                                    bool live0, bool live1, int nmod, char *a_stage, int rowi)
-{
-    char *arow = a_stage + rowi * 128;
-    dequant_step<D, BITS, JJ>(w[0], cb0, s2[0][JJ], live0, arow, rowi & 7);
-    if (nmod == 2)
-        dequant_step<D, BITS, JJ>(w[1], cb1, s2[1][JJ], live1, arow + A_TILE, rowi & 7);
 }
 
 // ------------------------------------------------------------------ kernel
@@ -297,8 +238,16 @@ template <int D, int BITS>
 __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __grid_constant__ PrefillArgs a)
 {
     using P = PG<D, BITS>;
+    // one code stage per module: the chunk's packed codes, then the scales of
+    // the 8-group block holding its k-steps
+    constexpr uint32_t CODE_STAGE = BM * P::CHW * 4 + BM * 16;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *smem = smem_raw;
+    if (smem_u32(smem) & 1023u) {   // the 128-byte swizzle needs 1024-byte aligned tiles
+        if (threadIdx.x == 0)
+            atomicExch(a.err, 20);
+        return;
+    }
     uint8_t *sm_a = smem + a.off_a;
     uint8_t *sm_b = smem + a.off_b;
     uint8_t *sm_c = smem + a.off_c;
@@ -312,13 +261,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nmod = a.nmod;
-    const int cb_bytes = (1 << BITS) * D * 2;
-
-    // codebooks (fp16 [K, d] per module) into shared memory
-    for (int i = threadIdx.x; i < nmod * cb_bytes / 16; i += NTHREADS) {
-        const int m = i / (cb_bytes / 16), j = i % (cb_bytes / 16);
-        reinterpret_cast<uint4 *>(sm_cb + m * cb_bytes)[j] =
-            reinterpret_cast<const uint4 *>(m == 0 ? a.mod[0].codebook : a.mod[1].codebook)[j];
+    // codebooks in shared memory: per module [K][R replicas][d] fp16, lane l
+    // reading replica l % R spreads a warp's random lookups over more banks
+    constexpr int log_rep = P::LREP;
+    const int cb_bytes = ((1 << BITS) << log_rep) * D * 2;
+    for (int i = threadIdx.x; i < nmod * (cb_bytes / 2); i += NTHREADS) {
+        const int m = i / (cb_bytes / 2), h = i % (cb_bytes / 2);
+        const int comp = h % D, slot = h / D;
+        reinterpret_cast<uint16_t *>(sm_cb + m * cb_bytes)[h] =
+            (m == 0 ? a.mod[0].codebook : a.mod[1].codebook)[(slot >> log_rep) * D + comp];
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < a.sa; ++s) {
@@ -328,7 +279,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
         }
         for (int s = 0; s < a.sc; ++s) {
             mbar_init(&full_c[s], 1);
-            mbar_init(&empty_c[s], 128);
+            mbar_init(&empty_c[s], 256);
         }
         mbar_init(acc_full, 1);
         *abort_flag = 0;
@@ -366,7 +317,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
         if (lane == 0) {
-            uint32_t ks = 0, cs = 0;
+            uint32_t ks = 0, st = 0, ph = 0, cst = 0, cph = 0;   // operand / code stage counters
             bool ok = true;
             for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
                 const Item itm = item_of(it, MT, tiles, n_act, a.active, a.offsets);
@@ -374,21 +325,30 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                 for (int m = 0; m < nmod; ++m)
                     prow0[m] = tile_prow0(a.mod[m], itm.e, itm.m0);
                 for (int c = 0; c < nchunks && ok; ++c) {
-                    const uint32_t cst = cs % a.sc, cph = (cs / a.sc) & 1;
                     if (!(ok = mbar_wait(&empty_c[cst], cph ^ 1, abort_flag, a.err, 1)))
                         break;
-                    mbar_expect_tx(&full_c[cst], (uint32_t)(nmod * BM * P::CHW * 4));
-                    for (int m = 0; m < nmod; ++m)
-                        tma_load_2d(sm_c + ((size_t)cst * nmod + m) * BM * P::CHW * 4, &a.tmap_c[m], c * P::CHW,
-                                    prow0[m], &full_c[cst]);
-                    ++cs;
+                    mbar_expect_tx(&full_c[cst], (uint32_t)(nmod * (a.scale_tma ? CODE_STAGE : BM * P::CHW * 4)));
+                    for (int m = 0; m < nmod; ++m) {
+                        uint8_t *stg = sm_c + ((size_t)cst * nmod + m) * CODE_STAGE;
+                        tma_load_2d(stg, &a.tmap_c[m], c * P::CHW, prow0[m], &full_c[cst]);
+                        if (a.scale_tma)
+                            tma_load_2d(stg + BM * P::CHW * 4, &a.tmap_s[m], (c * P::CH) & ~7, prow0[m],
+                                        &full_c[cst]);
+                    }
+                    if (++cst == (uint32_t)a.sc) {
+                        cst = 0;
+                        cph ^= 1;
+                    }
                     for (int j = 0; j < P::CH; ++j) {
-                        const uint32_t st = ks % a.sa, ph = (ks / a.sa) & 1;
                         if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag, a.err, 2)))
                             break;
                         mbar_expect_tx(&full_b[st], (uint32_t)B_TILE);
                         tma_load_2d(sm_b + (size_t)st * B_TILE, &a.tmap_b, (c * P::CH + j) * 64, itm.q0, &full_b[st]);
                         ++ks;
+                        if (++st == (uint32_t)a.sa) {
+                            st = 0;
+                            ph ^= 1;
+                        }
                     }
                 }
             }
@@ -402,14 +362,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            uint32_t ks = 0;
+            uint32_t st = 0, ph = 0;
             bool ok = true;
             for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
                 const Item itm = item_of(it, MT, tiles, n_act, a.active, a.offsets);
                 const int n16 = (itm.n + 15) & ~15;
-                const uint32_t idesc = idesc_f16(n16);
+                const uint32_t idesc = idesc_f16(BM, n16);
                 for (int k = 0; k < ksteps; ++k) {
-                    const uint32_t st = ks % a.sa, ph = (ks / a.sa) & 1;
                     if (!(ok = mbar_wait(&full_a[st], ph, abort_flag, a.err, 4)))
                         break;
                     if (!(ok = mbar_wait(&full_b[st], ph, abort_flag, a.err, 5)))
@@ -423,7 +382,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                             umma(tmem + m * BN, adesc + 2 * k16, bdesc + 2 * k16, idesc, (k | k16) != 0);
                     }
                     umma_commit(&empty[st]);
-                    ++ks;
+                    if (++st == (uint32_t)a.sa) {
+                        st = 0;
+                        ph ^= 1;
+                    }
                 }
                 if (ok)
                     umma_commit(acc_full);
@@ -431,9 +393,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
         }
     } else {
         // ---------------------------------------------------------- dequant + epilogue
+        const int wg = (warp - 2) >> 2;   // warpgroup: takes k-steps with (k & 1) == wg
         const int rowi = 32 * (warp & 3) + lane;
+        const uint32_t rep_off = (uint32_t)(lane & ((1 << log_rep) - 1)) * (2 * D);
         const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
-        uint32_t ks = 0, cs = 0, nit = 0;
+        uint32_t st = 0, ph = 0, cst = 0, cph = 0, nit = 0;
         bool ok = true;
         for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
             const Item itm = item_of(it, MT, tiles, n_act, a.active, a.offsets);
@@ -446,63 +410,64 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                 lrow[m] = prow[m] >= 0 ? (int)(prow[m] - tile_prow0(md, itm.e, itm.m0)) : -1;
             }
             for (int c = 0; c < nchunks && ok; ++c) {
-                // scales of this chunk's k-steps, then the chunk's code words
-                uint32_t s2[2][P::CH];
-#pragma unroll
-                for (int m = 0; m < 2; ++m)
-#pragma unroll
-                    for (int j = 0; j < P::CH; ++j) {
-                        uint32_t s = 0;
-                        if (m < nmod && prow[m] >= 0)
-                            s = ldg_u16(a.mod[m].scales + prow[m] * a.mod[m].ngroups + c * P::CH + j);
-                        s2[m][j] = s | (s << 16);
-                    }
-                const uint32_t cst = cs % a.sc, cph = (cs / a.sc) & 1;
                 if (!(ok = mbar_wait(&full_c[cst], cph, abort_flag, a.err, 6)))
                     break;
-                uint32_t w[2][P::CHW];
+                const uint8_t *crow[2];
+                const uint16_t *srow[2];
 #pragma unroll
                 for (int m = 0; m < 2; ++m) {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(
-                        sm_c + ((size_t)cst * nmod + (m < nmod ? m : 0)) * BM * P::CHW * 4 +
-                        (size_t)(lrow[m] >= 0 ? lrow[m] : 0) * P::CHW * 4);
-#pragma unroll
-                    for (int q = 0; q < P::CHW / 4; ++q) {
-                        const uint4 v = (m < nmod) ? src[q] : make_uint4(0u, 0u, 0u, 0u);
-                        w[m][4 * q] = v.x;
-                        w[m][4 * q + 1] = v.y;
-                        w[m][4 * q + 2] = v.z;
-                        w[m][4 * q + 3] = v.w;
-                    }
+                    const uint8_t *stg = sm_c + ((size_t)cst * nmod + (m < nmod ? m : 0)) * CODE_STAGE;
+                    const int lr = lrow[m] >= 0 ? lrow[m] : 0;
+                    crow[m] = stg + (size_t)lr * P::CHW * 4;
+                    srow[m] = reinterpret_cast<const uint16_t *>(stg + BM * P::CHW * 4) + lr * 8 + ((c * P::CH) & 7);
                 }
-                mbar_arrive(&empty_c[cst]);
-                ++cs;
+                // the row's fp16 scale of k-step j, as a half2 pair
+                auto sfetch = [&](int m, int j) {
+                    uint32_t sc;
+                    if (a.scale_tma)
+                        sc = srow[m][j];
+                    else
+                        sc = prow[m] >= 0 ? ldg_u16(a.mod[m].scales + prow[m] * a.mod[m].ngroups + c * P::CH + j) : 0u;
+                    return sc | (sc << 16);
+                };
                 auto step = [&](auto jj_c) {
                     constexpr int JJ = decltype(jj_c)::value;
                     if (!ok)
                         return;
-                    const uint32_t st = ks % a.sa, ph = (ks / a.sa) & 1;
-                    if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag, a.err, 7)))
-                        return;
-                    dequant_chunk_steps<D, BITS, JJ>(w, sm_cb, sm_cb + cb_bytes, s2, lrow[0] >= 0, lrow[1] >= 0,
-                                                     nmod, reinterpret_cast<char *>(sm_a) + (size_t)st * nmod * A_TILE,
-                                                     rowi);
-                    fence_async_smem();
-                    mbar_arrive(&full_a[st]);
-                    ++ks;
+                    if (((c * P::CH + JJ) & 1) == wg) {
+                        if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag, a.err, 7)))
+                            return;
+                        char *arow = reinterpret_cast<char *>(sm_a) + (size_t)st * nmod * A_TILE + rowi * 128;
+                        dequant_step<D, BITS, JJ>(crow[0], sm_cb, rep_off, sfetch(0, JJ), lrow[0] >= 0, arow, rowi & 7);
+                        if (nmod == 2)
+                            dequant_step<D, BITS, JJ>(crow[1], sm_cb + cb_bytes, rep_off, sfetch(1, JJ), lrow[1] >= 0,
+                                                      arow + A_TILE, rowi & 7);
+                        fence_async_smem();
+                        mbar_arrive(&full_a[st]);
+                    }
+                    if (++st == (uint32_t)a.sa) {
+                        st = 0;
+                        ph ^= 1;
+                    }
                 };
                 [&]<int... J>(std::integer_sequence<int, J...>) {
                     (step(std::integral_constant<int, J>{}), ...);
                 }(std::make_integer_sequence<int, P::CH>{});
+                mbar_arrive(&empty_c[cst]);
+                if (++cst == (uint32_t)a.sc) {
+                    cst = 0;
+                    cph ^= 1;
+                }
             }
             if (!ok)
                 break;
-            // epilogue: accumulators of this tile are complete
+            // epilogue: accumulators of this tile are complete; the warpgroups
+            // take alternate 32-column blocks
             if (!(ok = mbar_wait(acc_full, nit & 1, abort_flag, a.err, 8)))
                 break;
             ++nit;
             tc_fence_after();
-            for (int cb0 = 0; cb0 < itm.n; cb0 += 32) {
+            for (int cb0 = 32 * wg; cb0 < itm.n; cb0 += 64) {
                 uint32_t g[32], u[32];
                 tmem_ld32(tmem + lane_addr + cb0, g);
                 if (nmod == 2)
@@ -558,45 +523,27 @@ __global__ void vq_gather_kernel(const uint16_t *__restrict__ x, const int32_t *
 
 // ------------------------------------------------------------------ host side
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+int chw_of(int d, int bits);
+
+// fp16 activations [rows, cols]: boxes of 64 columns x BN rows, 128-byte swizzle
+bool map_act(CUtensorMap *map, const void *base, long rows, int cols)
 {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
+    return tma_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, (uint64_t)cols, (uint64_t)rows, 64, BN,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-bool make_map_f16(CUtensorMap *map, const void *base, long rows, int cols)
+// fp16 scales [live rows, ngroups]: boxes of 8 groups x BM rows
+bool map_scales(CUtensorMap *map, const ModDev &m)
 {
-    auto enc = encode_fn();
-    if (!enc)
-        return false;
-    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    cuuint32_t box[2] = {64, BN};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return tma_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, m.scales, (uint64_t)m.ngroups, (uint64_t)m.live_rows, 8,
+                      BM, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-bool make_map_codes(CUtensorMap *map, const ModDev &m, int chw)
+// packed codes [live rows, row_words]: boxes of one chunk x BM rows
+bool map_codes(CUtensorMap *map, const ModDev &m)
 {
-    auto enc = encode_fn();
-    if (!enc)
-        return false;
-    cuuint64_t dims[2] = {(cuuint64_t)m.row_words, (cuuint64_t)m.live_rows};
-    cuuint64_t strides[1] = {(cuuint64_t)m.row_words * 4};
-    cuuint32_t box[2] = {(cuuint32_t)chw, BM};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(m.codes), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return tma_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, m.codes, (uint64_t)m.row_words, (uint64_t)m.live_rows,
+                      (uint32_t)chw_of(m.d, m.bits), BM, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 int chw_of(int d, int bits)
@@ -615,8 +562,8 @@ struct SmemPlan {
 SmemPlan smem_plan(int nmod, int d, int bits, int E)
 {
     const uint32_t limit = 227 * 1024 - 1024;   // minus the alignment slack
-    const uint32_t code_stage = (uint32_t)nmod * BM * chw_of(d, bits) * 4;
-    const uint32_t cb = (uint32_t)align_up((size_t)nmod * ((size_t)1 << bits) * d * 2, 128);
+    const uint32_t code_stage = (uint32_t)nmod * (BM * chw_of(d, bits) * 4 + BM * 16);
+    const uint32_t cb = (uint32_t)align_up((size_t)nmod * ((size_t)1 << bits) * d * 2 << prefill_log_rep(d, bits), 128);
     const uint32_t tiles = (uint32_t)align_up((size_t)(E + 1) * 4, 128);
     SmemPlan p{};
     for (int sa = 4; sa >= 2; --sa) {
@@ -704,7 +651,7 @@ vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const flo
         return VQ_ERR_UNSUPPORTED;
     if (L->gate.d != L->up.d || L->gate.bits != L->up.bits)
         return VQ_ERR_UNSUPPORTED;   // gate and up share one fused tile
-    if (!encode_fn())
+    if (!tma_available())
         return VQ_ERR_CUDA;
     const int E = L->gate.E, H = L->gate.cols, I = L->gate.rows;
     if (T == 0)
@@ -752,9 +699,9 @@ vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const flo
         a.mod[0] = make_moddev(L->gate);
         a.mod[1] = make_moddev(L->up);
         a.nmod = 2;
-        if (!make_map_f16(&a.tmap_b, xg, tk, H) ||
-            !make_map_codes(&a.tmap_c[0], a.mod[0], chw_of(a.mod[0].d, a.mod[0].bits)) ||
-            !make_map_codes(&a.tmap_c[1], a.mod[1], chw_of(a.mod[1].d, a.mod[1].bits)))
+        if (!map_act(&a.tmap_b, xg, tk, H) || !map_codes(&a.tmap_c[0], a.mod[0]) || !map_codes(&a.tmap_c[1], a.mod[1]))
+            return VQ_ERR_CUDA;
+        if (a.mod[0].ngroups % 8 == 0 && (!map_scales(&a.tmap_s[0], a.mod[0]) || !map_scales(&a.tmap_s[1], a.mod[1])))
             return VQ_ERR_CUDA;
         a.offsets = offsets;
         a.active = active;
@@ -772,6 +719,7 @@ vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const flo
         a.off_cb = sp.off_cb;
         a.off_tiles = sp.off_tiles;
         a.off_bar = sp.off_bar;
+        a.scale_tma = a.mod[0].ngroups % 8 == 0;
         a.out = hh;
         a.swiglu = 1;
         a.err = err;
@@ -786,10 +734,12 @@ vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const flo
         a.mod[0] = make_moddev(L->down);
         a.mod[1] = a.mod[0];
         a.nmod = 1;
-        if (!make_map_f16(&a.tmap_b, hh, tk, I) ||
-            !make_map_codes(&a.tmap_c[0], a.mod[0], chw_of(a.mod[0].d, a.mod[0].bits)))
+        if (!map_act(&a.tmap_b, hh, tk, I) || !map_codes(&a.tmap_c[0], a.mod[0]))
+            return VQ_ERR_CUDA;
+        if (a.mod[0].ngroups % 8 == 0 && !map_scales(&a.tmap_s[0], a.mod[0]))
             return VQ_ERR_CUDA;
         a.tmap_c[1] = a.tmap_c[0];
+        a.tmap_s[1] = a.tmap_s[0];
         a.offsets = offsets;
         a.active = active;
         a.n_active = nact;
@@ -806,6 +756,7 @@ vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const flo
         a.off_cb = sp.off_cb;
         a.off_tiles = sp.off_tiles;
         a.off_bar = sp.off_bar;
+        a.scale_tma = a.mod[0].ngroups % 8 == 0;
         a.out = dp;
         a.swiglu = 0;
         a.err = err;
