@@ -16,12 +16,13 @@
 //   warp 1     owns the tensor memory; one thread issues tcgen05.mma
 //   warps 2-9  two warpgroups taking alternate k-steps: thread i of a
 //              warpgroup decodes row i of the weight tile (unpack, codebook
-//              lookup, x fp16 scale) into the swizzled K-major shared-memory
-//              layout the tensor core reads; both then run the epilogue from
-//              tensor memory (lane i = row i), on alternate 32-column blocks
+//              lookup, x fp16 scale) and stores it into tensor memory lane i,
+//              where tcgen05.mma reads its A operand; both then run the
+//              epilogue from tensor memory, on alternate 32-column blocks
 // D[row, token] = sum_k W[row, k] X[token, k]: the weight tile is the
-// M=128 operand, the tokens of the bucket the N operand (16..128), so small
-// buckets waste no M rows. Every mbarrier wait is bounded; on a timeout the
+// M=128 operand (in tensor memory), the tokens of the bucket the N operand
+// (16..128, shared memory), so small buckets waste no M rows. Tensor memory
+// holds the accumulators (nmod x 128 columns) and 4 stages of A tiles. Every mbarrier wait is bounded; on a timeout the
 // CTA records an error word, stops, and frees its tensor memory.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -39,7 +40,7 @@ namespace {
 constexpr int BM = 128;             // weight rows per tile = TMEM lanes
 constexpr int BN = 128;             // tokens per tile
 constexpr int NTHREADS = 320;       // 10 warps: TMA, MMA, 8 dequant/epilogue
-constexpr int A_TILE = BM * 128;    // bytes of one 128 x 64 fp16 tile
+constexpr int A_COLS = 32;          // tensor-memory columns of one 128 x 64 fp16 weight tile
 constexpr int B_TILE = BN * 128;
 
 __host__ __device__ constexpr int chunk_steps(int kb)
@@ -137,14 +138,14 @@ __device__ __forceinline__ uint32_t entry_off(const uint32_t (&w)[NW], int pos, 
     return (x & (((1u << BITS) - 1u) << L)) | rep_off;
 }
 
-// Row `row` of the 128 x 64 fp16 weight tile for k-step JJ of a code chunk:
+// One row of the 128 x 64 fp16 weight tile for k-step JJ of a code chunk:
 // 64 weights = 64/D codes read from the chunk row `crow` in shared memory,
 // each a codebook entry (the lane's replica) times the row's scale (fp16
-// product, rounded to nearest), stored as eight 16-byte chunks at swizzled
-// positions (chunk q of row r at q ^ (r & 7)).
+// product, rounded to nearest), as 32 words o[c] = weights (2c, 2c+1), the
+// layout of one tensor-memory lane of the MMA's A operand.
 template <int D, int BITS, int JJ>
 __device__ __forceinline__ void dequant_step(const uint8_t *crow, const char *cb, uint32_t rep_off, uint32_t s2,
-                                             bool live, char *arow, int rsw)
+                                             bool live, uint32_t (&o)[32])
 {
     using W = Win<D, BITS, JJ>;
     constexpr int NC = 64 / D;
@@ -158,7 +159,6 @@ __device__ __forceinline__ void dequant_step(const uint8_t *crow, const char *cb
         w[4 * v + 2] = q.z;
         w[4 * v + 3] = q.w;
     }
-    uint32_t o[32];
     if constexpr (D == 1) {
 #pragma unroll
         for (int c = 0; c < NC; c += 2) {
@@ -191,10 +191,10 @@ __device__ __forceinline__ void dequant_step(const uint8_t *crow, const char *cb
             o[4 * c + 3] = hmul2(v.w, s2);
         }
     }
+    if (!live) {
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        uint4 v = live ? make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]) : make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4 *>(arow + ((q ^ rsw) << 4)) = v;
+        for (int q = 0; q < 32; ++q)
+            o[q] = 0u;
     }
 }
 
@@ -248,7 +248,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
             atomicExch(a.err, 20);
         return;
     }
-    uint8_t *sm_a = smem + a.off_a;
     uint8_t *sm_b = smem + a.off_b;
     uint8_t *sm_c = smem + a.off_c;
     char *sm_cb = reinterpret_cast<char *>(smem + a.off_cb);
@@ -285,7 +284,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    const uint32_t tmem_cols = nmod == 2 ? 2 * BN : BN;
+    // accumulators: nmod x BN columns; then sa stages of nmod A tiles
+    const uint32_t acc_cols = (uint32_t)nmod * BN;
+    const uint32_t tmem_cols = nmod == 2 ? 512 : 256;
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(tmem_cols));
@@ -376,10 +377,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                     tc_fence_after();
                     const uint64_t bdesc = sw128_desc(smem_u32(sm_b + (size_t)st * B_TILE));
                     for (int m = 0; m < nmod; ++m) {
-                        const uint64_t adesc = sw128_desc(smem_u32(sm_a + ((size_t)st * nmod + m) * A_TILE));
+                        const uint32_t a_tmem = tmem + acc_cols + (st * nmod + m) * A_COLS;
 #pragma unroll
                         for (int k16 = 0; k16 < 4; ++k16)
-                            umma(tmem + m * BN, adesc + 2 * k16, bdesc + 2 * k16, idesc, (k | k16) != 0);
+                            umma_ts(tmem + m * BN, a_tmem + 8 * k16, bdesc + 2 * k16, idesc, (k | k16) != 0);
                     }
                     umma_commit(&empty[st]);
                     if (++st == (uint32_t)a.sa) {
@@ -437,12 +438,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                     if (((c * P::CH + JJ) & 1) == wg) {
                         if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag, a.err, 7)))
                             return;
-                        char *arow = reinterpret_cast<char *>(sm_a) + (size_t)st * nmod * A_TILE + rowi * 128;
-                        dequant_step<D, BITS, JJ>(crow[0], sm_cb, rep_off, sfetch(0, JJ), lrow[0] >= 0, arow, rowi & 7);
-                        if (nmod == 2)
-                            dequant_step<D, BITS, JJ>(crow[1], sm_cb + cb_bytes, rep_off, sfetch(1, JJ), lrow[1] >= 0,
-                                                      arow + A_TILE, rowi & 7);
-                        fence_async_smem();
+                        const uint32_t a_tmem = tmem + lane_addr + acc_cols + st * nmod * A_COLS;
+                        uint32_t o[32];
+                        dequant_step<D, BITS, JJ>(crow[0], sm_cb, rep_off, sfetch(0, JJ), lrow[0] >= 0, o);
+                        tmem_st32(a_tmem, o);
+                        if (nmod == 2) {
+                            dequant_step<D, BITS, JJ>(crow[1], sm_cb + cb_bytes, rep_off, sfetch(1, JJ),
+                                                      lrow[1] >= 0, o);
+                            tmem_st32(a_tmem + A_COLS, o);
+                        }
+                        tmem_wait_st();
+                        tc_fence_before();
                         mbar_arrive(&full_a[st]);
                     }
                     if (++st == (uint32_t)a.sa) {
@@ -566,11 +572,11 @@ SmemPlan smem_plan(int nmod, int d, int bits, int E)
     const uint32_t cb = (uint32_t)align_up((size_t)nmod * ((size_t)1 << bits) * d * 2 << prefill_log_rep(d, bits), 128);
     const uint32_t tiles = (uint32_t)align_up((size_t)(E + 1) * 4, 128);
     SmemPlan p{};
-    for (int sa = 4; sa >= 2; --sa) {
+    for (int sa = 4; sa >= 4; --sa) {   // tensor memory holds 4 A stages
         p.sa = sa;
         p.sc = 2;
         p.off_a = 0;
-        p.off_b = p.off_a + (uint32_t)sa * nmod * A_TILE;
+        p.off_b = 0;
         p.off_c = p.off_b + (uint32_t)sa * B_TILE;
         p.off_cb = p.off_c + p.sc * code_stage;
         p.off_tiles = p.off_cb + cb;
