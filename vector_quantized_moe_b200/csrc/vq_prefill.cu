@@ -51,25 +51,39 @@ __host__ __device__ constexpr int chunk_steps(int kb)
     return ch;
 }
 
-// codebook replicas in shared memory (log2): as many as fit 32 KB for two
-// modules, at most 16
-__host__ __device__ constexpr int prefill_log_rep(int d, int bits)
+__host__ __device__ constexpr int log2i(int v) { return v <= 1 ? 0 : 1 + log2i(v / 2); }
+
+constexpr int B_STAGES = 4;           // activation tiles in shared memory (= A stages in tensor memory)
+constexpr int CODE_STAGES = 2;
+constexpr long SMEM_LIMIT = 227L * 1024;
+constexpr long SMEM_RESERVE = 1024 + 17L * 1024;   // alignment slack, tile table (E <= 4096), barriers
+
+// bytes of one code stage of one module: the chunk's packed codes of BM rows,
+// then the scales of an 8-group block
+__host__ __device__ constexpr long code_stage_bytes(int d, int bits)
 {
+    return (long)128 * (chunk_steps((64 / d) * bits) * ((64 / d) * bits) / 32) * 4 + 128 * 16;
+}
+
+// codebook replicas in shared memory (log2, at most 16 replicas): as many as
+// fit next to the operand and code stages
+__host__ __device__ constexpr int prefill_log_rep(int d, int bits, int nmod)
+{
+    const long left = SMEM_LIMIT - SMEM_RESERVE - (long)B_STAGES * 128 * 128 -
+                      (long)CODE_STAGES * nmod * code_stage_bytes(d, bits);
     int lr = 0;
-    while (lr < 4 && 2L * (1L << bits) * d * 2 * (2L << lr) <= 32768)
+    while (lr < 4 && (long)nmod * (1L << bits) * d * 2 * (2L << lr) <= left)
         ++lr;
     return lr;
 }
 
-__host__ __device__ constexpr int log2i(int v) { return v <= 1 ? 0 : 1 + log2i(v / 2); }
-
-template <int D, int BITS>
+template <int D, int BITS, int NMOD>
 struct PG {
     static constexpr int KB = (64 / D) * BITS;       // code bits of one row per 64-column step
     static constexpr int CH = chunk_steps(KB);       // steps per code chunk (whole 16-byte units)
     static constexpr int CHW = CH * KB / 32;         // words per row per chunk
     static constexpr uint32_t MASK = (1u << BITS) - 1u;
-    static constexpr int LREP = prefill_log_rep(D, BITS);
+    static constexpr int LREP = prefill_log_rep(D, BITS, NMOD);
     static constexpr int L = LREP + 1 + log2i(D);    // code -> byte offset of its replica row
 };
 
@@ -112,7 +126,7 @@ __device__ __forceinline__ uint32_t code_at(const uint32_t (&w)[NW], int pos)
 // The 16-byte-aligned words of a chunk row that hold k-step JJ's code bits.
 template <int D, int BITS, int JJ>
 struct Win {
-    static constexpr int KB = PG<D, BITS>::KB;
+    static constexpr int KB = (64 / D) * BITS;
     static constexpr int W0 = ((JJ * KB) / 32) & ~3;
     static constexpr int W1 = (((JJ * KB + KB + 31) / 32) + 3) & ~3;
     static constexpr int NV = (W1 - W0) / 4;
@@ -143,13 +157,12 @@ __device__ __forceinline__ uint32_t entry_off(const uint32_t (&w)[NW], int pos, 
 // each a codebook entry (the lane's replica) times the row's scale (fp16
 // product, rounded to nearest), as 32 words o[c] = weights (2c, 2c+1), the
 // layout of one tensor-memory lane of the MMA's A operand.
-template <int D, int BITS, int JJ>
+template <int D, int BITS, int L, int JJ>
 __device__ __forceinline__ void dequant_step(const uint8_t *crow, const char *cb, uint32_t rep_off, uint32_t s2,
                                              bool live, uint32_t (&o)[32])
 {
     using W = Win<D, BITS, JJ>;
     constexpr int NC = 64 / D;
-    constexpr int L = PG<D, BITS>::L;
     uint32_t w[4 * W::NV];
 #pragma unroll
     for (int v = 0; v < W::NV; ++v) {
@@ -234,10 +247,10 @@ __device__ __forceinline__ int tile_prow0(const ModDev &m, int e, int m0)
     return (int)m.rank[(long)e * m.bm_words + (m0 >> 5)];
 }
 
-template <int D, int BITS>
+template <int D, int BITS, int NMOD>
 __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __grid_constant__ PrefillArgs a)
 {
-    using P = PG<D, BITS>;
+    using P = PG<D, BITS, NMOD>;
     // one code stage per module: the chunk's packed codes, then the scales of
     // the 8-group block holding its k-steps
     constexpr uint32_t CODE_STAGE = BM * P::CHW * 4 + BM * 16;
@@ -259,7 +272,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nmod = a.nmod;
+    constexpr int nmod = NMOD;
     // codebooks in shared memory: per module [K][R replicas][d] fp16, lane l
     // reading replica l % R spreads a warp's random lookups over more banks
     constexpr int log_rep = P::LREP;
@@ -440,11 +453,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                             return;
                         const uint32_t a_tmem = tmem + lane_addr + acc_cols + st * nmod * A_COLS;
                         uint32_t o[32];
-                        dequant_step<D, BITS, JJ>(crow[0], sm_cb, rep_off, sfetch(0, JJ), lrow[0] >= 0, o);
+                        dequant_step<D, BITS, P::L, JJ>(crow[0], sm_cb, rep_off, sfetch(0, JJ), lrow[0] >= 0, o);
                         tmem_st32(a_tmem, o);
                         if (nmod == 2) {
-                            dequant_step<D, BITS, JJ>(crow[1], sm_cb + cb_bytes, rep_off, sfetch(1, JJ),
-                                                      lrow[1] >= 0, o);
+                            dequant_step<D, BITS, P::L, JJ>(crow[1], sm_cb + cb_bytes, rep_off, sfetch(1, JJ),
+                                                            lrow[1] >= 0, o);
                             tmem_st32(a_tmem + A_COLS, o);
                         }
                         tmem_wait_st();
@@ -568,13 +581,14 @@ struct SmemPlan {
 SmemPlan smem_plan(int nmod, int d, int bits, int E)
 {
     const uint32_t limit = 227 * 1024 - 1024;   // minus the alignment slack
-    const uint32_t code_stage = (uint32_t)nmod * (BM * chw_of(d, bits) * 4 + BM * 16);
-    const uint32_t cb = (uint32_t)align_up((size_t)nmod * ((size_t)1 << bits) * d * 2 << prefill_log_rep(d, bits), 128);
+    const uint32_t code_stage = (uint32_t)(nmod * code_stage_bytes(d, bits));
+    const uint32_t cb =
+        (uint32_t)align_up((size_t)nmod * ((size_t)1 << bits) * d * 2 << prefill_log_rep(d, bits, nmod), 128);
     const uint32_t tiles = (uint32_t)align_up((size_t)(E + 1) * 4, 128);
     SmemPlan p{};
-    for (int sa = 4; sa >= 4; --sa) {   // tensor memory holds 4 A stages
+    for (int sa = B_STAGES; sa >= 2; --sa) {   // tensor memory holds up to B_STAGES A stages
         p.sa = sa;
-        p.sc = 2;
+        p.sc = CODE_STAGES;
         p.off_a = 0;
         p.off_b = 0;
         p.off_c = p.off_b + (uint32_t)sa * B_TILE;
@@ -589,10 +603,10 @@ SmemPlan smem_plan(int nmod, int d, int bits, int E)
     return p;
 }
 
-template <int D, int BITS>
+template <int D, int BITS, int NMOD>
 cudaError_t launch_gemm(const PrefillArgs &a, int ctas, uint32_t smem, cudaStream_t s)
 {
-    auto k = vq_prefill_gemm_kernel<D, BITS>;
+    auto k = vq_prefill_gemm_kernel<D, BITS, NMOD>;
     cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess)
         return err;
@@ -612,7 +626,8 @@ cudaError_t launch_gemm(const PrefillArgs &a, int ctas, uint32_t smem, cudaStrea
 cudaError_t dispatch_gemm(const PrefillArgs &a, int d, int bits, int ctas, uint32_t smem, cudaStream_t s)
 {
 #define VQ_PGEMM(D_, B_) \
-    if (d == D_ && bits == B_) return launch_gemm<D_, B_>(a, ctas, smem, s);
+    if (d == D_ && bits == B_) \
+        return a.nmod == 2 ? launch_gemm<D_, B_, 2>(a, ctas, smem, s) : launch_gemm<D_, B_, 1>(a, ctas, smem, s);
     VQ_GEOMETRIES(VQ_PGEMM)
 #undef VQ_PGEMM
     return cudaErrorInvalidValue;
