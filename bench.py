@@ -62,9 +62,15 @@ def _module_bytes(md):
     return live * per_row
 
 
-def _kernel_source_hash():
+KERNEL_SOURCES = {
+    "grouped_gemv_gate_up": ("vq_decode.cu", "vq_device.cuh", "vq_sm100.cuh"),
+    "prefill_gemm_gate_up": ("vq_prefill.cu", "vq_device.cuh", "vq_sm100.cuh"),
+}
+
+
+def _kernel_source_hash(tag):
     h = hashlib.sha256()
-    for f in ("vq_decode.cu", "vq_device.cuh"):
+    for f in KERNEL_SOURCES[tag]:
         with open(os.path.join(ROOT, "vector_quantized_moe_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -77,7 +83,7 @@ def _traffic_per_launch(kernel_tag):
     try:
         with open(path) as f:
             t = json.load(f).get(kernel_tag)
-        if t and t.get("source_hash") == _kernel_source_hash():
+        if t and t.get("source_hash") == _kernel_source_hash(kernel_tag):
             return float(t["dram_bytes_per_launch"])
     except Exception:
         pass
