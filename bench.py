@@ -147,6 +147,26 @@ def _dist():
     return ws, rank, local
 
 
+def dist_max(v, device, ws):
+    """Max of a float over the ranks (the slowest rank's time)."""
+    if ws == 1:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_sum(v, device, ws):
+    """Sum of a float over the ranks (bytes processed by all replicas)."""
+    if ws == 1:
+        return v
+    import torch
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t)
+    return float(t.item())
+
+
 def run_reference(args):
     """The oracle (CPU, float64) on bounded samples of the same workload."""
     ws, rank, _ = _dist()
@@ -243,18 +263,10 @@ def run_ours(args):
             torch.distributed.barrier()
 
     def max_over_ranks(v):
-        if ws == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+        return dist_max(v, dev, ws)
 
     def sum_over_ranks(v):
-        if ws == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t)
-        return float(t.item())
+        return dist_sum(v, dev, ws)
 
     for i in range(args.warmup):
         step(i)

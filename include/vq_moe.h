@@ -47,7 +47,7 @@ typedef enum vq_status {
     VQ_ERR_UNSUPPORTED = 3,   /* geometry (d, bits) or size the kernels do not implement */
     VQ_ERR_WORKSPACE = 4,     /* workspace NULL, misaligned or smaller than required */
     VQ_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
-    VQ_ERR_DEVICE_CHECK = 6   /* the device reported an inconsistency (see vq_moe_check) */
+    VQ_ERR_DEVICE_CHECK = 6   /* a kernel gave up a bounded wait (see vq_moe_check) */
 } vq_status;
 
 /* Output element types. */
@@ -198,6 +198,15 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
 vq_status vq_moe_prefill(const vq_moe_layer *L, const uint16_t *x, int32_t T, const float *logits,
                          int32_t top_k, int32_t renorm, void *y, int32_t y_dtype, void *workspace,
                          size_t ws_bytes, void *stream);
+
+/* Diagnostic (synchronises `stream`). Every wait of the library's pipelined
+ * kernels on an on-chip barrier is bounded; a kernel that gives up records a
+ * nonzero word at offset 0 of the MoE workspace it ran with (the routing
+ * kernel of each vq_moe_decode / vq_moe_prefill call clears it) and stops
+ * without completing its outputs. Returns VQ_ERR_DEVICE_CHECK when the word
+ * of `workspace` is set after the work queued on `stream`, VQ_OK when not,
+ * VQ_ERR_WORKSPACE for a NULL or misaligned workspace. */
+vq_status vq_moe_check(const void *workspace, void *stream);
 
 /* vq_moe_decode without a workspace argument, for callers that cannot
  * allocate device memory: code running inside a host framework that owns

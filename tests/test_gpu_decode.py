@@ -132,6 +132,7 @@ def test_moe_decode_small(geos, dead, T):
         yb = layer.decode(xt, lt, k, renorm, out_dtype=torch.bfloat16)
         torch.cuda.synchronize()
         assert_close(y.cpu().numpy(), ref, what=f"moe decode {geos} T{T}")
+        assert layer.check(vq.VQ_MODE_DECODE) == vq.VQ_OK
         assert np.array_equal(yb.view(torch.int16).cpu().numpy().view(np.uint16), _bf16_of(y))
 
 

@@ -52,6 +52,7 @@ def test_prefill_small(case, T):
     yd = layer.decode(xt, lt, k)
     torch.cuda.synchronize()
     assert_close(y.cpu().numpy(), ref, what=f"prefill case{case} T{T}")
+    assert layer.check(vq.VQ_MODE_PREFILL) == vq.VQ_OK
     assert np.array_equal(yb.view(torch.int16).cpu().numpy().view(np.uint16), _bf16_of(y))
     assert_close(y.cpu().numpy(), yd.cpu().numpy().astype(np.float64), what="prefill vs decode")
 

@@ -64,6 +64,7 @@ def _load():
         "vq_moe_decode": (ctypes.c_int, [LP, P, I32, P, I32, I32, P, I32, P, SZ, P]),
         "vq_moe_prefill": (ctypes.c_int, [LP, P, I32, P, I32, I32, P, I32, P, SZ, P]),
         "vq_set_trace_events": (ctypes.c_int, [P, I32]),
+        "vq_moe_check": (ctypes.c_int, [P, P]),
         "vq_moe_decode_noalloc": (ctypes.c_int, [LP, P, I32, P, I32, I32, P, I32, P]),
     }
     for name, (res, args) in sig.items():
@@ -294,6 +295,14 @@ class MoELayer:
         _check(fn(ctypes.byref(self._s), x.data_ptr(), T, logits.data_ptr(), top_k, int(bool(renorm)),
                   out.data_ptr(), _dt(out.dtype), aligned, nbytes, _stream(stream)), name)
         return out
+
+    def check(self, mode: int, stream=None) -> int:
+        """Status of the device error word of the cached workspace for `mode` (vq_moe_check)."""
+        ws = self._ws.get(mode)
+        if ws is None:
+            return VQ_OK
+        base = (ws.data_ptr() + 255) // 256 * 256
+        return int(_L().vq_moe_check(base, _stream(stream)))
 
     def decode(self, x, logits, top_k: int, renorm: bool = True, out=None, out_dtype=None, workspace=None,
                stream=None):

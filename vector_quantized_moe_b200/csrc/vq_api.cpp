@@ -71,7 +71,7 @@ struct DecodePlan {
     int T, k, E, H, I;
     int sa, sb;                  // slices of the gate/up and down passes
     RoutingLayout r;
-    size_t off_err, off_x16, off_G, off_U, off_h, off_D;
+    size_t off_x16, off_G, off_U, off_h, off_D;
     size_t total;
 };
 
@@ -108,7 +108,6 @@ DecodePlan plan_decode(const vq_moe_layer *L, int T, int k)
     size_t o = 0;
     p.r = plan_routing(o, T, k, p.E);
     const size_t tk = (size_t)T * k;
-    p.off_err = o; o = align_up(o + 16, 256);
     p.off_x16 = o; o = align_up(o + (size_t)T * p.H * 2, 256);
     p.off_G = o; o = align_up(o + (size_t)p.sa * tk * p.I * 4, 256);
     p.off_U = o; o = align_up(o + (size_t)p.sa * tk * p.I * 4, 256);
@@ -347,7 +346,7 @@ vq_status vq_route(const float *logits, int32_t T, int32_t E, int32_t top_k, int
         top_k > std::min(E, 32) || (long)T * top_k >= (1L << 31))
         return VQ_ERR_ARG;
     return cuda_status(launch_route(logits, T, E, top_k, renorm, ids, weights, offsets, perm, nullptr, nullptr,
-                                    nullptr, nullptr, nullptr, 0, (cudaStream_t)stream, false));
+                                    nullptr, nullptr, nullptr, 0, nullptr, (cudaStream_t)stream, false));
 }
 
 size_t vq_moe_workspace_size(const vq_moe_layer *L, int32_t T, int32_t top_k, int32_t mode)
@@ -396,7 +395,7 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     int32_t *pos = ws_at<int32_t>(workspace, p.r.pos);
     int32_t *active = ws_at<int32_t>(workspace, p.r.active);
     int32_t *nact = ws_at<int32_t>(workspace, p.r.nact);
-    int *errw = ws_at<int>(workspace, p.off_err);
+    int *errw = ws_at<int>(workspace, p.r.err);
     __half *x16 = ws_at<__half>(workspace, p.off_x16);
     float *G = ws_at<float>(workspace, p.off_G);
     float *U = ws_at<float>(workspace, p.off_U);
@@ -406,7 +405,7 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
 
     trace_point(0, s);
     cudaError_t err = launch_route(logits, T, p.E, top_k, renorm, ids, w, offsets, perm, pos, active, nact, x, x16,
-                                   p.H, s, true);
+                                   p.H, errw, s, true);
     if (err != cudaSuccess)
         return VQ_ERR_CUDA;
     trace_point(1, s);
@@ -474,6 +473,20 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     err = launch_combine(D, p.sb, tk * p.H, w, pos, T, top_k, p.H, y, y_dtype, s, true);
     trace_point(5, s);
     return cuda_status(err);
+}
+
+vq_status vq_moe_check(const void *workspace, void *stream)
+{
+    if (!workspace || !aligned(workspace, 256))
+        return VQ_ERR_WORKSPACE;
+    int word = 0;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess)
+        return cuda_status(e);
+    return word == 0 ? VQ_OK : VQ_ERR_DEVICE_CHECK;
 }
 
 vq_status vq_moe_prefill(const vq_moe_layer *L, const uint16_t *x, int32_t T, const float *logits, int32_t top_k,

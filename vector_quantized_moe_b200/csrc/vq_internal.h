@@ -65,10 +65,11 @@ int gemv_choose_slices(const ModDev *mods, int nmod, long n_act);
 size_t gemv_smem_bytes(const ModDev &m);
 
 // Routing + bucketing. pos = inverse of perm; active/n_active as above (may be NULL).
-// When x is not NULL the same launch also writes x16 = fp16(x) [T, H].
+// When x is not NULL the same launch also writes x16 = fp16(x) [T, H]; when
+// err is not NULL it is cleared.
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int32_t *ids, float *w,
                          int32_t *offsets, int32_t *perm, int32_t *pos, int32_t *active, int32_t *n_active,
-                         const uint16_t *x, __half *x16, int H, cudaStream_t s, bool pdl);
+                         const uint16_t *x, __half *x16, int H, int *err, cudaStream_t s, bool pdl);
 
 // h[q, c] = fp16( silu(sum_s G[s, q, c]) * sum_s U[s, q, c] )
 cudaError_t launch_swiglu(const float *G, const float *U, int slices, long slice_stride, int slots, int inter,
@@ -90,14 +91,17 @@ bool tma_map_2d(CUtensorMap *map, CUtensorMapDataType dtype, int elem_bytes, con
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Routing tables at the front of a MoE workspace (each section 256-byte aligned).
+// Front of a MoE workspace (each section 256-byte aligned): the device error
+// word at offset 0 (cleared by the routing kernel, set by a kernel whose
+// bounded wait gave up), then the routing tables.
 struct RoutingLayout {
-    size_t ids, w, offsets, perm, pos, active, nact;
+    size_t err, ids, w, offsets, perm, pos, active, nact;
 };
 inline RoutingLayout plan_routing(size_t &o, int T, int k, int E)
 {
     RoutingLayout r;
     const size_t tk = (size_t)T * k;
+    r.err = o;     o = align_up(o + 4, 256);
     r.ids = o;     o = align_up(o + tk * 4, 256);
     r.w = o;       o = align_up(o + tk * 4, 256);
     r.offsets = o; o = align_up(o + (size_t)(E + 1) * 4, 256);

@@ -635,7 +635,7 @@ cudaError_t dispatch_gemm(const PrefillArgs &a, int d, int bits, int ctas, uint3
 
 struct PrefillPlan {
     RoutingLayout r;
-    size_t err, xg, h, dp, total;
+    size_t xg, h, dp, total;
 };
 
 PrefillPlan plan_prefill(const vq_moe_layer *L, int T, int k)
@@ -644,7 +644,6 @@ PrefillPlan plan_prefill(const vq_moe_layer *L, int T, int k)
     size_t o = 0;
     p.r = plan_routing(o, T, k, L->gate.E);
     const size_t tk = (size_t)T * k;
-    p.err = o; o = align_up(o + 16, 256);
     p.xg = o; o = align_up(o + tk * L->gate.cols * 2, 256);
     p.h = o; o = align_up(o + tk * L->gate.rows * 2, 256);
     p.dp = o; o = align_up(o + tk * L->down.rows * 4, 256);
@@ -687,7 +686,7 @@ vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const flo
     int32_t *pos = ws_at<int32_t>(ws, p.r.pos);
     int32_t *active = ws_at<int32_t>(ws, p.r.active);
     int32_t *nact = ws_at<int32_t>(ws, p.r.nact);
-    int *err = ws_at<int>(ws, p.err);
+    int *err = ws_at<int>(ws, p.r.err);
     __half *xg = ws_at<__half>(ws, p.xg);
     __half *hh = ws_at<__half>(ws, p.h);
     float *dp = ws_at<float>(ws, p.dp);
@@ -695,10 +694,8 @@ vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const flo
 
     trace_point(0, s);
     cudaError_t e = launch_route(logits, T, E, k, renorm, ids, w, offsets, perm, pos, active, nact, nullptr, nullptr, 0,
-                                 s, true);
+                                 err, s, true);
     if (e != cudaSuccess)
-        return VQ_ERR_CUDA;
-    if (cudaMemsetAsync(err, 0, 4, s) != cudaSuccess)
         return VQ_ERR_CUDA;
     trace_point(1, s);
     {

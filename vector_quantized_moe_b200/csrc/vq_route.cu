@@ -219,9 +219,13 @@ __device__ void convert_rows(const uint16_t *x, __half *x16, int t0, int t1, int
         dst[i] = bf16x2_to_f16x2(src[i]);
 }
 
-__device__ __forceinline__ int bucket_chunks(int E)
+// Warps that scatter in parallel: one per 256 pairs (at most one per warp of the CTA).
+__host__ __device__ __forceinline__ int bucket_chunks(int E, int npairs)
 {
-    return E <= BUCKET_MAX_E_PARALLEL ? ROUTE_THREADS / 32 : 1;
+    if (E > BUCKET_MAX_E_PARALLEL)
+        return 1;
+    const int c = (npairs + 255) / 256;
+    return c < 1 ? 1 : (c > ROUTE_THREADS / 32 ? ROUTE_THREADS / 32 : c);
 }
 
 // Small T: one CTA routes every token and buckets the pairs.
@@ -229,14 +233,16 @@ __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_fused_kernel(const flo
                                                                       int renorm, int32_t *ids, float *w,
                                                                       int32_t *offsets, int32_t *perm, int32_t *pos,
                                                                       int32_t *active, int32_t *n_active,
-                                                                      const uint16_t *x, __half *x16, int H)
+                                                                      const uint16_t *x, __half *x16, int H, int *err)
 {
     extern __shared__ int32_t hist[];
     grid_dep_wait();
+    if (err && threadIdx.x == 0)
+        *err = 0;
     convert_rows(x, x16, 0, T, H);
     route_range(logits, 0, T, E, k, renorm, ids, w);
     __syncthreads();
-    bucket(ids, T * k, E, offsets, perm, pos, active, n_active, hist, bucket_chunks(E));
+    bucket(ids, T * k, E, offsets, perm, pos, active, n_active, hist, bucket_chunks(E, T * k));
 }
 
 // Large T: many CTAs route, then one CTA buckets.
@@ -244,9 +250,11 @@ constexpr int ROUTE_TOKENS_PER_CTA = 256;
 
 __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_topk_kernel(const float *logits, int T, int E, int k,
                                                                      int renorm, int32_t *ids, float *w,
-                                                                     const uint16_t *x, __half *x16, int H)
+                                                                     const uint16_t *x, __half *x16, int H, int *err)
 {
     grid_dep_wait();
+    if (err && blockIdx.x == 0 && threadIdx.x == 0)
+        *err = 0;
     const int t0 = blockIdx.x * ROUTE_TOKENS_PER_CTA;
     convert_rows(x, x16, t0, min(T, t0 + ROUTE_TOKENS_PER_CTA), H);
     route_range(logits, t0, min(T, t0 + ROUTE_TOKENS_PER_CTA), E, k, renorm, ids, w);
@@ -258,7 +266,7 @@ __global__ void __launch_bounds__(ROUTE_THREADS) vq_bucket_kernel(const int32_t 
 {
     extern __shared__ int32_t hist[];
     grid_dep_wait();
-    bucket(ids, npairs, E, offsets, perm, pos, active, n_active, hist, bucket_chunks(E));
+    bucket(ids, npairs, E, offsets, perm, pos, active, n_active, hist, bucket_chunks(E, npairs));
 }
 
 template <typename K, typename... Args>
@@ -281,7 +289,7 @@ cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
 
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int32_t *ids, float *w,
                          int32_t *offsets, int32_t *perm, int32_t *pos, int32_t *active, int32_t *n_active,
-                         const uint16_t *x, __half *x16, int H, cudaStream_t s, bool pdl)
+                         const uint16_t *x, __half *x16, int H, int *errw, cudaStream_t s, bool pdl)
 {
     static bool attr_set = false;
     if (!attr_set) {
@@ -293,14 +301,14 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
             return err;
         attr_set = true;
     }
-    const int chunks = E <= BUCKET_MAX_E_PARALLEL ? ROUTE_THREADS / 32 : 1;
+    const int chunks = bucket_chunks(E, T * k);
     const size_t smem = (size_t)chunks * E * sizeof(int32_t);
     if (T <= ROUTE_TOKENS_PER_CTA)
         return launch_ex(vq_route_fused_kernel, dim3(1), dim3(ROUTE_THREADS), smem, s, pdl, logits, T, E, k, renorm,
-                         ids, w, offsets, perm, pos, active, n_active, x, x16, H);
+                         ids, w, offsets, perm, pos, active, n_active, x, x16, H, errw);
     const int ctas = (T + ROUTE_TOKENS_PER_CTA - 1) / ROUTE_TOKENS_PER_CTA;
     cudaError_t err = launch_ex(vq_route_topk_kernel, dim3(ctas), dim3(ROUTE_THREADS), 0, s, pdl, logits, T, E, k,
-                                renorm, ids, w, x, x16, H);
+                                renorm, ids, w, x, x16, H, errw);
     if (err != cudaSuccess)
         return err;
     return launch_ex(vq_bucket_kernel, dim3(1), dim3(ROUTE_THREADS), smem, s, pdl, (const int32_t *)ids, T * k, E,
