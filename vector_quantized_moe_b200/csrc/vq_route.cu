@@ -125,10 +125,10 @@ __device__ void route_range(const float *logits, int t_begin, int t_end, int E, 
 }
 
 // Bucketing by one CTA (pos, active and n_active may be NULL). Warp c of `chunks` handles pairs [c*P, (c+1)*P) with
-// its own histogram row, so the stable scatter runs in parallel.
-// Shared memory: hist [chunks][E] int32.
+// its own histogram row, so the stable scatter runs in parallel. `ids` may point to global or shared memory; every
+// intermediate table lives in shared memory: hist [chunks][E] and base [E + 1] int32.
 __device__ void bucket(const int32_t *ids, int npairs, int E, int32_t *offsets, int32_t *perm, int32_t *pos,
-                       int32_t *active, int32_t *n_active, int32_t *hist, int chunks)
+                       int32_t *active, int32_t *n_active, int32_t *hist, int32_t *base, int chunks)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int i = threadIdx.x; i < chunks * E; i += blockDim.x)
@@ -149,15 +149,15 @@ __device__ void bucket(const int32_t *ids, int npairs, int E, int32_t *offsets, 
             hist[c * E + e] = run;
             run += v;
         }
-        offsets[e] = run;   // count for now
+        base[e] = run;   // count for now
     }
     __syncthreads();
     if (warp == 0) {
         int run = 0, act = 0;
         const unsigned lt = (1u << lane) - 1u;
-        for (int base = 0; base < E; base += 32) {
-            const int e = base + lane;
-            const int c = e < E ? offsets[e] : 0;
+        for (int b = 0; b < E; b += 32) {
+            const int e = b + lane;
+            const int c = e < E ? base[e] : 0;
             int incl = c;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -165,8 +165,10 @@ __device__ void bucket(const int32_t *ids, int npairs, int E, int32_t *offsets, 
                 if (lane >= o)
                     incl += v;
             }
-            if (e < E)
+            if (e < E) {
+                base[e] = run + incl - c;
                 offsets[e] = run + incl - c;
+            }
             const unsigned ball = __ballot_sync(0xFFFFFFFFu, c > 0);
             if (c > 0 && active)
                 active[act + __popc(ball & lt)] = e;
@@ -174,6 +176,7 @@ __device__ void bucket(const int32_t *ids, int npairs, int E, int32_t *offsets, 
             run += __shfl_sync(0xFFFFFFFFu, incl, 31);
         }
         if (lane == 0) {
+            base[E] = run;
             offsets[E] = run;
             if (n_active)
                 *n_active = act;
@@ -181,14 +184,14 @@ __device__ void bucket(const int32_t *ids, int npairs, int E, int32_t *offsets, 
     }
     __syncthreads();
     for (int i = threadIdx.x; i < chunks * E; i += blockDim.x)
-        hist[i] += offsets[i % E];
+        hist[i] += base[i % E];
     __syncthreads();
     if (warp < chunks) {
         int32_t *cur = hist + warp * E;
         const int p0 = warp * per, p1 = min(npairs, p0 + per);
         const unsigned lt = (1u << lane) - 1u;
-        for (int base = p0; base < p1; base += 32) {
-            const int p = base + lane;
+        for (int b = p0; b < p1; b += 32) {
+            const int p = b + lane;
             const bool v = p < p1;
             const int e = v ? ids[p] : -1;
             const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
@@ -208,15 +211,33 @@ __device__ void bucket(const int32_t *ids, int npairs, int E, int32_t *offsets, 
 
 // x16[t, c] = fp16(x[t, c]) for the tokens [t0, t1) (the tensor-core kernels
 // read fp16 activations; bf16 -> fp16 is exact for magnitudes in [2^-14, 65504]).
+// Rows of H % 8 == 0 elements are 16-byte aligned: four 16-byte loads per
+// thread are in flight before the first store.
 __device__ void convert_rows(const uint16_t *x, __half *x16, int t0, int t1, int H)
 {
     if (!x)
         return;
-    const long n = (long)(t1 - t0) * H / 2;
-    const uint32_t *src = reinterpret_cast<const uint32_t *>(x + (long)t0 * H);
-    uint32_t *dst = reinterpret_cast<uint32_t *>(x16 + (long)t0 * H);
-    for (long i = threadIdx.x; i < n; i += blockDim.x)
-        dst[i] = bf16x2_to_f16x2(src[i]);
+    const long n8 = (long)(t1 - t0) * H / 8;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (long)t0 * H);
+    uint4 *dst = reinterpret_cast<uint4 *>(x16 + (long)t0 * H);
+    const long step = blockDim.x;
+    for (long i0 = threadIdx.x; i0 < n8; i0 += 4 * step) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (i0 + u * step < n8)
+                v[u] = ldg_u128(src + i0 + u * step);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (i0 + u * step < n8) {
+                uint4 o;
+                o.x = bf16x2_to_f16x2(v[u].x);
+                o.y = bf16x2_to_f16x2(v[u].y);
+                o.z = bf16x2_to_f16x2(v[u].z);
+                o.w = bf16x2_to_f16x2(v[u].w);
+                dst[i0 + u * step] = o;
+            }
+    }
 }
 
 // Warps that scatter in parallel: one per 256 pairs (at most one per warp of the CTA).
@@ -228,6 +249,12 @@ __host__ __device__ __forceinline__ int bucket_chunks(int E, int npairs)
     return c < 1 ? 1 : (c > ROUTE_THREADS / 32 ? ROUTE_THREADS / 32 : c);
 }
 
+// Shared memory of a bucketing CTA: hist, base and (fused kernel) the pair ids.
+__host__ __device__ __forceinline__ size_t bucket_smem_ints(int E, int npairs, bool with_ids)
+{
+    return (size_t)bucket_chunks(E, npairs) * E + (size_t)E + 1 + (with_ids ? (size_t)npairs : 0);
+}
+
 // Small T: one CTA routes every token and buckets the pairs.
 __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_fused_kernel(const float *logits, int T, int E, int k,
                                                                       int renorm, int32_t *ids, float *w,
@@ -235,14 +262,19 @@ __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_fused_kernel(const flo
                                                                       int32_t *active, int32_t *n_active,
                                                                       const uint16_t *x, __half *x16, int H, int *err)
 {
-    extern __shared__ int32_t hist[];
+    extern __shared__ int32_t sm[];
+    const int npairs = T * k, chunks = bucket_chunks(E, npairs);
+    int32_t *hist = sm, *base = sm + (size_t)chunks * E, *s_ids = base + E + 1;
     grid_dep_wait();
     if (err && threadIdx.x == 0)
         *err = 0;
-    convert_rows(x, x16, 0, T, H);
     route_range(logits, 0, T, E, k, renorm, ids, w);
+    convert_rows(x, x16, 0, T, H);
     __syncthreads();
-    bucket(ids, T * k, E, offsets, perm, pos, active, n_active, hist, bucket_chunks(E, T * k));
+    for (int p = threadIdx.x; p < npairs; p += blockDim.x)
+        s_ids[p] = ids[p];   // written by this CTA above; read back once
+    __syncthreads();
+    bucket(s_ids, npairs, E, offsets, perm, pos, active, n_active, hist, base, chunks);
 }
 
 // Large T: many CTAs route, then one CTA buckets.
@@ -264,9 +296,10 @@ __global__ void __launch_bounds__(ROUTE_THREADS) vq_bucket_kernel(const int32_t 
                                                                  int32_t *offsets, int32_t *perm, int32_t *pos,
                                                                  int32_t *active, int32_t *n_active)
 {
-    extern __shared__ int32_t hist[];
+    extern __shared__ int32_t sm[];
+    const int chunks = bucket_chunks(E, npairs);
     grid_dep_wait();
-    bucket(ids, npairs, E, offsets, perm, pos, active, n_active, hist, bucket_chunks(E, npairs));
+    bucket(ids, npairs, E, offsets, perm, pos, active, n_active, sm, sm + (size_t)chunks * E, chunks);
 }
 
 template <typename K, typename... Args>
@@ -301,17 +334,17 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
             return err;
         attr_set = true;
     }
-    const int chunks = bucket_chunks(E, T * k);
-    const size_t smem = (size_t)chunks * E * sizeof(int32_t);
     if (T <= ROUTE_TOKENS_PER_CTA)
-        return launch_ex(vq_route_fused_kernel, dim3(1), dim3(ROUTE_THREADS), smem, s, pdl, logits, T, E, k, renorm,
+        return launch_ex(vq_route_fused_kernel, dim3(1), dim3(ROUTE_THREADS),
+                         bucket_smem_ints(E, T * k, true) * sizeof(int32_t), s, pdl, logits, T, E, k, renorm,
                          ids, w, offsets, perm, pos, active, n_active, x, x16, H, errw);
     const int ctas = (T + ROUTE_TOKENS_PER_CTA - 1) / ROUTE_TOKENS_PER_CTA;
     cudaError_t err = launch_ex(vq_route_topk_kernel, dim3(ctas), dim3(ROUTE_THREADS), 0, s, pdl, logits, T, E, k,
                                 renorm, ids, w, x, x16, H, errw);
     if (err != cudaSuccess)
         return err;
-    return launch_ex(vq_bucket_kernel, dim3(1), dim3(ROUTE_THREADS), smem, s, pdl, (const int32_t *)ids, T * k, E,
+    return launch_ex(vq_bucket_kernel, dim3(1), dim3(ROUTE_THREADS), bucket_smem_ints(E, T * k, false) * sizeof(int32_t),
+                     s, pdl, (const int32_t *)ids, T * k, E,
                      offsets, perm, pos, active, n_active);
 }
 
