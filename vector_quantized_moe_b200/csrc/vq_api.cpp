@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -69,7 +70,9 @@ vq_status cuda_status(cudaError_t e)
 
 struct DecodePlan {
     int T, k, E, H, I;
-    int sa, sb;                  // slices of the gate/up and down passes
+    int sa, sb;                  // output slices of the gate/up and down passes
+    GemvPlan pg, pu, pd;         // GEMV plans of gate, up (pg covers both when they share a launch) and down
+    bool gu_shared;              // gate and up in one launch
     RoutingLayout r;
     size_t off_x16, off_G, off_U, off_h, off_D;
     size_t total;
@@ -98,13 +101,22 @@ DecodePlan plan_decode(const vq_moe_layer *L, int T, int k)
     p.E = L->gate.E;
     p.H = L->gate.cols;
     p.I = L->gate.rows;
-    const long n_act = std::min<long>(p.E, (long)T * k);
+    // expected experts with tokens under uniform routing (the plan's size hint;
+    // any actual routing is handled correctly)
+    const double n_exp = p.E * (1.0 - std::pow(1.0 - (double)k / p.E, (double)T));
     const ModDev gu[2] = {make_moddev(L->gate), make_moddev(L->up)};
     const ModDev dn = make_moddev(L->down);
-    const bool same = gu[0].d == gu[1].d && gu[0].bits == gu[1].bits && gu[0].rep == gu[1].rep;
-    p.sa = same ? gemv_choose_slices(gu, 2, n_act)
-                : std::min(gemv_choose_slices(&gu[0], 1, n_act), gemv_choose_slices(&gu[1], 1, n_act));
-    p.sb = gemv_choose_slices(&dn, 1, n_act);
+    p.gu_shared = gu[0].d == gu[1].d && gu[0].bits == gu[1].bits && gu[0].rep == gu[1].rep;
+    if (p.gu_shared) {
+        p.pg = p.pu = gemv_plan(gu, 2, n_exp);
+    } else {
+        const int s = std::max(gemv_plan(&gu[0], 1, n_exp).slices, gemv_plan(&gu[1], 1, n_exp).slices);
+        p.pg = gemv_plan(&gu[0], 1, n_exp, s);
+        p.pu = gemv_plan(&gu[1], 1, n_exp, s);
+    }
+    p.pd = gemv_plan(&dn, 1, n_exp);
+    p.sa = p.pg.slices;
+    p.sb = p.pd.slices;
     size_t o = 0;
     p.r = plan_routing(o, T, k, p.E);
     const size_t tk = (size_t)T * k;
@@ -331,6 +343,7 @@ vq_status vq_gemv(const vq_module *m, int32_t expert, const uint16_t *x, int32_t
     a.expert = expert;
     a.T = T;
     a.slices = 1;
+    a.min_units = 0;
     a.out[0] = y;
     a.out[1] = y;
     a.out_dtype = y_dtype;
@@ -346,7 +359,8 @@ vq_status vq_route(const float *logits, int32_t T, int32_t E, int32_t top_k, int
         top_k > std::min(E, 32) || (long)T * top_k >= (1L << 31))
         return VQ_ERR_ARG;
     return cuda_status(launch_route(logits, T, E, top_k, renorm, ids, weights, offsets, perm, nullptr, nullptr,
-                                    nullptr, nullptr, nullptr, 0, nullptr, (cudaStream_t)stream, false));
+                                    nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, (cudaStream_t)stream,
+                                    false));
 }
 
 size_t vq_moe_workspace_size(const vq_moe_layer *L, int32_t T, int32_t top_k, int32_t mode)
@@ -404,8 +418,10 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     const long tk = (long)T * top_k;
 
     trace_point(0, s);
-    cudaError_t err = launch_route(logits, T, p.E, top_k, renorm, ids, w, offsets, perm, pos, active, nact, x, x16,
-                                   p.H, errw, s, true);
+    int2 *passes = ws_at<int2>(workspace, p.r.passes);
+    int32_t *npass = ws_at<int32_t>(workspace, p.r.npass);
+    cudaError_t err = launch_route(logits, T, p.E, top_k, renorm, ids, w, offsets, perm, pos, active, nact, passes,
+                                   npass, x, x16, p.H, errw, s, true);
     if (err != cudaSuccess)
         return VQ_ERR_CUDA;
     trace_point(1, s);
@@ -421,13 +437,15 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     a.top_k = top_k;
     a.active = active;
     a.n_active = nact;
+    a.passes = passes;
+    a.n_passes = npass;
     a.slices = p.sa;
+    a.min_units = p.pg.min_units;
     a.out_dtype = VQ_F32;
     a.out_slice_stride = tk * p.I;
     a.err = errw;
     const ModDev mg = make_moddev(L->gate), mu = make_moddev(L->up);
-    const bool same = mg.d == mu.d && mg.bits == mu.bits && mg.rep == mu.rep;
-    if (same) {
+    if (p.gu_shared) {
         a.mod[0] = mg;
         a.mod[1] = mu;
         a.nmod = 2;
@@ -441,6 +459,7 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
         err = launch_gemv(a, s, true);
         if (err == cudaSuccess) {
             a.mod[0] = a.mod[1] = mu;
+            a.min_units = p.pu.min_units;
             a.out[0] = a.out[1] = U;
             err = launch_gemv(a, s, true);
         }
@@ -463,6 +482,7 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     b.act_by_slot = 1;
     b.act_rows = tk;
     b.slices = p.sb;
+    b.min_units = p.pd.min_units;
     b.out[0] = b.out[1] = D;
     b.out_slice_stride = tk * p.H;
     err = launch_gemv(b, s, true);

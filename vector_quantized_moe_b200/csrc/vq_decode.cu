@@ -19,6 +19,9 @@
 // decodes its own codes. Inside a group the four k16 steps all lie in the
 // group, so the tensor core sums exactly one scale group per step and the
 // fp32 scale is applied once per group to the partial sums.
+#include <algorithm>
+#include <cmath>
+
 #include "vq_device.cuh"
 #include "vq_internal.h"
 #include "vq_sm100.cuh"
@@ -200,7 +203,6 @@ __global__ void __launch_bounds__(GEMV_THREADS, 2) vq_grouped_gemv_kernel(const 
     const ModDev m0 = FAST ? a.mod[0] : (blockIdx.y == 0 ? a.mod[0] : a.mod[1]);
     const int nblk = (m0.rows + 31) >> 5;
     const int S = a.slices;
-    const int gps = m0.ngroups / S;
     const long n_items = (long)n_act * nblk * S * cta_mods;
 
     for (long it = gwarp; it < n_items; it += nwarps) {
@@ -228,7 +230,8 @@ __global__ void __launch_bounds__(GEMV_THREADS, 2) vq_grouped_gemv_kernel(const 
             const int r = blk * 32 + 8 * i + g;
             prow[i] = r < m.rows ? (int)live_row(m.bitmap, m.rank, m.bm_words, m.rows, e, r) : -1;
         }
-        const int gbeg = slice * gps, gend = gbeg + gps;
+        // slice s covers groups [s * ngroups / S, (s + 1) * ngroups / S) (possibly none)
+        const int gbeg = (int)((long)slice * m.ngroups / S), gend = (int)((long)(slice + 1) * m.ngroups / S);
 
         for (int tok0 = 0; tok0 < n; tok0 += 8) {
             const bool has_tok = tok0 + g < n;
@@ -355,21 +358,37 @@ __global__ void __launch_bounds__(GEMV_THREADS, 2) vq_grouped_gemv_kernel(const 
 
 // ------------------------------------------------------------ TMA-fed grouped GEMV
 //
-// The same decomposition, with the packed codes streamed by TMA through a
-// ring of shared-memory stages instead of per-lane global loads. A CTA has 8
-// consumer warps (32 rows each, 256 rows per work item) and one producer
-// warp whose lane 0 issues one 2D tensor load per stage: 256 rows x CG
-// groups of codes. Consumers read their lane-quarters from shared memory.
-// For d=2/8-bit codes a stage row is 128 bytes loaded with the 128-byte
-// swizzle, and m16 row g of a warp is weight row sigma(g) (even rows in the
-// first half-warp, odd rows in the second), so a warp's 8-byte code reads hit
-// distinct banks. Each wait on a stage barrier is bounded.
+// The same warp-level decomposition, with the packed codes, the group scales
+// and the token tile's activations streamed by TMA through a ring of
+// shared-memory stages of 256 weight rows x CG scale groups. A CTA has 16
+// consumer warps in two halves and one producer warp whose lane 0 issues the
+// stage's tensor loads. Consumer warp w takes rows [32 (w % 8), +32) of the
+// stage and half w / 8 of its groups; the two halves' partial sums of a row
+// tile meet in shared memory when a piece of work ends. For d=2/8-bit codes a
+// stage row is 128 bytes loaded with the 128-byte swizzle, and m16 row g of a
+// warp is weight row sigma(g) (even rows in the first half-warp, odd rows in
+// the second), so a warp's 8-byte code reads hit distinct banks. Each wait on
+// a barrier is bounded.
+//
+// Work split. A work item is (token tile, module, 256-row block) and has
+// spp = groups / CG stages. The stages of all items form one sequence that is
+// cut into contiguous ranges of L stages, one per CTA, so every CTA streams
+// about the same number of bytes whatever the number of items. An item cut
+// between CTAs yields one partial sum per CTA (a piece), written to output
+// slice (CTA - first CTA of the item); the CTA that holds the item's last
+// stage writes zeros to the slices past its piece. L >= min_units bounds the
+// pieces of an item by the slice count, and readers sum the slices in a fixed
+// order, so results do not depend on timing.
 
-constexpr int TG_CONSUMERS = 8;
+constexpr int TG_WPH = 8;                        // consumer warps per half
+constexpr int TG_CONSUMERS = 2 * TG_WPH;
 constexpr int TG_THREADS = 32 * (TG_CONSUMERS + 1);
-constexpr int TG_ROWS = 32 * TG_CONSUMERS;
-constexpr int TG_NT = 1;   // token tiles of 8 per pass (the kernel body assumes one)
+constexpr int TG_ROWS = 32 * TG_WPH;
+constexpr int TG_XCHG_BYTES = TG_WPH * 2 * 8 * 32 * 4;   // per warp pair: 2 buffers of 8 floats per lane
+constexpr int TG_BAR_BYTES = 1024;
 
+// Scale groups per stage: the codes of one row of a stage fill whole 16-byte
+// units, and the count is even so the two halves get the same share.
 __host__ __device__ constexpr int tg_stage_groups(int d, int bits)
 {
     if (d == 2 && bits == 8)
@@ -378,13 +397,14 @@ __host__ __device__ constexpr int tg_stage_groups(int d, int bits)
     int cg = 1;
     while ((cg * gb) % 128)
         ++cg;
-    return cg;
+    return cg % 2 ? 2 * cg : cg;
 }
 
 template <int D, int BITS>
 struct TGeo {
     static constexpr bool SWZ = (D == 2 && BITS == 8);
     static constexpr int CG = tg_stage_groups(D, BITS);
+    static constexpr int HG = CG / 2;               // groups of one half
     static constexpr int GB = (64 / D) * BITS;      // bits per row per group
     static constexpr int SRB = CG * GB / 8;         // bytes per row per stage
     static constexpr int ACOLS = CG * 64;           // activation columns per stage
@@ -398,7 +418,7 @@ struct GemvTmaArgs {
     GemvArgs g;
     int ns;
     uint32_t stage_bytes, off_sc, off_act;   // stage layout: codes | scales | activations
-    uint32_t off_stage, off_bar;
+    uint32_t off_stage, off_xchg, off_bar;
     int *err;
 };
 
@@ -440,12 +460,42 @@ __device__ __forceinline__ void tg_read_quarter(const uint8_t *row, int gq, int 
     }
 }
 
+// One work item as both the producer and the consumers see it.
+struct TgItem {
+    int e;    // expert
+    int q0;   // first output slot of the token tile (bucket slot, or token in single-expert mode)
+    int n;    // tokens in the tile
+    int mi;   // module
+    int rb;   // 256-row block
+};
+
+__device__ __forceinline__ TgItem tg_item(const GemvArgs &a, long item, int nrb, int cta_mods, bool fast)
+{
+    TgItem r;
+    r.rb = (int)(item % nrb);
+    const long rest = item / nrb;
+    r.mi = fast ? (int)(rest % cta_mods) : (int)blockIdx.y;
+    const long tile = fast ? rest / cta_mods : rest;
+    if (a.passes) {
+        const int2 pt = a.passes[tile];
+        r.e = pt.x & 0xFFFF;
+        r.n = pt.x >> 16;
+        r.q0 = pt.y;
+    } else {
+        r.e = a.expert;
+        r.q0 = (int)tile * VQ_PASS_TOKENS;
+        r.n = min(VQ_PASS_TOKENS, a.T - r.q0);
+    }
+    return r;
+}
+
 template <int D, int BITS>
 __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid_constant__ GemvTmaArgs A)
 {
     using G = Geo<D, BITS>;
     using TG = TGeo<D, BITS>;
     constexpr bool FAST = FastByteCodes<D, BITS>::value;
+    constexpr int GP = TG::HG >= 2 ? 2 : 1;   // groups decoded together by a warp
     const GemvArgs &a = A.g;
     extern __shared__ __align__(1024) uint8_t tg_smem_raw[];
     uint8_t *smem = tg_smem_raw;
@@ -456,9 +506,12 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
     }
     uint32_t *cbs = reinterpret_cast<uint32_t *>(smem);
     uint8_t *stages = smem + A.off_stage;
+    float *xchg = reinterpret_cast<float *>(smem + A.off_xchg);   // [pair][buffer][8][32]
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + A.off_bar);
     uint64_t *empty = full + A.ns;
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + A.ns);
+    uint64_t *xfull = empty + A.ns;          // [pair][buffer]: the second half's sums are in the buffer
+    uint64_t *xempty = xfull + 2 * TG_WPH;   // [pair][buffer]: the first half has read the buffer
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(xempty + 2 * TG_WPH);
 
     const int cta_mods = FAST ? a.nmod : 1;
     if constexpr (FAST)
@@ -471,6 +524,10 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], TG_CONSUMERS);
         }
+        for (int i = 0; i < 2 * TG_WPH; ++i) {
+            mbar_init(&xfull[i], 32);
+            mbar_init(&xempty[i], 32);
+        }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -478,70 +535,61 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
     grid_dep_wait();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const ModDev m0 = FAST ? a.mod[0] : (blockIdx.y == 0 ? a.mod[0] : a.mod[1]);
-    const int n_act = a.offsets ? *a.n_active : 1;
+    const ModDev &m0 = FAST ? a.mod[0] : (blockIdx.y == 0 ? a.mod[0] : a.mod[1]);
     const int nrb = (m0.rows + TG_ROWS - 1) / TG_ROWS;
-    const int S = a.slices;
-    const int gps = m0.ngroups / S;
-    const int spp = gps / TG::CG;
-    const long n_items = (long)n_act * nrb * S * cta_mods;
+    const int spp = m0.ngroups / TG::CG;
+    const long n_tiles = a.passes ? (long)*a.n_passes : (long)((a.T + VQ_PASS_TOKENS - 1) / VQ_PASS_TOKENS);
+    const long U = n_tiles * cta_mods * nrb * spp;
+    long L = (U + gridDim.x - 1) / gridDim.x;
+    if (L < a.min_units)
+        L = a.min_units;
+    if (a.slices == 1)
+        L = (L + spp - 1) / spp * spp;   // whole items only
+    const long u0 = min(U, (long)blockIdx.x * L);
+    const long u1 = min(U, u0 + L);
     const uint32_t stage_bytes_codes = (uint32_t)TG_ROWS * TG::SRB;
-
-    auto decode_item = [&](long it, int &slice, int &rb, int &mi, int &e, int &q0, int &n) {
-        long rest = it;
-        slice = (int)(rest % S);
-        rest /= S;
-        rb = (int)(rest % nrb);
-        rest /= nrb;
-        mi = FAST ? (int)(rest % cta_mods) : (int)blockIdx.y;
-        const int ai = FAST ? (int)(rest / cta_mods) : (int)rest;
-        e = a.offsets ? a.active[ai] : a.expert;
-        q0 = a.offsets ? a.offsets[e] : 0;
-        n = a.offsets ? a.offsets[e + 1] - q0 : a.T;
-    };
 
     if (warp == TG_CONSUMERS) {
         // ------------------------------------------------ producer: codes, scales and the
-        // activation rows of the pass's tokens for every stage, one barrier per stage
+        // activation rows of the item's tokens for every stage, one barrier per stage
         if (lane == 0) {
             uint32_t k = 0, slot = 0, ph = 0;   // stages issued; ring slot and phase of stage k
             bool ok = true;
-            for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-                int slice, rb, mi, e, q0, n;
-                decode_item(it, slice, rb, mi, e, q0, n);
-                const ModDev &m = mi == 0 ? a.mod[0] : a.mod[1];
-                const int prow0 = tg_prow0(m, e, rb * TG_ROWS);
-                const int passes = (n + 8 * TG_NT - 1) / (8 * TG_NT);
-                for (int p = 0; p < passes && ok; ++p) {
-                    const int tok0 = p * 8 * TG_NT;
-                    const int np = min(8 * TG_NT, n - tok0);
-                    int arow[8 * TG_NT];
-                    for (int i = 0; i < np; ++i) {
-                        const int q = q0 + tok0 + i;
-                        arow[i] = a.act_by_slot ? q : (a.perm ? a.perm[q] / a.top_k : tok0 + i);
+            TgItem it{};
+            int prow0 = 0, mi = 0;
+            int arow[VQ_PASS_TOKENS];
+            uint32_t tx = 0;
+            for (long u = u0; u < u1 && ok; ++u) {
+                const long item = u / spp;
+                const int j = (int)(u % spp);
+                if (u == u0 || j == 0) {
+                    it = tg_item(a, item, nrb, cta_mods, FAST);
+                    mi = it.mi;
+                    prow0 = tg_prow0(mi == 0 ? a.mod[0] : a.mod[1], it.e, it.rb * TG_ROWS);
+                    for (int i = 0; i < it.n; ++i) {
+                        const int q = it.q0 + i;
+                        arow[i] = a.act_by_slot ? q : (a.perm ? a.perm[q] / a.top_k : q);
                     }
-                    const uint32_t tx = stage_bytes_codes + (uint32_t)TG_ROWS * 16 + (uint32_t)np * TG::ACOLS * 2;
-                    for (int j = 0; j < spp; ++j) {
-                        if (!(ok = mbar_wait(&empty[slot], ph ^ 1, abort_flag, A.err, 11)))
-                            break;
-                        uint8_t *sb = stages + (size_t)slot * A.stage_bytes;
-                        mbar_expect_tx(&full[slot], tx);
-                        const int g0 = slice * gps + j * TG::CG;
-                        tma_load_2d(sb, &A.tmap[mi], g0 * TG::GB / 32, prow0, &full[slot]);
-                        tma_load_2d(sb + A.off_sc, &A.tmap_sc[mi], g0 & ~7, prow0, &full[slot]);
-                        for (int i = 0; i < np; ++i)
-                            for (int c = 0; c < TG::ACOLS; c += TG::ACW)
-                                tma_load_2d(sb + A.off_act + (size_t)i * TG::ACOLS * 2 + c * 2, &A.tmap_act,
-                                            g0 * 64 + c, arow[i], &full[slot]);
-                        ++k;
-                        if (++slot == (uint32_t)A.ns) {
-                            slot = 0;
-                            ph ^= 1;
-                        }
-                    }
+                    tx = stage_bytes_codes + (uint32_t)TG_ROWS * 16 + (uint32_t)it.n * TG::ACOLS * 2;
+                }
+                if (!(ok = mbar_wait(&empty[slot], ph ^ 1, abort_flag, A.err, 11)))
+                    break;
+                uint8_t *sb = stages + (size_t)slot * A.stage_bytes;
+                mbar_expect_tx(&full[slot], tx);
+                const int g0 = j * TG::CG;
+                tma_load_2d(sb, &A.tmap[mi], g0 * TG::GB / 32, prow0, &full[slot]);
+                tma_load_2d(sb + A.off_sc, &A.tmap_sc[mi], g0 & ~7, prow0, &full[slot]);
+                for (int i = 0; i < it.n; ++i)
+                    for (int c = 0; c < TG::ACOLS; c += TG::ACW)
+                        tma_load_2d(sb + A.off_act + (size_t)i * TG::ACOLS * 2 + c * 2, &A.tmap_act, g0 * 64 + c,
+                                    arow[i], &full[slot]);
+                ++k;
+                if (++slot == (uint32_t)A.ns) {
+                    slot = 0;
+                    ph ^= 1;
                 }
             }
-            if (!ok) {
+            if (!ok) {   // let the copies in flight land before the CTA exits
                 for (uint32_t s = 0; s < (uint32_t)A.ns && s < k; ++s) {
                     const uint32_t kk = k - 1 - s;
                     mbar_wait(&full[kk % A.ns], (kk / A.ns) & 1, abort_flag, A.err, 12);
@@ -552,177 +600,196 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
     }
 
     // ---------------------------------------------------- consumers
+    const int half = warp / TG_WPH, wr = warp % TG_WPH;
     const int g = lane >> 2, t = lane & 3;
-    uint32_t slot = 0, ph = 0;
+    uint32_t slot = 0, ph = 0, xk = 0;   // stage ring; pieces exchanged by this warp pair
     bool ok = true;
-    for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-        int slice, rb, mi, e, q0, n;
-        decode_item(it, slice, rb, mi, e, q0, n);
-        const ModDev &m = mi == 0 ? a.mod[0] : a.mod[1];
-        void *const out = mi == 0 ? a.out[0] : a.out[1];
-        const int rep = lane & (m.rep - 1);
-        const uint32_t lane_sel = (uint32_t)(mi * 128 + lane * 4);
-        const int r0 = rb * TG_ROWS;
-        const int prow0 = tg_prow0(m, e, r0);
-        int br[4], prow[4];
+    TgItem it{};
+    int br[4], prow[4];
+    int rep = 0, r0 = 0;
+    uint32_t lane_sel = 0;
+    bool has_tok = false;
+    float acc[2][4];
+    for (long u = u0; u < u1 && ok; ++u) {
+        const long item = u / spp;
+        const int j = (int)(u % spp);
+        if (u == u0 || j == 0) {
+            it = tg_item(a, item, nrb, cta_mods, FAST);
+            const ModDev &m = it.mi == 0 ? a.mod[0] : a.mod[1];
+            rep = lane & (m.rep - 1);
+            lane_sel = (uint32_t)(it.mi * 128 + lane * 4);
+            r0 = it.rb * TG_ROWS;
+            const int prow0 = tg_prow0(m, it.e, r0);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = r0 + 32 * warp + 8 * i + tg_sigma(g);
-            prow[i] = r < m.rows ? (int)live_row(m.bitmap, m.rank, m.bm_words, m.rows, e, r) : -1;
-            br[i] = prow[i] >= 0 ? prow[i] - prow0 : -1;
+            for (int i = 0; i < 4; ++i) {
+                const int r = r0 + 32 * wr + 8 * i + tg_sigma(g);
+                prow[i] = r < m.rows ? (int)live_row(m.bitmap, m.rank, m.bm_words, m.rows, it.e, r) : -1;
+                br[i] = prow[i] >= 0 ? prow[i] - prow0 : -1;
+            }
+            has_tok = g < it.n;
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    acc[i][q] = 0.f;
         }
-        const int passes = (n + 8 * TG_NT - 1) / (8 * TG_NT);
-        for (int p = 0; p < passes && ok; ++p) {
-            const int tok0 = p * 8 * TG_NT;
-            const int ntiles = min(TG_NT, (n - tok0 + 7) / 8);
-            bool has_tok[TG_NT];
+        const ModDev &m = it.mi == 0 ? a.mod[0] : a.mod[1];
+
+        if (!(ok = mbar_wait(&full[slot], ph, abort_flag, A.err, 13)))
+            break;
+        const uint8_t *sbase = stages + (size_t)slot * A.stage_bytes;
+        const int g0 = j * TG::CG;
+        const uint16_t *ssc = reinterpret_cast<const uint16_t *>(sbase + A.off_sc) + (g0 & 7);
+        const uint8_t *sact = sbase + A.off_act;
 #pragma unroll
-            for (int nt = 0; nt < TG_NT; ++nt)
-                has_tok[nt] = nt < ntiles && tok0 + 8 * nt + g < n;
-            float acc[TG_NT][2][4];
+        for (int gh = 0; gh < TG::HG; gh += GP) {
+            uint32_t cw[GP][4][G::LW];
+            int co[GP][4];
+            uint32_t bw[GP][8];
+            float sv[GP][4];
 #pragma unroll
-            for (int nt = 0; nt < TG_NT; ++nt)
+            for (int uu = 0; uu < GP; ++uu) {
+                const int gq = half * TG::HG + gh + uu;   // group within the stage
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if (br[i] >= 0) {
+                        tg_read_quarter<D, BITS>(sbase + (size_t)br[i] * TG::SRB, gq, t, br[i], cw[uu][i],
+                                                 co[uu][i]);
+                        sv[uu][i] = f16_to_f32(ssc[(size_t)br[i] * 8 + gq]);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < G::LW; ++q)
+                            cw[uu][i][q] = 0u;
+                        co[uu][i] = 0;
+                        sv[uu][i] = 0.f;
+                    }
+                }
+                uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+                if (has_tok) {
+                    const uint4 *ap =
+                        reinterpret_cast<const uint4 *>(sact + (size_t)g * TG::ACOLS * 2 + gq * 128 + t * 32);
+                    v0 = ap[0];
+                    v1 = ap[1];
+                }
+                bw[uu][0] = v0.x; bw[uu][1] = v0.y; bw[uu][2] = v0.z; bw[uu][3] = v0.w;
+                bw[uu][4] = v1.x; bw[uu][5] = v1.y; bw[uu][6] = v1.z; bw[uu][7] = v1.w;
+                if (a.act_bf16) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        bw[uu][q] = bf16x2_to_f16x2(bw[uu][q]);
+                }
+            }
+            if (gh + GP >= TG::HG) {   // every read of this stage by the warp is done
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&empty[slot]);
+            }
+            uint32_t c[GP][4][G::CODES];
+            if constexpr (!FAST) {
+#pragma unroll
+                for (int uu = 0; uu < GP; ++uu)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        extract_codes<D, BITS>(cw[uu][i], co[uu][i], c[uu][i]);
+            }
+            float tmp[GP][2][4];
+#pragma unroll
+            for (int uu = 0; uu < GP; ++uu)
 #pragma unroll
                 for (int i = 0; i < 2; ++i)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        acc[nt][i][j] = 0.f;
-
-            for (int j = 0; j < spp; ++j) {
-                const int g0 = slice * gps + j * TG::CG;
-                if (!(ok = mbar_wait(&full[slot], ph, abort_flag, A.err, 13)))
-                    break;
-                const uint8_t *sbase = stages + (size_t)slot * A.stage_bytes;
-                const uint16_t *ssc = reinterpret_cast<const uint16_t *>(sbase + A.off_sc) + (g0 & 7);
-                const uint8_t *sact = sbase + A.off_act;
-                // groups are taken GP at a time so that a warp has 2 * GP independent
-                // accumulation chains in flight
-                constexpr int GP = TG::CG >= 2 ? 2 : 1;
+                    for (int q = 0; q < 4; ++q)
+                        tmp[uu][i][q] = 0.f;
 #pragma unroll
-                for (int gp = 0; gp < TG::CG; gp += GP) {
-                    uint32_t cw[GP][4][G::LW];
-                    int co[GP][4];
-                    uint32_t bw[GP][8];
-                    float sv[GP][4];
+            for (int s = 0; s < 4; ++s) {
 #pragma unroll
-                    for (int u = 0; u < GP; ++u) {
-                        const int gq = gp + u;
+                for (int uu = 0; uu < GP; ++uu) {
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            if (br[i] >= 0) {
-                                tg_read_quarter<D, BITS>(sbase + (size_t)br[i] * TG::SRB, gq, t, br[i], cw[u][i],
-                                                         co[u][i]);
-                                sv[u][i] = f16_to_f32(ssc[(size_t)br[i] * 8 + gq]);
-                            } else {
+                    for (int rt = 0; rt < 2; ++rt) {
+                        uint32_t Aw[4];
+                        if constexpr (FAST) {
+                            const char *cbb = reinterpret_cast<const char *>(cbs);
 #pragma unroll
-                                for (int q = 0; q < G::LW; ++q)
-                                    cw[u][i][q] = 0u;
-                                co[u][i] = 0;
-                                sv[u][i] = 0.f;
+                            for (int h = 0; h < 2; ++h) {
+                                const uint32_t sel = 0x5504u | ((uint32_t)(2 * (s & 1) + h) << 4);
+                                Aw[2 * h] = *reinterpret_cast<const uint32_t *>(
+                                    cbb + __byte_perm(cw[uu][2 * rt][s >> 1], lane_sel, sel));
+                                Aw[2 * h + 1] = *reinterpret_cast<const uint32_t *>(
+                                    cbb + __byte_perm(cw[uu][2 * rt + 1][s >> 1], lane_sel, sel));
                             }
+                        } else {
+                            a_words<D>(cbs, m.log_rep, rep, c[uu][2 * rt], s, Aw[0], Aw[2]);
+                            a_words<D>(cbs, m.log_rep, rep, c[uu][2 * rt + 1], s, Aw[1], Aw[3]);
                         }
-                        uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
-                        if (has_tok[0]) {
-                            const uint4 *ap =
-                                reinterpret_cast<const uint4 *>(sact + (size_t)g * TG::ACOLS * 2 + gq * 128 + t * 32);
-                            v0 = ap[0];
-                            v1 = ap[1];
-                        }
-                        bw[u][0] = v0.x; bw[u][1] = v0.y; bw[u][2] = v0.z; bw[u][3] = v0.w;
-                        bw[u][4] = v1.x; bw[u][5] = v1.y; bw[u][6] = v1.z; bw[u][7] = v1.w;
-                        if (a.act_bf16) {
-#pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                bw[u][q] = bf16x2_to_f16x2(bw[u][q]);
-                        }
+                        mma_16816(tmp[uu][rt], Aw, bw[uu][2 * s], bw[uu][2 * s + 1]);
                     }
-                    if (gp + GP >= TG::CG) {   // every code read of this stage is done
-                        __syncwarp();
-                        if (lane == 0)
-                            mbar_arrive(&empty[slot]);
-                    }
-                    uint32_t c[GP][4][G::CODES];
-                    if constexpr (!FAST) {
-#pragma unroll
-                        for (int u = 0; u < GP; ++u)
-#pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                extract_codes<D, BITS>(cw[u][i], co[u][i], c[u][i]);
-                    }
-                    float tmp[GP][2][4];
-#pragma unroll
-                    for (int u = 0; u < GP; ++u)
-#pragma unroll
-                        for (int i = 0; i < 2; ++i)
-#pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                tmp[u][i][q] = 0.f;
-#pragma unroll
-                    for (int s = 0; s < 4; ++s) {
-#pragma unroll
-                        for (int u = 0; u < GP; ++u) {
-#pragma unroll
-                            for (int rt = 0; rt < 2; ++rt) {
-                                uint32_t Aw[4];
-                                if constexpr (FAST) {
-                                    const char *cbb = reinterpret_cast<const char *>(cbs);
-#pragma unroll
-                                    for (int h = 0; h < 2; ++h) {
-                                        const uint32_t sel = 0x5504u | ((uint32_t)(2 * (s & 1) + h) << 4);
-                                        Aw[2 * h] = *reinterpret_cast<const uint32_t *>(
-                                            cbb + __byte_perm(cw[u][2 * rt][s >> 1], lane_sel, sel));
-                                        Aw[2 * h + 1] = *reinterpret_cast<const uint32_t *>(
-                                            cbb + __byte_perm(cw[u][2 * rt + 1][s >> 1], lane_sel, sel));
-                                    }
-                                } else {
-                                    a_words<D>(cbs, m.log_rep, rep, c[u][2 * rt], s, Aw[0], Aw[2]);
-                                    a_words<D>(cbs, m.log_rep, rep, c[u][2 * rt + 1], s, Aw[1], Aw[3]);
-                                }
-                                if (ntiles > 0)
-                                    mma_16816(tmp[u][rt], Aw, bw[u][2 * s], bw[u][2 * s + 1]);
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int u = 0; u < GP; ++u)
-#pragma unroll
-                        for (int rt = 0; rt < 2; ++rt) {
-                            const float slo = sv[u][2 * rt], shi = sv[u][2 * rt + 1];
-                            acc[0][rt][0] = fmaf(tmp[u][rt][0], slo, acc[0][rt][0]);
-                            acc[0][rt][1] = fmaf(tmp[u][rt][1], slo, acc[0][rt][1]);
-                            acc[0][rt][2] = fmaf(tmp[u][rt][2], shi, acc[0][rt][2]);
-                            acc[0][rt][3] = fmaf(tmp[u][rt][3], shi, acc[0][rt][3]);
-                        }
-                }
-                if (++slot == (uint32_t)A.ns) {
-                    slot = 0;
-                    ph ^= 1;
                 }
             }
-            if (!ok)
-                break;
-            // lane holds rows sigma(g) (+8i) for bucket tokens tok0 + 8nt + 2t + {0, 1}
 #pragma unroll
-            for (int nt = 0; nt < TG_NT; ++nt)
+            for (int uu = 0; uu < GP; ++uu)
 #pragma unroll
-                for (int rt = 0; rt < 2; ++rt)
-#pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
-                        const int i = 2 * rt + hf;
-                        const int r = r0 + 32 * warp + 8 * i + tg_sigma(g);
-                        if (r >= m.rows)
-                            continue;
-#pragma unroll
-                        for (int cc = 0; cc < 2; ++cc) {
-                            const int tk = tok0 + 8 * nt + 2 * t + cc;
-                            if (nt >= ntiles || tk >= n)
-                                continue;
-                            const float v = prow[i] >= 0 ? acc[nt][rt][2 * hf + cc] : 0.f;
-                            store_out(out, a.out_dtype,
-                                      (long)slice * a.out_slice_stride + (long)(q0 + tk) * m.rows + r, v);
-                        }
-                    }
+                for (int rt = 0; rt < 2; ++rt) {
+                    const float slo = sv[uu][2 * rt], shi = sv[uu][2 * rt + 1];
+                    acc[rt][0] = fmaf(tmp[uu][rt][0], slo, acc[rt][0]);
+                    acc[rt][1] = fmaf(tmp[uu][rt][1], slo, acc[rt][1]);
+                    acc[rt][2] = fmaf(tmp[uu][rt][2], shi, acc[rt][2]);
+                    acc[rt][3] = fmaf(tmp[uu][rt][3], shi, acc[rt][3]);
+                }
         }
+        if (++slot == (uint32_t)A.ns) {
+            slot = 0;
+            ph ^= 1;
+        }
+
+        if (j != spp - 1 && u != u1 - 1)
+            continue;
+        // ------------------------------------------------ end of a piece: the second half hands its
+        // sums to the first through a 2-buffer ring per warp pair; the first half adds them (always in
+        // this order) and stores the piece
+        const int xb = (int)(xk & 1);
+        const uint32_t xph = (xk >> 1) & 1;
+        ++xk;
+        float *xs = xchg + (size_t)(wr * 2 + xb) * 8 * 32;
+        if (half == 1) {
+            if (!(ok = mbar_wait(&xempty[wr * 2 + xb], xph ^ 1, abort_flag, A.err, 14)))
+                break;
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+                xs[v * 32 + lane] = acc[v >> 2][v & 3];
+            mbar_arrive(&xfull[wr * 2 + xb]);
+            continue;
+        }
+        if (!(ok = mbar_wait(&xfull[wr * 2 + xb], xph, abort_flag, A.err, 15)))
+            break;
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+            acc[v >> 2][v & 3] += xs[v * 32 + lane];
+        mbar_arrive(&xempty[wr * 2 + xb]);
+
+        void *const out = it.mi == 0 ? a.out[0] : a.out[1];
+        const int piece = (int)(blockIdx.x - (item * spp) / L);
+        const int last = j == spp - 1 ? a.slices : piece + 1;   // zeros past the item's last piece
+        // lane holds rows r0 + 32 wr + 8 i + sigma(g) for tile tokens 2t + {0, 1}
+#pragma unroll
+        for (int rt = 0; rt < 2; ++rt)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int i = 2 * rt + hf;
+                const int r = r0 + 32 * wr + 8 * i + tg_sigma(g);
+                if (r >= m.rows)
+                    continue;
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int tk = 2 * t + cc;
+                    if (tk >= it.n)
+                        continue;
+                    const float v = prow[i] >= 0 ? acc[rt][2 * hf + cc] : 0.f;
+                    const long o = (long)(it.q0 + tk) * m.rows + r;
+                    store_out(out, a.out_dtype, (long)piece * a.out_slice_stride + o, v);
+                    for (int sl = piece + 1; sl < last; ++sl)
+                        store_out(out, a.out_dtype, (long)sl * a.out_slice_stride + o, 0.f);
+                }
+            }
     }
 }
 
@@ -874,7 +941,7 @@ cudaError_t gemv_dispatch(const GemvArgs &a, cudaStream_t s, bool pdl)
 
 struct TgPlan {
     int ns;
-    uint32_t stage, off_sc, off_act, off_stage, off_bar, total;
+    uint32_t stage, off_sc, off_act, off_stage, off_xchg, off_bar, total;
 };
 
 TgPlan tg_plan(const ModDev &m)
@@ -885,20 +952,24 @@ TgPlan tg_plan(const ModDev &m)
     const uint32_t codes = (uint32_t)TG_ROWS * (uint32_t)(cg * (64 / m.d) * m.bits / 8);
     p.off_sc = codes;
     p.off_act = codes + (uint32_t)TG_ROWS * 16;
-    p.stage = (uint32_t)align_up(p.off_act + 8u * TG_NT * cg * 64 * 2, 1024);
-    const uint32_t limit = 227 * 1024 - 1024 - 256;
-    p.ns = limit > cb ? (int)std::min<uint32_t>(8, (limit - cb) / p.stage) : 0;
+    p.stage = (uint32_t)align_up(p.off_act + (uint32_t)VQ_PASS_TOKENS * cg * 64 * 2, 1024);
+    const uint32_t limit = 227 * 1024 - 1024;   // opt-in maximum less the alignment slack
+    const uint32_t fixed = cb + TG_XCHG_BYTES + TG_BAR_BYTES;
+    p.ns = limit > fixed ? (int)std::min<uint32_t>(8, (limit - fixed) / p.stage) : 0;
     p.off_stage = cb;
-    p.off_bar = cb + p.ns * p.stage;
-    p.total = p.off_bar + 16 * p.ns + 16 + 1024;
+    p.off_xchg = cb + p.ns * p.stage;
+    p.off_bar = p.off_xchg + TG_XCHG_BYTES;
+    p.total = p.off_bar + TG_BAR_BYTES + 1024;
     return p;
 }
 
-bool tg_ok(const ModDev &m, int slices)
+// The TMA kernel takes the module: 16-byte packed rows, 8-group scale rows,
+// whole stages per row and at least two stages in shared memory.
+bool tg_ok(const ModDev &m)
 {
     const int cg = tg_stage_groups(m.d, m.bits);
-    return tma_available() && m.row_words % 4 == 0 && m.ngroups % 8 == 0 && m.ngroups % slices == 0 &&
-           (m.ngroups / slices) % cg == 0 && tg_plan(m).ns >= 2;
+    return tma_available() && m.row_words % 4 == 0 && m.ngroups % 8 == 0 && m.ngroups % cg == 0 &&
+           tg_plan(m).ns >= 2;
 }
 
 template <int D, int BITS>
@@ -933,6 +1004,7 @@ cudaError_t gemv_tma_dispatch(const GemvArgs &a, cudaStream_t s, bool pdl)
     A.off_sc = p.off_sc;
     A.off_act = p.off_act;
     A.off_stage = p.off_stage;
+    A.off_xchg = p.off_xchg;
     A.off_bar = p.off_bar;
     A.err = a.err;
     auto k = vq_gemv_tma_kernel<D, BITS>;
@@ -945,6 +1017,14 @@ cudaError_t gemv_tma_dispatch(const GemvArgs &a, cudaStream_t s, bool pdl)
     return launch(k, dim3(ctas, gy), dim3(TG_THREADS), p.total, s, pdl, A);
 }
 
+bool tma_for(const ModDev *mods, int nmod)
+{
+    bool tma = true;
+    for (int i = 0; i < nmod; ++i)
+        tma = tma && tg_ok(mods[i]);
+    return tma;
+}
+
 }  // namespace
 
 size_t gemv_smem_bytes(const ModDev &m)
@@ -955,30 +1035,46 @@ size_t gemv_smem_bytes(const ModDev &m)
     return ((size_t)1 << m.bits) * (size_t)m.rep * ew * 4;
 }
 
-int gemv_choose_slices(const ModDev *mods, int nmod, long n_act)
+GemvPlan gemv_plan(const ModDev *mods, int nmod, double n_tiles_expected, int slices)
 {
     const ModDev &m = mods[0];
-    bool tma = tg_ok(m, 1);
-    for (int i = 1; i < nmod; ++i)
-        tma = tma && tg_ok(mods[i], 1);
-    const int cg = tma ? tg_stage_groups(m.d, m.bits) : 1;
-    // work items: 256-row CTA items (TMA kernel) or 32-row warp items
-    const long per = tma ? (long)((m.rows + TG_ROWS - 1) / TG_ROWS) : (long)((m.rows + 31) / 32);
-    const long target = tma ? 2L * num_sms() : 32L * num_sms();
-    const long items1 = n_act * per * nmod;
+    GemvPlan p{1, 0};
+    if (tma_for(mods, nmod)) {
+        // stage ranges of about U / CTAs; an item of spp stages then spans at most
+        // ceil((spp - 1) / L) + 1 CTAs, which sets the slice count (at most 4)
+        const int cg = tg_stage_groups(m.d, m.bits);
+        const long spp = m.ngroups / cg;
+        const bool both = m.d == 2 && m.bits == 8;
+        const int cta_mods = both ? nmod : 1;
+        const int ctas = std::max(1, num_sms() / (both ? 1 : nmod));
+        const long nrb = (m.rows + TG_ROWS - 1) / TG_ROWS;
+        const double units = std::max(1.0, n_tiles_expected) * cta_mods * nrb * spp;
+        const long L = std::max(1L, (long)std::ceil(units / ctas));
+        const long pieces = spp > 1 ? (spp - 2) / L + 2 : 1;
+        p.slices = slices > 0 ? slices : (int)std::min(4L, pieces);
+        // L >= min_units keeps the pieces of an item within the slices
+        p.min_units = p.slices > 1 ? (int)((spp - 1 + p.slices - 2) / (p.slices - 1)) : (int)spp;
+        return p;
+    }
+    // register-prefetch kernel: split the 64-column groups into slices until
+    // there are about 32 warp items per SM
+    if (slices > 0) {
+        p.slices = slices;
+        return p;
+    }
+    const long per = (m.rows + 31) / 32;
+    const long items1 = (long)std::ceil(std::max(1.0, n_tiles_expected)) * per * nmod;
     int s = 1;
-    while (m.ngroups % (2 * s) == 0 && (m.ngroups / (2 * s)) % cg == 0 && m.ngroups / (2 * s) >= 2 * cg &&
-           items1 * s < target)
+    while (m.ngroups % (2 * s) == 0 && m.ngroups / (2 * s) >= 2 && items1 * s < 32L * num_sms())
         s *= 2;
-    return s;
+    p.slices = s;
+    return p;
 }
 
 cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, bool pdl)
 {
     const ModDev &m = a.mod[0];
-    bool tma = tg_ok(m, a.slices);
-    for (int i = 1; i < a.nmod; ++i)
-        tma = tma && tg_ok(a.mod[i], a.slices);
+    const bool tma = tma_for(a.mod, a.nmod);
 #define VQ_GEMV(D_, B_)                                                        \
     if (m.d == D_ && m.bits == B_)                                             \
         return tma ? gemv_tma_dispatch<D_, B_>(a, s, pdl) : gemv_dispatch<D_, B_>(a, s, pdl);

@@ -13,6 +13,9 @@
 #define VQ_GEOMETRIES(X) \
     X(1, 3) X(1, 4) X(2, 8) X(2, 10) X(2, 11) X(4, 8) X(4, 9) X(4, 11) X(4, 13) X(8, 12)
 
+// Token tile of the decode GEMV: bucket slots contracted together per pass over a weight tile.
+#define VQ_PASS_TOKENS 8
+
 namespace vq {
 
 // A module as the kernels see it.
@@ -47,9 +50,12 @@ struct GemvArgs {
     int top_k;
     const int32_t *active;  // experts with tokens, ascending
     const int32_t *n_active;
+    const int2 *passes;     // token tiles of the buckets (route: passes / n_passes); NULL in single-expert mode
+    const int32_t *n_passes;
     int expert;             // single-expert mode
     int T;                  // single-expert mode: tokens
-    int slices;             // split of the 64-column groups (partial sums per slice)
+    int slices;             // partial-sum slices of the output (the reader sums them in order)
+    int min_units;          // TMA kernel: least weight stages per CTA (bounds the pieces of a work item)
     void *out[2];           // per module: [slices][slots][rows]
     int out_dtype;          // VQ_F32 or VQ_BF16
     long out_slice_stride;  // elements between slices
@@ -57,19 +63,27 @@ struct GemvArgs {
 };
 
 // Launches the TMA-fed kernel when the modules allow it (16-byte packed rows,
-// whole stages per slice), else the register-prefetch kernel.
+// whole stages), else the register-prefetch kernel. a.slices and a.min_units
+// must come from gemv_plan for the same modules.
 cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, bool pdl);
-// Slices of the 64-column groups for nmod modules sharing a launch and about
-// n_act experts with tokens (consistent with the kernel launch_gemv picks).
-int gemv_choose_slices(const ModDev *mods, int nmod, long n_act);
+// Output slices and least stages per CTA for nmod modules sharing a launch,
+// sized for the expected number of token tiles; slices > 0 fixes the slice
+// count instead (any count >= 1 is valid for either kernel).
+struct GemvPlan {
+    int slices;
+    int min_units;
+};
+GemvPlan gemv_plan(const ModDev *mods, int nmod, double n_tiles_expected, int slices = 0);
 size_t gemv_smem_bytes(const ModDev &m);
 
 // Routing + bucketing. pos = inverse of perm; active/n_active as above (may be NULL).
 // When x is not NULL the same launch also writes x16 = fp16(x) [T, H]; when
 // err is not NULL it is cleared.
+// passes / n_passes (may be NULL): the token tiles of the buckets, see VQ_PASS_TOKENS.
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int32_t *ids, float *w,
                          int32_t *offsets, int32_t *perm, int32_t *pos, int32_t *active, int32_t *n_active,
-                         const uint16_t *x, __half *x16, int H, int *err, cudaStream_t s, bool pdl);
+                         int2 *passes, int32_t *n_passes, const uint16_t *x, __half *x16, int H, int *err,
+                         cudaStream_t s, bool pdl);
 
 // h[q, c] = fp16( silu(sum_s G[s, q, c]) * sum_s U[s, q, c] )
 cudaError_t launch_swiglu(const float *G, const float *U, int slices, long slice_stride, int slots, int inter,
@@ -95,8 +109,14 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // word at offset 0 (cleared by the routing kernel, set by a kernel whose
 // bounded wait gave up), then the routing tables.
 struct RoutingLayout {
-    size_t err, ids, w, offsets, perm, pos, active, nact;
+    size_t err, ids, w, offsets, perm, pos, active, nact, npass, passes;
 };
+// Upper bound on the token tiles of T*k pairs over E experts.
+inline size_t max_passes(int T, int k, int E)
+{
+    const size_t tk = (size_t)T * k;
+    return tk / VQ_PASS_TOKENS + (tk < (size_t)E ? tk : (size_t)E) + 1;
+}
 inline RoutingLayout plan_routing(size_t &o, int T, int k, int E)
 {
     RoutingLayout r;
@@ -109,6 +129,8 @@ inline RoutingLayout plan_routing(size_t &o, int T, int k, int E)
     r.pos = o;     o = align_up(o + tk * 4, 256);
     r.active = o;  o = align_up(o + (size_t)E * 4, 256);
     r.nact = o;    o = align_up(o + 4, 256);
+    r.npass = o;   o = align_up(o + 4, 256);
+    r.passes = o;  o = align_up(o + max_passes(T, k, E) * 8, 256);
     return r;
 }
 

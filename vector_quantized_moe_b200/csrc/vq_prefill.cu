@@ -693,8 +693,8 @@ vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const flo
     const long tk = (long)T * k;
 
     trace_point(0, s);
-    cudaError_t e = launch_route(logits, T, E, k, renorm, ids, w, offsets, perm, pos, active, nact, nullptr, nullptr, 0,
-                                 err, s, true);
+    cudaError_t e = launch_route(logits, T, E, k, renorm, ids, w, offsets, perm, pos, active, nact, nullptr, nullptr,
+                                 nullptr, nullptr, 0, err, s, true);
     if (e != cudaSuccess)
         return VQ_ERR_CUDA;
     trace_point(1, s);

@@ -124,11 +124,14 @@ __device__ void route_range(const float *logits, int t_begin, int t_end, int E, 
         route_tokens<0>(logits, t_begin, t_end, E, k, renorm, ids, w);
 }
 
-// Bucketing by one CTA (pos, active and n_active may be NULL). Warp c of `chunks` handles pairs [c*P, (c+1)*P) with
+// Bucketing by one CTA (pos, active, n_active, passes and n_passes may be NULL). passes[i] describes the i-th tile
+// of VQ_PASS_TOKENS consecutive bucket slots, experts ascending: x = expert | (slots in the tile << 16), y = first
+// slot; n_passes receives their number. Warp c of `chunks` handles pairs [c*P, (c+1)*P) with
 // its own histogram row, so the stable scatter runs in parallel. `ids` may point to global or shared memory; every
 // intermediate table lives in shared memory: hist [chunks][E] and base [E + 1] int32.
 __device__ void bucket(const int32_t *ids, int npairs, int E, int32_t *offsets, int32_t *perm, int32_t *pos,
-                       int32_t *active, int32_t *n_active, int32_t *hist, int32_t *base, int chunks)
+                       int32_t *active, int32_t *n_active, int2 *passes, int32_t *n_passes, int32_t *hist,
+                       int32_t *base, int chunks)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int i = threadIdx.x; i < chunks * E; i += blockDim.x)
@@ -153,33 +156,48 @@ __device__ void bucket(const int32_t *ids, int npairs, int E, int32_t *offsets, 
     }
     __syncthreads();
     if (warp == 0) {
-        int run = 0, act = 0;
+        int run = 0, act = 0, prun = 0;
         const unsigned lt = (1u << lane) - 1u;
         for (int b = 0; b < E; b += 32) {
             const int e = b + lane;
             const int c = e < E ? base[e] : 0;
-            int incl = c;
+            const int np = (c + VQ_PASS_TOKENS - 1) / VQ_PASS_TOKENS;
+            int incl = c, pincl = np;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-                if (lane >= o)
+                const int pv = __shfl_up_sync(0xFFFFFFFFu, pincl, o);
+                if (lane >= o) {
                     incl += v;
+                    pincl += pv;
+                }
             }
+            const int off = run + incl - c;
             if (e < E) {
-                base[e] = run + incl - c;
-                offsets[e] = run + incl - c;
+                base[e] = off;
+                offsets[e] = off;
             }
             const unsigned ball = __ballot_sync(0xFFFFFFFFu, c > 0);
             if (c > 0 && active)
                 active[act + __popc(ball & lt)] = e;
+            if (passes) {
+                // tiles of VQ_PASS_TOKENS slots of this expert's bucket, in bucket order
+                const int p0 = prun + pincl - np;
+                for (int i = 0; i < np; ++i)
+                    passes[p0 + i] = make_int2(e | (min(VQ_PASS_TOKENS, c - VQ_PASS_TOKENS * i) << 16),
+                                               off + VQ_PASS_TOKENS * i);
+            }
             act += __popc(ball);
             run += __shfl_sync(0xFFFFFFFFu, incl, 31);
+            prun += __shfl_sync(0xFFFFFFFFu, pincl, 31);
         }
         if (lane == 0) {
             base[E] = run;
             offsets[E] = run;
             if (n_active)
                 *n_active = act;
+            if (n_passes)
+                *n_passes = prun;
         }
     }
     __syncthreads();
@@ -260,6 +278,7 @@ __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_fused_kernel(const flo
                                                                       int renorm, int32_t *ids, float *w,
                                                                       int32_t *offsets, int32_t *perm, int32_t *pos,
                                                                       int32_t *active, int32_t *n_active,
+                                                                      int2 *passes, int32_t *n_passes,
                                                                       const uint16_t *x, __half *x16, int H, int *err)
 {
     extern __shared__ int32_t sm[];
@@ -274,7 +293,7 @@ __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_fused_kernel(const flo
     for (int p = threadIdx.x; p < npairs; p += blockDim.x)
         s_ids[p] = ids[p];   // written by this CTA above; read back once
     __syncthreads();
-    bucket(s_ids, npairs, E, offsets, perm, pos, active, n_active, hist, base, chunks);
+    bucket(s_ids, npairs, E, offsets, perm, pos, active, n_active, passes, n_passes, hist, base, chunks);
 }
 
 // Large T: many CTAs route, then one CTA buckets.
@@ -294,12 +313,14 @@ __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_topk_kernel(const floa
 
 __global__ void __launch_bounds__(ROUTE_THREADS) vq_bucket_kernel(const int32_t *ids, int npairs, int E,
                                                                  int32_t *offsets, int32_t *perm, int32_t *pos,
-                                                                 int32_t *active, int32_t *n_active)
+                                                                 int32_t *active, int32_t *n_active, int2 *passes,
+                                                                 int32_t *n_passes)
 {
     extern __shared__ int32_t sm[];
     const int chunks = bucket_chunks(E, npairs);
     grid_dep_wait();
-    bucket(ids, npairs, E, offsets, perm, pos, active, n_active, sm, sm + (size_t)chunks * E, chunks);
+    bucket(ids, npairs, E, offsets, perm, pos, active, n_active, passes, n_passes, sm, sm + (size_t)chunks * E,
+           chunks);
 }
 
 template <typename K, typename... Args>
@@ -322,7 +343,8 @@ cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
 
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int32_t *ids, float *w,
                          int32_t *offsets, int32_t *perm, int32_t *pos, int32_t *active, int32_t *n_active,
-                         const uint16_t *x, __half *x16, int H, int *errw, cudaStream_t s, bool pdl)
+                         int2 *passes, int32_t *n_passes, const uint16_t *x, __half *x16, int H, int *errw,
+                         cudaStream_t s, bool pdl)
 {
     static bool attr_set = false;
     if (!attr_set) {
@@ -337,7 +359,7 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
     if (T <= ROUTE_TOKENS_PER_CTA)
         return launch_ex(vq_route_fused_kernel, dim3(1), dim3(ROUTE_THREADS),
                          bucket_smem_ints(E, T * k, true) * sizeof(int32_t), s, pdl, logits, T, E, k, renorm,
-                         ids, w, offsets, perm, pos, active, n_active, x, x16, H, errw);
+                         ids, w, offsets, perm, pos, active, n_active, passes, n_passes, x, x16, H, errw);
     const int ctas = (T + ROUTE_TOKENS_PER_CTA - 1) / ROUTE_TOKENS_PER_CTA;
     cudaError_t err = launch_ex(vq_route_topk_kernel, dim3(ctas), dim3(ROUTE_THREADS), 0, s, pdl, logits, T, E, k,
                                 renorm, ids, w, x, x16, H, errw);
@@ -345,7 +367,7 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
         return err;
     return launch_ex(vq_bucket_kernel, dim3(1), dim3(ROUTE_THREADS), bucket_smem_ints(E, T * k, false) * sizeof(int32_t),
                      s, pdl, (const int32_t *)ids, T * k, E,
-                     offsets, perm, pos, active, n_active);
+                     offsets, perm, pos, active, n_active, passes, n_passes);
 }
 
 }  // namespace vq
