@@ -489,13 +489,14 @@ __device__ __forceinline__ TgItem tg_item(const GemvArgs &a, long item, int nrb,
     return r;
 }
 
-template <int D, int BITS>
+// ABF16: activations in bf16 (else fp16). DENSE: no module of the launch has a
+// live bitmap.
+template <int D, int BITS, bool ABF16, bool DENSE>
 __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid_constant__ GemvTmaArgs A)
 {
     using G = Geo<D, BITS>;
     using TG = TGeo<D, BITS>;
     constexpr bool FAST = FastByteCodes<D, BITS>::value;
-    constexpr int GP = TG::HG >= 2 ? 2 : 1;   // groups decoded together by a warp
     const GemvArgs &a = A.g;
     extern __shared__ __align__(1024) uint8_t tg_smem_raw[];
     uint8_t *smem = tg_smem_raw;
@@ -559,9 +560,9 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
             int prow0 = 0, mi = 0;
             int arow[VQ_PASS_TOKENS];
             uint32_t tx = 0;
-            for (long u = u0; u < u1 && ok; ++u) {
-                const long item = u / spp;
-                const int j = (int)(u % spp);
+            long item = u0 / spp;
+            int j = (int)(u0 % spp);
+            for (long u = u0; u < u1 && ok; ++u, j = (j + 1 == spp) ? 0 : j + 1, item += (j == 0)) {
                 if (u == u0 || j == 0) {
                     it = tg_item(a, item, nrb, cta_mods, FAST);
                     mi = it.mi;
@@ -602,139 +603,153 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
     // ---------------------------------------------------- consumers
     const int half = warp / TG_WPH, wr = warp % TG_WPH;
     const int g = lane >> 2, t = lane & 3;
+    const int sg = tg_sigma(g);
     uint32_t slot = 0, ph = 0, xk = 0;   // stage ring; pieces exchanged by this warp pair
     bool ok = true;
     TgItem it{};
-    int br[4], prow[4];
-    int rep = 0, r0 = 0;
-    uint32_t lane_sel = 0;
-    bool has_tok = false;
+    int prow[4];
+    // Row b of a stage holds the codes of packed row prow0 + b. Without a live
+    // bitmap this lane's rows are b = 32 wr + 8 i + sigma(g), so one base and
+    // immediates address all four; with one, each row has its own offsets
+    // (a dead row reads row 0: its sums are never stored, so the inner loop
+    // has no branches).
+    const int bd = 32 * wr + sg;
+    uint32_t roff[4], soff[4];
+    int swz[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        roff[i] = (uint32_t)((bd + 8 * i) * TG::SRB);
+        soff[i] = A.off_sc + (uint32_t)((bd + 8 * i) * 16);
+        swz[i] = sg;
+    }
+    int rows = 0, rep = 0, log_rep = 0, r0 = 0;
+    uint32_t lane_sel = 0, aoff = 0;
     float acc[2][4];
-    for (long u = u0; u < u1 && ok; ++u) {
-        const long item = u / spp;
-        const int j = (int)(u % spp);
+    long item = u0 / spp;
+    int j = (int)(u0 % spp);
+    for (long u = u0; u < u1 && ok; ++u, j = (j + 1 == spp) ? 0 : j + 1, item += (j == 0)) {
         if (u == u0 || j == 0) {
             it = tg_item(a, item, nrb, cta_mods, FAST);
             const ModDev &m = it.mi == 0 ? a.mod[0] : a.mod[1];
+            rows = m.rows;
             rep = lane & (m.rep - 1);
+            log_rep = m.log_rep;
             lane_sel = (uint32_t)(it.mi * 128 + lane * 4);
             r0 = it.rb * TG_ROWS;
             const int prow0 = tg_prow0(m, it.e, r0);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int r = r0 + 32 * wr + 8 * i + tg_sigma(g);
-                prow[i] = r < m.rows ? (int)live_row(m.bitmap, m.rank, m.bm_words, m.rows, it.e, r) : -1;
-                br[i] = prow[i] >= 0 ? prow[i] - prow0 : -1;
+                const int r = r0 + 32 * wr + 8 * i + sg;
+                if constexpr (DENSE) {
+                    prow[i] = r < rows ? 0 : -1;
+                } else {
+                    prow[i] = r < rows ? (int)live_row(m.bitmap, m.rank, m.bm_words, rows, it.e, r) : -1;
+                    const int b = prow[i] >= 0 ? prow[i] - prow0 : 0;
+                    roff[i] = (uint32_t)(b * TG::SRB);
+                    soff[i] = A.off_sc + (uint32_t)(b * 16);
+                    swz[i] = b & 7;
+                }
             }
-            has_tok = g < it.n;
+            // token g of the tile; lanes past the tile's count read token 0 (a broadcast,
+            // no extra shared-memory traffic) and their output columns are never stored
+            aoff = A.off_act + (uint32_t)((g < it.n ? g : 0) * TG::ACOLS * 2 + t * 32);
 #pragma unroll
             for (int i = 0; i < 2; ++i)
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
                     acc[i][q] = 0.f;
         }
-        const ModDev &m = it.mi == 0 ? a.mod[0] : a.mod[1];
 
         if (!(ok = mbar_wait(&full[slot], ph, abort_flag, A.err, 13)))
             break;
-        const uint8_t *sbase = stages + (size_t)slot * A.stage_bytes;
-        const int g0 = j * TG::CG;
-        const uint16_t *ssc = reinterpret_cast<const uint16_t *>(sbase + A.off_sc) + (g0 & 7);
-        const uint8_t *sact = sbase + A.off_act;
+        const uint8_t *sb = stages + (size_t)slot * A.stage_bytes;
+        const uint8_t *ssc = sb + 2 * ((j * TG::CG) & 7);
 #pragma unroll
-        for (int gh = 0; gh < TG::HG; gh += GP) {
-            uint32_t cw[GP][4][G::LW];
-            int co[GP][4];
-            uint32_t bw[GP][8];
-            float sv[GP][4];
-#pragma unroll
-            for (int uu = 0; uu < GP; ++uu) {
-                const int gq = half * TG::HG + gh + uu;   // group within the stage
+        for (int gh = 0; gh < TG::HG; ++gh) {
+            const int gq = half * TG::HG + gh;   // group within the stage
+            uint32_t cw[4][G::LW];
+            int co = 0;
+            if constexpr (TG::SWZ) {
+                const int c = 2 * gq + (t >> 1);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    if (br[i] >= 0) {
-                        tg_read_quarter<D, BITS>(sbase + (size_t)br[i] * TG::SRB, gq, t, br[i], cw[uu][i],
-                                                 co[uu][i]);
-                        sv[uu][i] = f16_to_f32(ssc[(size_t)br[i] * 8 + gq]);
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < G::LW; ++q)
-                            cw[uu][i][q] = 0u;
-                        co[uu][i] = 0;
-                        sv[uu][i] = 0.f;
-                    }
+                    const uint2 v = *reinterpret_cast<const uint2 *>(
+                        sb + roff[i] + ((uint32_t)((c ^ swz[i]) << 4) | ((uint32_t)(t & 1) << 3)));
+                    cw[i][0] = v.x;
+                    cw[i][1] = v.y;
                 }
-                uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
-                if (has_tok) {
-                    const uint4 *ap =
-                        reinterpret_cast<const uint4 *>(sact + (size_t)g * TG::ACOLS * 2 + gq * 128 + t * 32);
-                    v0 = ap[0];
-                    v1 = ap[1];
-                }
-                bw[uu][0] = v0.x; bw[uu][1] = v0.y; bw[uu][2] = v0.z; bw[uu][3] = v0.w;
-                bw[uu][4] = v1.x; bw[uu][5] = v1.y; bw[uu][6] = v1.z; bw[uu][7] = v1.w;
-                if (a.act_bf16) {
+            } else {
+                // the lane's bit range [bit, bit + QB) of the row; reading LW words may take
+                // one word past it (still inside the stage), whose bits are masked off
+                const int bit = (4 * gq + t) * G::QB;
+                co = bit & 31;
 #pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        bw[uu][q] = bf16x2_to_f16x2(bw[uu][q]);
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t *p = reinterpret_cast<const uint32_t *>(sb + roff[i]) + (bit >> 5);
+#pragma unroll
+                    for (int q = 0; q < G::LW; ++q)
+                        cw[i][q] = p[q];
                 }
             }
-            if (gh + GP >= TG::HG) {   // every read of this stage by the warp is done
+            float sv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                sv[i] = f16_to_f32(*reinterpret_cast<const uint16_t *>(ssc + soff[i] + 2 * gq));
+            const uint4 v0 = *reinterpret_cast<const uint4 *>(sb + aoff + gq * 128);
+            const uint4 v1 = *reinterpret_cast<const uint4 *>(sb + aoff + gq * 128 + 16);
+            uint32_t bw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            if constexpr (ABF16) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    bw[q] = bf16x2_to_f16x2(bw[q]);
+            }
+            if (gh + 1 == TG::HG) {   // every read of this stage by the warp is done
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&empty[slot]);
             }
-            uint32_t c[GP][4][G::CODES];
+            uint32_t c[4][G::CODES];
             if constexpr (!FAST) {
 #pragma unroll
-                for (int uu = 0; uu < GP; ++uu)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        extract_codes<D, BITS>(cw[uu][i], co[uu][i], c[uu][i]);
+                for (int i = 0; i < 4; ++i)
+                    extract_codes<D, BITS>(cw[i], co, c[i]);
             }
-            float tmp[GP][2][4];
+            float tmp[2][4];
 #pragma unroll
-            for (int uu = 0; uu < GP; ++uu)
+            for (int i = 0; i < 2; ++i)
 #pragma unroll
-                for (int i = 0; i < 2; ++i)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        tmp[uu][i][q] = 0.f;
+                for (int q = 0; q < 4; ++q)
+                    tmp[i][q] = 0.f;
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
 #pragma unroll
-                for (int uu = 0; uu < GP; ++uu) {
+                for (int rt = 0; rt < 2; ++rt) {
+                    uint32_t Aw[4];
+                    if constexpr (FAST) {
+                        const char *cbb = reinterpret_cast<const char *>(cbs);
 #pragma unroll
-                    for (int rt = 0; rt < 2; ++rt) {
-                        uint32_t Aw[4];
-                        if constexpr (FAST) {
-                            const char *cbb = reinterpret_cast<const char *>(cbs);
-#pragma unroll
-                            for (int h = 0; h < 2; ++h) {
-                                const uint32_t sel = 0x5504u | ((uint32_t)(2 * (s & 1) + h) << 4);
-                                Aw[2 * h] = *reinterpret_cast<const uint32_t *>(
-                                    cbb + __byte_perm(cw[uu][2 * rt][s >> 1], lane_sel, sel));
-                                Aw[2 * h + 1] = *reinterpret_cast<const uint32_t *>(
-                                    cbb + __byte_perm(cw[uu][2 * rt + 1][s >> 1], lane_sel, sel));
-                            }
-                        } else {
-                            a_words<D>(cbs, m.log_rep, rep, c[uu][2 * rt], s, Aw[0], Aw[2]);
-                            a_words<D>(cbs, m.log_rep, rep, c[uu][2 * rt + 1], s, Aw[1], Aw[3]);
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t sel = 0x5504u | ((uint32_t)(2 * (s & 1) + h) << 4);
+                            Aw[2 * h] =
+                                *reinterpret_cast<const uint32_t *>(cbb + __byte_perm(cw[2 * rt][s >> 1], lane_sel, sel));
+                            Aw[2 * h + 1] = *reinterpret_cast<const uint32_t *>(
+                                cbb + __byte_perm(cw[2 * rt + 1][s >> 1], lane_sel, sel));
                         }
-                        mma_16816(tmp[uu][rt], Aw, bw[uu][2 * s], bw[uu][2 * s + 1]);
+                    } else {
+                        a_words<D>(cbs, log_rep, rep, c[2 * rt], s, Aw[0], Aw[2]);
+                        a_words<D>(cbs, log_rep, rep, c[2 * rt + 1], s, Aw[1], Aw[3]);
                     }
+                    mma_16816(tmp[rt], Aw, bw[2 * s], bw[2 * s + 1]);
                 }
             }
 #pragma unroll
-            for (int uu = 0; uu < GP; ++uu)
-#pragma unroll
-                for (int rt = 0; rt < 2; ++rt) {
-                    const float slo = sv[uu][2 * rt], shi = sv[uu][2 * rt + 1];
-                    acc[rt][0] = fmaf(tmp[uu][rt][0], slo, acc[rt][0]);
-                    acc[rt][1] = fmaf(tmp[uu][rt][1], slo, acc[rt][1]);
-                    acc[rt][2] = fmaf(tmp[uu][rt][2], shi, acc[rt][2]);
-                    acc[rt][3] = fmaf(tmp[uu][rt][3], shi, acc[rt][3]);
-                }
+            for (int rt = 0; rt < 2; ++rt) {
+                const float slo = sv[2 * rt], shi = sv[2 * rt + 1];
+                acc[rt][0] = fmaf(tmp[rt][0], slo, acc[rt][0]);
+                acc[rt][1] = fmaf(tmp[rt][1], slo, acc[rt][1]);
+                acc[rt][2] = fmaf(tmp[rt][2], shi, acc[rt][2]);
+                acc[rt][3] = fmaf(tmp[rt][3], shi, acc[rt][3]);
+            }
         }
         if (++slot == (uint32_t)A.ns) {
             slot = 0;
@@ -776,7 +791,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
             for (int hf = 0; hf < 2; ++hf) {
                 const int i = 2 * rt + hf;
                 const int r = r0 + 32 * wr + 8 * i + tg_sigma(g);
-                if (r >= m.rows)
+                if (r >= rows)
                     continue;
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
@@ -784,7 +799,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                     if (tk >= it.n)
                         continue;
                     const float v = prow[i] >= 0 ? acc[rt][2 * hf + cc] : 0.f;
-                    const long o = (long)(it.q0 + tk) * m.rows + r;
+                    const long o = (long)(it.q0 + tk) * rows + r;
                     store_out(out, a.out_dtype, (long)piece * a.out_slice_stride + o, v);
                     for (int sl = piece + 1; sl < last; ++sl)
                         store_out(out, a.out_dtype, (long)sl * a.out_slice_stride + o, 0.f);
@@ -1007,7 +1022,11 @@ cudaError_t gemv_tma_dispatch(const GemvArgs &a, cudaStream_t s, bool pdl)
     A.off_xchg = p.off_xchg;
     A.off_bar = p.off_bar;
     A.err = a.err;
-    auto k = vq_gemv_tma_kernel<D, BITS>;
+    bool dense = true;
+    for (int i = 0; i < a.nmod; ++i)
+        dense = dense && !a.mod[i].bitmap;
+    auto k = a.act_bf16 ? (dense ? vq_gemv_tma_kernel<D, BITS, true, true> : vq_gemv_tma_kernel<D, BITS, true, false>)
+                        : (dense ? vq_gemv_tma_kernel<D, BITS, false, true> : vq_gemv_tma_kernel<D, BITS, false, false>);
     cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.total);
     if (err != cudaSuccess)
         return err;

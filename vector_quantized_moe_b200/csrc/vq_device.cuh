@@ -38,6 +38,20 @@ __device__ __forceinline__ uint16_t ldg_u16(const uint16_t *p)
     return v;
 }
 
+// 16 bytes of shared memory when pred holds, else zeros (a predicated load, no branch).
+__device__ __forceinline__ uint4 lds128_if(const void *p, bool pred)
+{
+    uint4 v;
+    asm volatile(
+        "{\n\t.reg .pred q;\n\t"
+        "setp.ne.b32 q, %5, 0;\n\t"
+        "mov.b32 %0, 0;\n\tmov.b32 %1, 0;\n\tmov.b32 %2, 0;\n\tmov.b32 %3, 0;\n\t"
+        "@q ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n\t}"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "r"((uint32_t)__cvta_generic_to_shared(p)), "r"((int)pred));
+    return v;
+}
+
 // ---------------------------------------------------------------- numbers
 
 __device__ __forceinline__ float f16_to_f32(uint16_t h)
