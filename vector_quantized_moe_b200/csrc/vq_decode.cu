@@ -380,11 +380,13 @@ __global__ void __launch_bounds__(GEMV_THREADS, 2) vq_grouped_gemv_kernel(const 
 // pieces of an item by the slice count, and readers sum the slices in a fixed
 // order, so results do not depend on timing.
 
+constexpr int TG_HALVES = 2;                     // consumer warp sets splitting a stage's groups
 constexpr int TG_WPH = 8;                        // consumer warps per half
-constexpr int TG_CONSUMERS = 2 * TG_WPH;
+constexpr int TG_CONSUMERS = TG_HALVES * TG_WPH;
 constexpr int TG_THREADS = 32 * (TG_CONSUMERS + 1);
 constexpr int TG_ROWS = 32 * TG_WPH;
-constexpr int TG_XCHG_BYTES = TG_WPH * 2 * 8 * 32 * 4;   // per warp pair: 2 buffers of 8 floats per lane
+// per warp pair: 2 buffers of 8 floats per lane
+constexpr int TG_XCHG_BYTES = TG_HALVES > 1 ? TG_WPH * 2 * 8 * 32 * 4 : 0;
 constexpr int TG_BAR_BYTES = 1024;
 
 // Scale groups per stage: the codes of one row of a stage fill whole 16-byte
@@ -397,14 +399,14 @@ __host__ __device__ constexpr int tg_stage_groups(int d, int bits)
     int cg = 1;
     while ((cg * gb) % 128)
         ++cg;
-    return cg % 2 ? 2 * cg : cg;
+    return (cg % TG_HALVES) ? TG_HALVES * cg : cg;
 }
 
 template <int D, int BITS>
 struct TGeo {
     static constexpr bool SWZ = (D == 2 && BITS == 8);
     static constexpr int CG = tg_stage_groups(D, BITS);
-    static constexpr int HG = CG / 2;               // groups of one half
+    static constexpr int HG = CG / TG_HALVES;       // groups of one half
     static constexpr int GB = (64 / D) * BITS;      // bits per row per group
     static constexpr int SRB = CG * GB / 8;         // bytes per row per stage
     static constexpr int ACOLS = CG * 64;           // activation columns per stage
@@ -497,6 +499,9 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
     using G = Geo<D, BITS>;
     using TG = TGeo<D, BITS>;
     constexpr bool FAST = FastByteCodes<D, BITS>::value;
+    // groups decoded together by a warp: one when 16 consumer warps share the
+    // register file (96 per thread), two with 8
+    constexpr int GP = (TG_HALVES == 1 && TG::HG % 2 == 0) ? 2 : 1;
     const GemvArgs &a = A.g;
     extern __shared__ __align__(1024) uint8_t tg_smem_raw[];
     uint8_t *smem = tg_smem_raw;
@@ -614,6 +619,10 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
     // (a dead row reads row 0: its sums are never stored, so the inner loop
     // has no branches).
     const int bd = 32 * wr + sg;
+    // 128-byte swizzled rows (d=2, 8-bit codes): 16-byte chunk c of row b sits at
+    // chunk c ^ (b & 7); this lane reads chunk 2 gq + t/2, half t%2, and with the
+    // group's bits kept apart that is koff ^ ((gq - first group of the half) << 5)
+    const uint32_t koff = ((uint32_t)(((2 * half * TG::HG) | (t >> 1)) ^ sg) << 4) | ((uint32_t)(t & 1) << 3);
     uint32_t roff[4], soff[4];
     int swz[4];
 #pragma unroll
@@ -665,91 +674,131 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
         const uint8_t *sb = stages + (size_t)slot * A.stage_bytes;
         const uint8_t *ssc = sb + 2 * ((j * TG::CG) & 7);
 #pragma unroll
-        for (int gh = 0; gh < TG::HG; ++gh) {
-            const int gq = half * TG::HG + gh;   // group within the stage
-            uint32_t cw[4][G::LW];
-            int co = 0;
-            if constexpr (TG::SWZ) {
-                const int c = 2 * gq + (t >> 1);
+        for (int gh = 0; gh < TG::HG; gh += GP) {
+            uint32_t cw[GP][4][G::LW];
+            int co[GP];
+            float sv[GP][4];
+            uint32_t bw[GP][8];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint2 v = *reinterpret_cast<const uint2 *>(
-                        sb + roff[i] + ((uint32_t)((c ^ swz[i]) << 4) | ((uint32_t)(t & 1) << 3)));
-                    cw[i][0] = v.x;
-                    cw[i][1] = v.y;
+            for (int uu = 0; uu < GP; ++uu) {
+                const int gq = half * TG::HG + gh + uu;   // group within the stage
+                co[uu] = 0;
+                if constexpr (TG::SWZ && DENSE) {
+                    // rows bd + 8i share the swizzle key sigma(g): one offset, then immediates
+                    const uint8_t *p = sb + roff[0] + (koff ^ (uint32_t)((gq - half * TG::HG) << 5));
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint2 v = *reinterpret_cast<const uint2 *>(p + i * 8 * TG::SRB);
+                        cw[uu][i][0] = v.x;
+                        cw[uu][i][1] = v.y;
+                    }
+                } else if constexpr (TG::SWZ) {
+                    const int c = 2 * gq + (t >> 1);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint2 v = *reinterpret_cast<const uint2 *>(
+                            sb + roff[i] + ((uint32_t)((c ^ swz[i]) << 4) | ((uint32_t)(t & 1) << 3)));
+                        cw[uu][i][0] = v.x;
+                        cw[uu][i][1] = v.y;
+                    }
+                } else if constexpr (DENSE) {
+                    const int bit = (4 * gq + t) * G::QB;
+                    co[uu] = bit & 31;
+                    const uint32_t *p = reinterpret_cast<const uint32_t *>(sb + roff[0]) + (bit >> 5);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+#pragma unroll
+                        for (int q = 0; q < G::LW; ++q)
+                            cw[uu][i][q] = p[i * 8 * TG::SRB / 4 + q];
+                } else {
+                    // the lane's bit range [bit, bit + QB) of the row; reading LW words may take
+                    // one word past it (still inside the stage), whose bits are masked off
+                    const int bit = (4 * gq + t) * G::QB;
+                    co[uu] = bit & 31;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t *p = reinterpret_cast<const uint32_t *>(sb + roff[i]) + (bit >> 5);
+#pragma unroll
+                        for (int q = 0; q < G::LW; ++q)
+                            cw[uu][i][q] = p[q];
+                    }
                 }
-            } else {
-                // the lane's bit range [bit, bit + QB) of the row; reading LW words may take
-                // one word past it (still inside the stage), whose bits are masked off
-                const int bit = (4 * gq + t) * G::QB;
-                co = bit & 31;
+                if constexpr (DENSE) {
+                    const uint8_t *p = ssc + soff[0] + 2 * gq;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t *p = reinterpret_cast<const uint32_t *>(sb + roff[i]) + (bit >> 5);
+                    for (int i = 0; i < 4; ++i)
+                        sv[uu][i] = f16_to_f32(*reinterpret_cast<const uint16_t *>(p + i * 8 * 16));
+                } else {
 #pragma unroll
-                    for (int q = 0; q < G::LW; ++q)
-                        cw[i][q] = p[q];
+                    for (int i = 0; i < 4; ++i)
+                        sv[uu][i] = f16_to_f32(*reinterpret_cast<const uint16_t *>(ssc + soff[i] + 2 * gq));
+                }
+                const uint4 v0 = *reinterpret_cast<const uint4 *>(sb + aoff + gq * 128);
+                const uint4 v1 = *reinterpret_cast<const uint4 *>(sb + aoff + gq * 128 + 16);
+                bw[uu][0] = v0.x; bw[uu][1] = v0.y; bw[uu][2] = v0.z; bw[uu][3] = v0.w;
+                bw[uu][4] = v1.x; bw[uu][5] = v1.y; bw[uu][6] = v1.z; bw[uu][7] = v1.w;
+                if constexpr (ABF16) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        bw[uu][q] = bf16x2_to_f16x2(bw[uu][q]);
                 }
             }
-            float sv[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                sv[i] = f16_to_f32(*reinterpret_cast<const uint16_t *>(ssc + soff[i] + 2 * gq));
-            const uint4 v0 = *reinterpret_cast<const uint4 *>(sb + aoff + gq * 128);
-            const uint4 v1 = *reinterpret_cast<const uint4 *>(sb + aoff + gq * 128 + 16);
-            uint32_t bw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            if constexpr (ABF16) {
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    bw[q] = bf16x2_to_f16x2(bw[q]);
-            }
-            if (gh + 1 == TG::HG) {   // every read of this stage by the warp is done
+            if (gh + GP >= TG::HG) {   // every read of this stage by the warp is done
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(&empty[slot]);
             }
-            uint32_t c[4][G::CODES];
+            uint32_t c[GP][4][G::CODES];
             if constexpr (!FAST) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    extract_codes<D, BITS>(cw[i], co, c[i]);
+                for (int uu = 0; uu < GP; ++uu)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        extract_codes<D, BITS>(cw[uu][i], co[uu], c[uu][i]);
             }
-            float tmp[2][4];
+            float tmp[GP][2][4];
 #pragma unroll
-            for (int i = 0; i < 2; ++i)
+            for (int uu = 0; uu < GP; ++uu)
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    tmp[i][q] = 0.f;
+                for (int i = 0; i < 2; ++i)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        tmp[uu][i][q] = 0.f;
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
 #pragma unroll
-                for (int rt = 0; rt < 2; ++rt) {
-                    uint32_t Aw[4];
-                    if constexpr (FAST) {
-                        const char *cbb = reinterpret_cast<const char *>(cbs);
+                for (int uu = 0; uu < GP; ++uu) {
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const uint32_t sel = 0x5504u | ((uint32_t)(2 * (s & 1) + h) << 4);
-                            Aw[2 * h] =
-                                *reinterpret_cast<const uint32_t *>(cbb + __byte_perm(cw[2 * rt][s >> 1], lane_sel, sel));
-                            Aw[2 * h + 1] = *reinterpret_cast<const uint32_t *>(
-                                cbb + __byte_perm(cw[2 * rt + 1][s >> 1], lane_sel, sel));
+                    for (int rt = 0; rt < 2; ++rt) {
+                        uint32_t Aw[4];
+                        if constexpr (FAST) {
+                            const char *cbb = reinterpret_cast<const char *>(cbs);
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const uint32_t sel = 0x5504u | ((uint32_t)(2 * (s & 1) + h) << 4);
+                                Aw[2 * h] = *reinterpret_cast<const uint32_t *>(
+                                    cbb + __byte_perm(cw[uu][2 * rt][s >> 1], lane_sel, sel));
+                                Aw[2 * h + 1] = *reinterpret_cast<const uint32_t *>(
+                                    cbb + __byte_perm(cw[uu][2 * rt + 1][s >> 1], lane_sel, sel));
+                            }
+                        } else {
+                            a_words<D>(cbs, log_rep, rep, c[uu][2 * rt], s, Aw[0], Aw[2]);
+                            a_words<D>(cbs, log_rep, rep, c[uu][2 * rt + 1], s, Aw[1], Aw[3]);
                         }
-                    } else {
-                        a_words<D>(cbs, log_rep, rep, c[2 * rt], s, Aw[0], Aw[2]);
-                        a_words<D>(cbs, log_rep, rep, c[2 * rt + 1], s, Aw[1], Aw[3]);
+                        mma_16816(tmp[uu][rt], Aw, bw[uu][2 * s], bw[uu][2 * s + 1]);
                     }
-                    mma_16816(tmp[rt], Aw, bw[2 * s], bw[2 * s + 1]);
                 }
             }
 #pragma unroll
-            for (int rt = 0; rt < 2; ++rt) {
-                const float slo = sv[2 * rt], shi = sv[2 * rt + 1];
-                acc[rt][0] = fmaf(tmp[rt][0], slo, acc[rt][0]);
-                acc[rt][1] = fmaf(tmp[rt][1], slo, acc[rt][1]);
-                acc[rt][2] = fmaf(tmp[rt][2], shi, acc[rt][2]);
-                acc[rt][3] = fmaf(tmp[rt][3], shi, acc[rt][3]);
-            }
+            for (int uu = 0; uu < GP; ++uu)
+#pragma unroll
+                for (int rt = 0; rt < 2; ++rt) {
+                    const float slo = sv[uu][2 * rt], shi = sv[uu][2 * rt + 1];
+                    acc[rt][0] = fmaf(tmp[uu][rt][0], slo, acc[rt][0]);
+                    acc[rt][1] = fmaf(tmp[uu][rt][1], slo, acc[rt][1]);
+                    acc[rt][2] = fmaf(tmp[uu][rt][2], shi, acc[rt][2]);
+                    acc[rt][3] = fmaf(tmp[uu][rt][3], shi, acc[rt][3]);
+                }
         }
         if (++slot == (uint32_t)A.ns) {
             slot = 0;
@@ -765,7 +814,9 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
         const uint32_t xph = (xk >> 1) & 1;
         ++xk;
         float *xs = xchg + (size_t)(wr * 2 + xb) * 8 * 32;
-        if (half == 1) {
+        if (TG_HALVES == 1) {
+            // one warp set: the sums are complete
+        } else if (half == 1) {
             if (!(ok = mbar_wait(&xempty[wr * 2 + xb], xph ^ 1, abort_flag, A.err, 14)))
                 break;
 #pragma unroll
@@ -773,13 +824,14 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                 xs[v * 32 + lane] = acc[v >> 2][v & 3];
             mbar_arrive(&xfull[wr * 2 + xb]);
             continue;
-        }
-        if (!(ok = mbar_wait(&xfull[wr * 2 + xb], xph, abort_flag, A.err, 15)))
-            break;
+        } else {
+            if (!(ok = mbar_wait(&xfull[wr * 2 + xb], xph, abort_flag, A.err, 15)))
+                break;
 #pragma unroll
-        for (int v = 0; v < 8; ++v)
-            acc[v >> 2][v & 3] += xs[v * 32 + lane];
-        mbar_arrive(&xempty[wr * 2 + xb]);
+            for (int v = 0; v < 8; ++v)
+                acc[v >> 2][v & 3] += xs[v * 32 + lane];
+            mbar_arrive(&xempty[wr * 2 + xb]);
+        }
 
         void *const out = it.mi == 0 ? a.out[0] : a.out[1];
         const int piece = (int)(blockIdx.x - (item * spp) / L);
