@@ -191,6 +191,7 @@ __global__ void __launch_bounds__(GEMV_THREADS, 2) vq_grouped_gemv_kernel(const 
         fill_codebook<D, BITS>(cbs, (blockIdx.y == 0 ? a.mod[0] : a.mod[1]).codebook,
                                (blockIdx.y == 0 ? a.mod[0] : a.mod[1]).log_rep);
     __syncthreads();
+    grid_dep_launch();   // the next kernel may start its prologue; it waits for this one's results
     grid_dep_wait();
 
     const int lane = threadIdx.x & 31;
@@ -538,6 +539,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
+    grid_dep_launch();   // the next kernel may start its prologue; it waits for this one's results
     grid_dep_wait();
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -865,6 +867,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
 __global__ void vq_swiglu_kernel(const float *__restrict__ G, const float *__restrict__ U, int slices, long slice_stride,
                                  long n, __half *__restrict__ h)
 {
+    grid_dep_launch();   // the next kernel may start its prologue; it waits for this one's results
     grid_dep_wait();
     for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
         float gs = 0.f, us = 0.f;
@@ -885,6 +888,7 @@ __global__ void __launch_bounds__(256) vq_combine_kernel(const float *__restrict
 {
     __shared__ long q_s[32];
     __shared__ float w_s[32];
+    grid_dep_launch();   // the next kernel may start its prologue; it waits for this one's results
     grid_dep_wait();
     const int h4 = hidden >> 2;
     for (int tok = blockIdx.x; tok < T; tok += gridDim.x) {

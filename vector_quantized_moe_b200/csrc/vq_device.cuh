@@ -101,7 +101,8 @@ __device__ __forceinline__ void grid_dep_wait()
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-// Allow the next kernel on the stream to start its prologue.
+// Allow the next kernel on the stream to start its prologue (its own
+// griddepcontrol.wait still waits for this kernel's completion and memory).
 __device__ __forceinline__ void grid_dep_launch()
 {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

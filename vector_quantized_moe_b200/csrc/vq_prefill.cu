@@ -305,6 +305,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                      "r"(tmem_cols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
+    grid_dep_launch();   // the next kernel may start its prologue; it waits for this one's results
     grid_dep_wait();
 
     // tile prefix over the active experts: tiles[ai] = first global n-tile of expert active[ai]
@@ -524,6 +525,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
 __global__ void vq_gather_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ perm, int k, long slots,
                                  int H, __half *__restrict__ xg)
 {
+    grid_dep_launch();   // the next kernel may start its prologue; it waits for this one's results
     grid_dep_wait();
     const int per_row = H / 8;
     for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < slots * per_row; i += (long)gridDim.x * blockDim.x) {

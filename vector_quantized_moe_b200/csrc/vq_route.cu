@@ -17,7 +17,8 @@
 namespace vq {
 namespace {
 
-constexpr int ROUTE_THREADS = 1024;
+constexpr int ROUTE_THREADS = 512;    // routing CTAs: 128 registers per thread hold a lane's sorted keys
+constexpr int BUCKET_THREADS = 1024;  // the bucketing CTA of large batches
 constexpr int BUCKET_MAX_E_PARALLEL = 1024;   // per-warp histograms fit shared memory up to here
 
 // Monotone map of a float to uint32: NaN -> 0 (lowest), -0 -> +0.
@@ -45,11 +46,25 @@ __device__ __forceinline__ float warp_sum(float v)
     return v;
 }
 
+// Inverse of order_key (NaN comes back as a NaN, -0 as +0).
+__device__ __forceinline__ float key_value(uint32_t key)
+{
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
 // One warp routes one token. Lane j < k ends with the j-th selection.
+// Round j takes the largest key below the previous round's winner: a scan of
+// the lane's keys (held in registers for E <= 512, re-read otherwise), then
+// two 32-bit max reductions over the warp (the value word, then the index
+// word among the lanes that tie on it). The round loop is kept rolled: the
+// kernel runs once per layer with a cold instruction cache, so short code
+// matters more than unrolling.
 template <int PER_LANE>
 __device__ __forceinline__ void route_token(const float *__restrict__ l, int E, int k, int renorm, int lane,
                                             int32_t *ids, float *w)
 {
+    int my_id = 0;
+    float my_l = 0.f, top = 0.f;
     uint64_t keys[PER_LANE > 0 ? PER_LANE : 1];
     if constexpr (PER_LANE > 0) {
 #pragma unroll
@@ -59,34 +74,30 @@ __device__ __forceinline__ void route_token(const float *__restrict__ l, int E, 
         }
     }
     uint64_t prev = ~0ull;
-    int my_id = 0;
-    float my_l = 0.f;
+#pragma unroll 1
     for (int j = 0; j < k; ++j) {
         uint64_t best = 0ull;
         if constexpr (PER_LANE > 0) {
 #pragma unroll
             for (int i = 0; i < PER_LANE; ++i)
-                if (keys[i] < prev && keys[i] > best)
-                    best = keys[i];
+                best = (keys[i] < prev && keys[i] > best) ? keys[i] : best;
         } else {
             for (int e = lane; e < E; e += 32) {
                 const uint64_t key = expert_key(l[e], e);
-                if (key < prev && key > best)
-                    best = key;
+                best = (key < prev && key > best) ? key : best;
             }
         }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) {
-            const uint64_t other = __shfl_xor_sync(0xFFFFFFFFu, best, o);
-            best = other > best ? other : best;
-        }
-        prev = best;
+        const uint32_t hi = (uint32_t)(best >> 32);
+        const uint32_t H = __reduce_max_sync(0xFFFFFFFFu, hi);
+        const uint32_t Lw = __reduce_max_sync(0xFFFFFFFFu, hi == H ? (uint32_t)best : 0u);
+        prev = ((uint64_t)H << 32) | Lw;
+        if (j == 0)
+            top = key_value(H);
         if (lane == j) {
-            my_id = (int)(0xFFFFFFFFu - (uint32_t)best);
-            my_l = l[my_id];
+            my_id = (int)(0xFFFFFFFFu - Lw);
+            my_l = key_value(H);
         }
     }
-    const float top = __shfl_sync(0xFFFFFFFFu, my_l, 0);
     const float num = lane < k ? expf(my_l - top) : 0.f;
     float den;
     if (renorm) {
@@ -103,25 +114,26 @@ __device__ __forceinline__ void route_token(const float *__restrict__ l, int E, 
     }
 }
 
+// Tokens [t_begin, t_end), one per warp, over warps [w0, w0 + nw) of the CTA.
 template <int PER_LANE>
 __device__ void route_tokens(const float *logits, int t_begin, int t_end, int E, int k, int renorm, int32_t *ids,
-                             float *w)
+                             float *w, int w0, int nw)
 {
     const int lane = threadIdx.x & 31;
-    const int nw = blockDim.x >> 5;
-    for (int t = t_begin + (threadIdx.x >> 5); t < t_end; t += nw)
+    for (int t = t_begin + (threadIdx.x >> 5) - w0; t < t_end; t += nw)
         route_token<PER_LANE>(logits + (long)t * E, E, k, renorm, lane, ids + (long)t * k, w + (long)t * k);
 }
 
+// Called by the warps [w0, w0 + nw) of the CTA.
 __device__ void route_range(const float *logits, int t_begin, int t_end, int E, int k, int renorm, int32_t *ids,
-                            float *w)
+                            float *w, int w0, int nw)
 {
     if (E <= 128)
-        route_tokens<4>(logits, t_begin, t_end, E, k, renorm, ids, w);
+        route_tokens<4>(logits, t_begin, t_end, E, k, renorm, ids, w, w0, nw);
     else if (E <= 512)
-        route_tokens<16>(logits, t_begin, t_end, E, k, renorm, ids, w);
+        route_tokens<16>(logits, t_begin, t_end, E, k, renorm, ids, w, w0, nw);
     else
-        route_tokens<0>(logits, t_begin, t_end, E, k, renorm, ids, w);
+        route_tokens<0>(logits, t_begin, t_end, E, k, renorm, ids, w, w0, nw);
 }
 
 // Bucketing by one CTA (pos, active, n_active, passes and n_passes may be NULL). passes[i] describes the i-th tile
@@ -155,49 +167,83 @@ __device__ void bucket(const int32_t *ids, int npairs, int E, int32_t *offsets, 
         base[e] = run;   // count for now
     }
     __syncthreads();
-    if (warp == 0) {
-        int run = 0, act = 0, prun = 0;
-        const unsigned lt = (1u << lane) - 1u;
-        for (int b = 0; b < E; b += 32) {
-            const int e = b + lane;
+    // exclusive scans over the experts of (pairs, active experts, token tiles): thread i owns the
+    // experts [i*EPT, (i+1)*EPT); a warp scan, a scan of the warp totals, then each thread writes
+    // its experts' offsets, active-list entries and token tiles
+    {
+        __shared__ int wtot[32][3];
+        const int EPT = (E + blockDim.x - 1) / blockDim.x;
+        const int e0 = threadIdx.x * EPT;
+        int v[3] = {0, 0, 0};
+        for (int i = 0; i < EPT; ++i) {
+            const int e = e0 + i;
             const int c = e < E ? base[e] : 0;
-            const int np = (c + VQ_PASS_TOKENS - 1) / VQ_PASS_TOKENS;
-            int incl = c, pincl = np;
+            v[0] += c;
+            v[1] += c > 0;
+            v[2] += (c + VQ_PASS_TOKENS - 1) / VQ_PASS_TOKENS;
+        }
+        int inc[3] = {v[0], v[1], v[2]};
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-                const int pv = __shfl_up_sync(0xFFFFFFFFu, pincl, o);
-                if (lane >= o) {
-                    incl += v;
-                    pincl += pv;
+        for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+            for (int q = 0; q < 3; ++q) {
+                const int x = __shfl_up_sync(0xFFFFFFFFu, inc[q], o);
+                if (lane >= o)
+                    inc[q] += x;
+            }
+        if (lane == 31)
+            for (int q = 0; q < 3; ++q)
+                wtot[warp][q] = inc[q];
+        __syncthreads();
+        const int nw = blockDim.x >> 5;
+        if (warp == 0) {
+#pragma unroll
+            for (int q = 0; q < 3; ++q) {
+                int t = lane < nw ? wtot[lane][q] : 0;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int x = __shfl_up_sync(0xFFFFFFFFu, t, o);
+                    if (lane >= o)
+                        t += x;
+                }
+                if (lane < nw)
+                    wtot[lane][q] = t;   // inclusive over warps
+            }
+        }
+        __syncthreads();
+        int run[3];
+#pragma unroll
+        for (int q = 0; q < 3; ++q)
+            run[q] = (warp > 0 ? wtot[warp - 1][q] : 0) + inc[q] - v[q];
+        for (int i = 0; i < EPT; ++i) {
+            const int e = e0 + i;
+            if (e >= E)
+                break;
+            const int c = base[e];
+            base[e] = run[0];
+            offsets[e] = run[0];
+            if (c > 0) {
+                if (active)
+                    active[run[1]] = e;
+                if (passes) {
+                    // tiles of VQ_PASS_TOKENS slots of this expert's bucket, in bucket order
+                    const int np = (c + VQ_PASS_TOKENS - 1) / VQ_PASS_TOKENS;
+                    for (int t = 0; t < np; ++t)
+                        passes[run[2] + t] = make_int2(e | (min(VQ_PASS_TOKENS, c - VQ_PASS_TOKENS * t) << 16),
+                                                       run[0] + VQ_PASS_TOKENS * t);
                 }
             }
-            const int off = run + incl - c;
-            if (e < E) {
-                base[e] = off;
-                offsets[e] = off;
-            }
-            const unsigned ball = __ballot_sync(0xFFFFFFFFu, c > 0);
-            if (c > 0 && active)
-                active[act + __popc(ball & lt)] = e;
-            if (passes) {
-                // tiles of VQ_PASS_TOKENS slots of this expert's bucket, in bucket order
-                const int p0 = prun + pincl - np;
-                for (int i = 0; i < np; ++i)
-                    passes[p0 + i] = make_int2(e | (min(VQ_PASS_TOKENS, c - VQ_PASS_TOKENS * i) << 16),
-                                               off + VQ_PASS_TOKENS * i);
-            }
-            act += __popc(ball);
-            run += __shfl_sync(0xFFFFFFFFu, incl, 31);
-            prun += __shfl_sync(0xFFFFFFFFu, pincl, 31);
+            run[0] += c;
+            run[1] += c > 0;
+            run[2] += (c + VQ_PASS_TOKENS - 1) / VQ_PASS_TOKENS;
         }
-        if (lane == 0) {
-            base[E] = run;
-            offsets[E] = run;
+        if (threadIdx.x == 0) {
+            base[E] = wtot[nw - 1][0];
+            offsets[E] = wtot[nw - 1][0];
             if (n_active)
-                *n_active = act;
+                *n_active = wtot[nw - 1][1];
             if (n_passes)
-                *n_passes = prun;
+                *n_passes = wtot[nw - 1][2];
         }
     }
     __syncthreads();
@@ -231,15 +277,15 @@ __device__ void bucket(const int32_t *ids, int npairs, int E, int32_t *offsets, 
 // read fp16 activations; bf16 -> fp16 is exact for magnitudes in [2^-14, 65504]).
 // Rows of H % 8 == 0 elements are 16-byte aligned: four 16-byte loads per
 // thread are in flight before the first store.
-__device__ void convert_rows(const uint16_t *x, __half *x16, int t0, int t1, int H)
+__device__ void convert_rows(const uint16_t *x, __half *x16, int t0, int t1, int H, int tid, int nthr)
 {
     if (!x)
         return;
     const long n8 = (long)(t1 - t0) * H / 8;
     const uint4 *src = reinterpret_cast<const uint4 *>(x + (long)t0 * H);
     uint4 *dst = reinterpret_cast<uint4 *>(x16 + (long)t0 * H);
-    const long step = blockDim.x;
-    for (long i0 = threadIdx.x; i0 < n8; i0 += 4 * step) {
+    const long step = nthr;
+    for (long i0 = tid; i0 < n8; i0 += 4 * step) {
         uint4 v[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u)
@@ -259,18 +305,18 @@ __device__ void convert_rows(const uint16_t *x, __half *x16, int t0, int t1, int
 }
 
 // Warps that scatter in parallel: one per 256 pairs (at most one per warp of the CTA).
-__host__ __device__ __forceinline__ int bucket_chunks(int E, int npairs)
+__host__ __device__ __forceinline__ int bucket_chunks(int E, int npairs, int threads)
 {
     if (E > BUCKET_MAX_E_PARALLEL)
         return 1;
     const int c = (npairs + 255) / 256;
-    return c < 1 ? 1 : (c > ROUTE_THREADS / 32 ? ROUTE_THREADS / 32 : c);
+    return c < 1 ? 1 : (c > threads / 32 ? threads / 32 : c);
 }
 
 // Shared memory of a bucketing CTA: hist, base and (fused kernel) the pair ids.
-__host__ __device__ __forceinline__ size_t bucket_smem_ints(int E, int npairs, bool with_ids)
+__host__ __device__ __forceinline__ size_t bucket_smem_ints(int E, int npairs, bool with_ids, int threads)
 {
-    return (size_t)bucket_chunks(E, npairs) * E + (size_t)E + 1 + (with_ids ? (size_t)npairs : 0);
+    return (size_t)bucket_chunks(E, npairs, threads) * E + (size_t)E + 1 + (with_ids ? (size_t)npairs : 0);
 }
 
 // Small T: one CTA routes every token and buckets the pairs.
@@ -282,13 +328,23 @@ __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_fused_kernel(const flo
                                                                       const uint16_t *x, __half *x16, int H, int *err)
 {
     extern __shared__ int32_t sm[];
-    const int npairs = T * k, chunks = bucket_chunks(E, npairs);
+    const int npairs = T * k, chunks = bucket_chunks(E, npairs, ROUTE_THREADS);
     int32_t *hist = sm, *base = sm + (size_t)chunks * E, *s_ids = base + E + 1;
+    grid_dep_launch();   // the next kernel may start its prologue; it waits for this one's results
     grid_dep_wait();
     if (err && threadIdx.x == 0)
         *err = 0;
-    route_range(logits, 0, T, E, k, renorm, ids, w);
-    convert_rows(x, x16, 0, T, H);
+    const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5;
+    if (T < nw) {
+        // warps [0, T) route one token each while the others convert the activations
+        if (warp < T)
+            route_range(logits, 0, T, E, k, renorm, ids, w, 0, T);
+        else
+            convert_rows(x, x16, 0, T, H, threadIdx.x - 32 * T, blockDim.x - 32 * T);
+    } else {
+        route_range(logits, 0, T, E, k, renorm, ids, w, 0, nw);
+        convert_rows(x, x16, 0, T, H, threadIdx.x, blockDim.x);
+    }
     __syncthreads();
     for (int p = threadIdx.x; p < npairs; p += blockDim.x)
         s_ids[p] = ids[p];   // written by this CTA above; read back once
@@ -303,21 +359,23 @@ __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_topk_kernel(const floa
                                                                      int renorm, int32_t *ids, float *w,
                                                                      const uint16_t *x, __half *x16, int H, int *err)
 {
+    grid_dep_launch();   // the next kernel may start its prologue; it waits for this one's results
     grid_dep_wait();
     if (err && blockIdx.x == 0 && threadIdx.x == 0)
         *err = 0;
     const int t0 = blockIdx.x * ROUTE_TOKENS_PER_CTA;
-    convert_rows(x, x16, t0, min(T, t0 + ROUTE_TOKENS_PER_CTA), H);
-    route_range(logits, t0, min(T, t0 + ROUTE_TOKENS_PER_CTA), E, k, renorm, ids, w);
+    convert_rows(x, x16, t0, min(T, t0 + ROUTE_TOKENS_PER_CTA), H, threadIdx.x, blockDim.x);
+    route_range(logits, t0, min(T, t0 + ROUTE_TOKENS_PER_CTA), E, k, renorm, ids, w, 0, blockDim.x >> 5);
 }
 
-__global__ void __launch_bounds__(ROUTE_THREADS) vq_bucket_kernel(const int32_t *ids, int npairs, int E,
+__global__ void __launch_bounds__(BUCKET_THREADS) vq_bucket_kernel(const int32_t *ids, int npairs, int E,
                                                                  int32_t *offsets, int32_t *perm, int32_t *pos,
                                                                  int32_t *active, int32_t *n_active, int2 *passes,
                                                                  int32_t *n_passes)
 {
     extern __shared__ int32_t sm[];
-    const int chunks = bucket_chunks(E, npairs);
+    const int chunks = bucket_chunks(E, npairs, BUCKET_THREADS);
+    grid_dep_launch();   // the next kernel may start its prologue; it waits for this one's results
     grid_dep_wait();
     bucket(ids, npairs, E, offsets, perm, pos, active, n_active, passes, n_passes, sm, sm + (size_t)chunks * E,
            chunks);
@@ -346,27 +404,34 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
                          int2 *passes, int32_t *n_passes, const uint16_t *x, __half *x16, int H, int *errw,
                          cudaStream_t s, bool pdl)
 {
+    // dynamic shared memory of the bucketing CTA: at most 32 x 1024 histogram
+    // rows + bases + 8192 pair ids (T <= 256 tokens of k <= 32) = 168 KB; the
+    // kernels' static tables come on top
+    constexpr size_t ROUTE_SMEM_MAX = 170 * 1024;
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t err = cudaFuncSetAttribute(vq_route_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               227 * 1024);
+                                               (int)ROUTE_SMEM_MAX);
         if (err == cudaSuccess)
-            err = cudaFuncSetAttribute(vq_bucket_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+            err = cudaFuncSetAttribute(vq_bucket_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)ROUTE_SMEM_MAX);
         if (err != cudaSuccess)
             return err;
         attr_set = true;
     }
-    if (T <= ROUTE_TOKENS_PER_CTA)
-        return launch_ex(vq_route_fused_kernel, dim3(1), dim3(ROUTE_THREADS),
-                         bucket_smem_ints(E, T * k, true) * sizeof(int32_t), s, pdl, logits, T, E, k, renorm,
+    const bool fused = T <= ROUTE_TOKENS_PER_CTA;
+    const size_t smem = bucket_smem_ints(E, T * k, fused, fused ? ROUTE_THREADS : BUCKET_THREADS) * sizeof(int32_t);
+    if (smem > ROUTE_SMEM_MAX)
+        return cudaErrorInvalidValue;
+    if (fused)
+        return launch_ex(vq_route_fused_kernel, dim3(1), dim3(ROUTE_THREADS), smem, s, pdl, logits, T, E, k, renorm,
                          ids, w, offsets, perm, pos, active, n_active, passes, n_passes, x, x16, H, errw);
     const int ctas = (T + ROUTE_TOKENS_PER_CTA - 1) / ROUTE_TOKENS_PER_CTA;
     cudaError_t err = launch_ex(vq_route_topk_kernel, dim3(ctas), dim3(ROUTE_THREADS), 0, s, pdl, logits, T, E, k,
                                 renorm, ids, w, x, x16, H, errw);
     if (err != cudaSuccess)
         return err;
-    return launch_ex(vq_bucket_kernel, dim3(1), dim3(ROUTE_THREADS), bucket_smem_ints(E, T * k, false) * sizeof(int32_t),
-                     s, pdl, (const int32_t *)ids, T * k, E,
+    return launch_ex(vq_bucket_kernel, dim3(1), dim3(BUCKET_THREADS), smem, s, pdl, (const int32_t *)ids, T * k, E,
                      offsets, perm, pos, active, n_active, passes, n_passes);
 }
 
