@@ -14,11 +14,13 @@
 //   warp 0     TMA: activation tiles (fp16, 128B-swizzled, one 64-column
 //              k-step per stage) and packed-code tiles (a chunk of CH k-steps)
 //   warp 1     owns the tensor memory; one thread issues tcgen05.mma
-//   warps 2-9  two warpgroups taking alternate k-steps: thread i of a
+//   warps 2+   NWG warpgroups taking the k-steps in turn: thread i of a
 //              warpgroup decodes row i of the weight tile (unpack, codebook
-//              lookup, x fp16 scale) and stores it into tensor memory lane i,
-//              where tcgen05.mma reads its A operand; both then run the
-//              epilogue from tensor memory, on alternate 32-column blocks
+//              lookup, x fp16 scale) into registers, waits until the MMA that
+//              last read the tensor-memory stage has finished, and stores the
+//              row into lane i, where tcgen05.mma reads its A operand; all
+//              then run the epilogue from tensor memory, on interleaved
+//              32-column blocks
 // D[row, token] = sum_k W[row, k] X[token, k]: the weight tile is the
 // M=128 operand (in tensor memory), the tokens of the bucket the N operand
 // (16..128, shared memory), so small buckets waste no M rows. Tensor memory
@@ -38,10 +40,12 @@ namespace vq {
 namespace {
 
 constexpr int BM = 128;             // weight rows per tile = TMEM lanes
-constexpr int BN = 128;             // tokens per tile
-constexpr int NTHREADS = 320;       // 10 warps: TMA, MMA, 8 dequant/epilogue
+// tokens per tile: the accumulators of nmod modules (nmod x BN fp32 columns)
+// and 4 A stages (nmod x 32 columns each) share the 512 tensor-memory columns
+__host__ __device__ constexpr int bn_of(int nmod) { return nmod == 2 ? 128 : 256; }
+constexpr int NWG = 2;              // dequant/epilogue warpgroups (take k-steps in turn)
+constexpr int NTHREADS = 64 + 128 * NWG;   // TMA warp, MMA warp, the warpgroups
 constexpr int A_COLS = 32;          // tensor-memory columns of one 128 x 64 fp16 weight tile
-constexpr int B_TILE = BN * 128;
 
 __host__ __device__ constexpr int chunk_steps(int kb)
 {
@@ -69,7 +73,7 @@ __host__ __device__ constexpr long code_stage_bytes(int d, int bits)
 // fit next to the operand and code stages
 __host__ __device__ constexpr int prefill_log_rep(int d, int bits, int nmod)
 {
-    const long left = SMEM_LIMIT - SMEM_RESERVE - (long)B_STAGES * 128 * 128 -
+    const long left = SMEM_LIMIT - SMEM_RESERVE - (long)B_STAGES * bn_of(nmod) * 128 -
                       (long)CODE_STAGES * nmod * code_stage_bytes(d, bits);
     int lr = 0;
     while (lr < 4 && (long)nmod * (1L << bits) * d * 2 * (2L << lr) <= left)
@@ -217,6 +221,7 @@ struct Item {
     int e, m0, q0, n;
 };
 
+template <int BN>
 __device__ __forceinline__ Item item_of(long it, int MT, const int *tiles, int n_act, const int32_t *active,
                                         const int32_t *offsets)
 {
@@ -251,6 +256,8 @@ template <int D, int BITS, int NMOD>
 __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __grid_constant__ PrefillArgs a)
 {
     using P = PG<D, BITS, NMOD>;
+    constexpr int BN = bn_of(NMOD);
+    constexpr uint32_t B_TILE = BN * 128;
     // one code stage per module: the chunk's packed codes, then the scales of
     // the 8-group block holding its k-steps
     constexpr uint32_t CODE_STAGE = BM * P::CHW * 4 + BM * 16;
@@ -291,7 +298,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
         }
         for (int s = 0; s < a.sc; ++s) {
             mbar_init(&full_c[s], 1);
-            mbar_init(&empty_c[s], 256);
+            mbar_init(&empty_c[s], 128 * NWG);
         }
         mbar_init(acc_full, 1);
         *abort_flag = 0;
@@ -299,7 +306,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
     }
     // accumulators: nmod x BN columns; then sa stages of nmod A tiles
     const uint32_t acc_cols = (uint32_t)nmod * BN;
-    const uint32_t tmem_cols = nmod == 2 ? 512 : 256;
+    const uint32_t tmem_cols = 512;
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(tmem_cols));
@@ -335,7 +342,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
             uint32_t ks = 0, st = 0, ph = 0, cst = 0, cph = 0;   // operand / code stage counters
             bool ok = true;
             for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-                const Item itm = item_of(it, MT, tiles, n_act, a.active, a.offsets);
+                const Item itm = item_of<BN>(it, MT, tiles, n_act, a.active, a.offsets);
                 int prow0[2];
                 for (int m = 0; m < nmod; ++m)
                     prow0[m] = tile_prow0(a.mod[m], itm.e, itm.m0);
@@ -380,7 +387,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
             uint32_t st = 0, ph = 0;
             bool ok = true;
             for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-                const Item itm = item_of(it, MT, tiles, n_act, a.active, a.offsets);
+                const Item itm = item_of<BN>(it, MT, tiles, n_act, a.active, a.offsets);
                 const int n16 = (itm.n + 15) & ~15;
                 const uint32_t idesc = idesc_f16(BM, n16);
                 for (int k = 0; k < ksteps; ++k) {
@@ -408,14 +415,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
         }
     } else {
         // ---------------------------------------------------------- dequant + epilogue
-        const int wg = (warp - 2) >> 2;   // warpgroup: takes k-steps with (k & 1) == wg
+        const int wg = (warp - 2) >> 2;   // warpgroup: takes k-steps with k % NWG == wg
         const int rowi = 32 * (warp & 3) + lane;
         const uint32_t rep_off = (uint32_t)(lane & ((1 << log_rep) - 1)) * (2 * D);
         const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
         uint32_t st = 0, ph = 0, cst = 0, cph = 0, nit = 0;
         bool ok = true;
         for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-            const Item itm = item_of(it, MT, tiles, n_act, a.active, a.offsets);
+            const Item itm = item_of<BN>(it, MT, tiles, n_act, a.active, a.offsets);
             const int r = itm.m0 + rowi;
             int lrow[2] = {-1, -1};
             long prow[2] = {-1, -1};
@@ -449,18 +456,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                     constexpr int JJ = decltype(jj_c)::value;
                     if (!ok)
                         return;
-                    if (((c * P::CH + JJ) & 1) == wg) {
+                    if ((c * P::CH + JJ) % NWG == wg) {
+                        const uint32_t a_tmem = tmem + lane_addr + acc_cols + st * nmod * A_COLS;
+                        // decode both modules first (their A tiles are adjacent columns of the
+                        // stage, stored with one instruction); the wait for the stage's previous
+                        // MMA overlaps the decode
+                        uint32_t o[32 * NMOD];
+                        dequant_step<D, BITS, P::L, JJ>(crow[0], sm_cb, rep_off, sfetch(0, JJ), lrow[0] >= 0,
+                                                        *reinterpret_cast<uint32_t(*)[32]>(o));
+                        if constexpr (NMOD == 2)
+                            dequant_step<D, BITS, P::L, JJ>(crow[1], sm_cb + cb_bytes, rep_off, sfetch(1, JJ),
+                                                            lrow[1] >= 0, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
                         if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag, a.err, 7)))
                             return;
-                        const uint32_t a_tmem = tmem + lane_addr + acc_cols + st * nmod * A_COLS;
-                        uint32_t o[32];
-                        dequant_step<D, BITS, P::L, JJ>(crow[0], sm_cb, rep_off, sfetch(0, JJ), lrow[0] >= 0, o);
-                        tmem_st32(a_tmem, o);
-                        if (nmod == 2) {
-                            dequant_step<D, BITS, P::L, JJ>(crow[1], sm_cb + cb_bytes, rep_off, sfetch(1, JJ),
-                                                            lrow[1] >= 0, o);
-                            tmem_st32(a_tmem + A_COLS, o);
-                        }
+                        tc_fence_after();   // the stage's previous MMA has read it
+                        if constexpr (NMOD == 2)
+                            tmem_st64(a_tmem, o);
+                        else
+                            tmem_st32(a_tmem, *reinterpret_cast<uint32_t(*)[32]>(o));
                         tmem_wait_st();
                         tc_fence_before();
                         mbar_arrive(&full_a[st]);
@@ -487,7 +500,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                 break;
             ++nit;
             tc_fence_after();
-            for (int cb0 = 32 * wg; cb0 < itm.n; cb0 += 64) {
+            for (int cb0 = 32 * wg; cb0 < itm.n; cb0 += 32 * NWG) {
                 uint32_t g[32], u[32];
                 tmem_ld32(tmem + lane_addr + cb0, g);
                 if (nmod == 2)
@@ -546,10 +559,10 @@ __global__ void vq_gather_kernel(const uint16_t *__restrict__ x, const int32_t *
 
 int chw_of(int d, int bits);
 
-// fp16 activations [rows, cols]: boxes of 64 columns x BN rows, 128-byte swizzle
-bool map_act(CUtensorMap *map, const void *base, long rows, int cols)
+// fp16 activations [rows, cols]: boxes of 64 columns x bn rows, 128-byte swizzle
+bool map_act(CUtensorMap *map, const void *base, long rows, int cols, int bn)
 {
-    return tma_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, (uint64_t)cols, (uint64_t)rows, 64, BN,
+    return tma_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, (uint64_t)cols, (uint64_t)rows, 64, (uint32_t)bn,
                       CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
@@ -593,7 +606,7 @@ SmemPlan smem_plan(int nmod, int d, int bits, int E)
         p.sc = CODE_STAGES;
         p.off_a = 0;
         p.off_b = 0;
-        p.off_c = p.off_b + (uint32_t)sa * B_TILE;
+        p.off_c = p.off_b + (uint32_t)sa * bn_of(nmod) * 128;
         p.off_cb = p.off_c + p.sc * code_stage;
         p.off_tiles = p.off_cb + cb;
         p.off_bar = (uint32_t)align_up(p.off_tiles + tiles, 8);
@@ -719,7 +732,7 @@ vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const flo
         a.mod[0] = make_moddev(L->gate);
         a.mod[1] = make_moddev(L->up);
         a.nmod = 2;
-        if (!map_act(&a.tmap_b, xg, tk, H) || !map_codes(&a.tmap_c[0], a.mod[0]) || !map_codes(&a.tmap_c[1], a.mod[1]))
+        if (!map_act(&a.tmap_b, xg, tk, H, bn_of(2)) || !map_codes(&a.tmap_c[0], a.mod[0]) || !map_codes(&a.tmap_c[1], a.mod[1]))
             return VQ_ERR_CUDA;
         if (a.mod[0].ngroups % 8 == 0 && (!map_scales(&a.tmap_s[0], a.mod[0]) || !map_scales(&a.tmap_s[1], a.mod[1])))
             return VQ_ERR_CUDA;
@@ -754,7 +767,7 @@ vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const flo
         a.mod[0] = make_moddev(L->down);
         a.mod[1] = a.mod[0];
         a.nmod = 1;
-        if (!map_act(&a.tmap_b, hh, tk, I) || !map_codes(&a.tmap_c[0], a.mod[0]))
+        if (!map_act(&a.tmap_b, hh, tk, I, bn_of(1)) || !map_codes(&a.tmap_c[0], a.mod[0]))
             return VQ_ERR_CUDA;
         if (a.mod[0].ngroups % 8 == 0 && !map_scales(&a.tmap_s[0], a.mod[0]))
             return VQ_ERR_CUDA;
