@@ -366,7 +366,7 @@ def run_ours(args):
                    "tokens_per_s": T * args.steps * ws / (ms_total * 1e-3)},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "traffic": _traffic_per_launch("grouped_gemv_gate_up"),
-                     "kernel": "vq_grouped_gemv_kernel<2,8> (gate+up)", "peak_source": f"{src} hbm_gbs",
+                     "kernel": "vq_gemv_tma_kernel<2,8,fp16,dense> (gate+up)", "peak_source": f"{src} hbm_gbs",
                      "bytes_per_launch": gu_avg_bytes, "ms_per_launch": gu_ms},
         "stage_ms": {"route": float(stage_ms[0]), "gate_up_gemv": gu_ms, "swiglu": float(stage_ms[2]),
                      "down_gemv": float(stage_ms[3]), "combine": float(stage_ms[4])},
@@ -462,7 +462,7 @@ def measure_prefill(torch, vq, dev, steps, warmup, small=False, ncu_mode=False):
                         "down_gemm": float(stage[3]), "combine": float(stage[4])},
            "roofline": {"bound": "tensor", "achieved": gu_tflops, "peak": tf_burst, "unit": "TFLOP/s",
                         "frac": gu_tflops / tf_burst, "traffic": _traffic_per_launch("prefill_gemm_gate_up"),
-                        "kernel": "vq_prefill_gemm_kernel<4,9> (gate+up, SwiGLU epilogue)",
+                        "kernel": "vq_prefill_gemm_kernel<4,9,2> (gate+up, SwiGLU epilogue)",
                         "peak_source": f"{src} bf16_tflops (fp16 runs at the bf16 rate)",
                         "flops_per_launch": flops_gu, "ms_per_launch": float(stage[2])},
            "launches_per_step": 7}
