@@ -864,6 +864,10 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
 
 // ------------------------------------------------------------ SwiGLU and combine
 
+// h = fp16(silu(sum_s G[s]) * sum_s U[s]), slices summed in order. S > 0: the
+// slice count is a compile-time constant, so every load is issued before the
+// first add; S == 0: any slice count.
+template <int S>
 __global__ void vq_swiglu_kernel(const float *__restrict__ G, const float *__restrict__ U, int slices, long slice_stride,
                                  long n, __half *__restrict__ h)
 {
@@ -871,17 +875,33 @@ __global__ void vq_swiglu_kernel(const float *__restrict__ G, const float *__res
     grid_dep_wait();
     for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
         float gs = 0.f, us = 0.f;
-        for (int s = 0; s < slices; ++s) {
-            gs += G[s * slice_stride + i];
-            us += U[s * slice_stride + i];
+        if constexpr (S > 0) {
+            float gv[S], uv[S];
+#pragma unroll
+            for (int q = 0; q < S; ++q) {
+                gv[q] = G[q * slice_stride + i];
+                uv[q] = U[q * slice_stride + i];
+            }
+#pragma unroll
+            for (int q = 0; q < S; ++q) {
+                gs += gv[q];
+                us += uv[q];
+            }
+        } else {
+            for (int q = 0; q < slices; ++q) {
+                gs += G[q * slice_stride + i];
+                us += U[q * slice_stride + i];
+            }
         }
         const float silu = gs / (1.f + __expf(-gs));
         h[i] = __float2half_rn(silu * us);
     }
 }
 
-// y[t, :] = sum_j w[t, j] * sum_s D[s, pos[t*k + j], :], slots in order j, one
-// block per token, four columns per thread.
+// y[t, :] = sum_j w[t, j] * sum_s D[s, pos[t*k + j], :], slots in order j and
+// slices in order s; a block per token (and column range), four columns per
+// thread. The loads of 8 slots x S slices are issued before any is used.
+template <int S>
 __global__ void __launch_bounds__(256) vq_combine_kernel(const float *__restrict__ D, int slices, long slice_stride,
                                                          const float *__restrict__ w, const int32_t *__restrict__ pos,
                                                          int T, int k, int hidden, void *y, int y_dtype)
@@ -900,20 +920,50 @@ __global__ void __launch_bounds__(256) vq_combine_kernel(const float *__restrict
         __syncthreads();
         for (int c4 = blockIdx.y * blockDim.x + threadIdx.x; c4 < h4; c4 += gridDim.y * blockDim.x) {
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int j = 0; j < k; ++j) {
-                float4 part = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int s = 0; s < slices; ++s) {
-                    const float4 v = reinterpret_cast<const float4 *>(D + s * slice_stride + q_s[j])[c4];
-                    part.x += v.x;
-                    part.y += v.y;
-                    part.z += v.z;
-                    part.w += v.w;
+            if constexpr (S == 0) {   // any slice count
+                for (int j = 0; j < k; ++j) {
+                    float4 part = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int q = 0; q < slices; ++q) {
+                        const float4 v = reinterpret_cast<const float4 *>(D + q * slice_stride + q_s[j])[c4];
+                        part.x += v.x;
+                        part.y += v.y;
+                        part.z += v.z;
+                        part.w += v.w;
+                    }
+                    const float wj = w_s[j];
+                    acc.x = fmaf(wj, part.x, acc.x);
+                    acc.y = fmaf(wj, part.y, acc.y);
+                    acc.z = fmaf(wj, part.z, acc.z);
+                    acc.w = fmaf(wj, part.w, acc.w);
                 }
-                const float wj = w_s[j];
-                acc.x = fmaf(wj, part.x, acc.x);
-                acc.y = fmaf(wj, part.y, acc.y);
-                acc.z = fmaf(wj, part.z, acc.z);
-                acc.w = fmaf(wj, part.w, acc.w);
+            }
+            for (int j0 = 0; S > 0 && j0 < k; j0 += 8) {
+                float4 v[8][S > 0 ? S : 1];
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+                    for (int q = 0; q < S; ++q)
+                        v[jj][q] = j0 + jj < k ? reinterpret_cast<const float4 *>(D + q * slice_stride + q_s[j0 + jj])[c4]
+                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    if (j0 + jj >= k)
+                        break;
+                    // 0 + v[0] as in the slice-loop form (turns a -0 sum into +0)
+                    float4 part = make_float4(0.f + v[jj][0].x, 0.f + v[jj][0].y, 0.f + v[jj][0].z, 0.f + v[jj][0].w);
+#pragma unroll
+                    for (int q = 1; q < S; ++q) {
+                        part.x += v[jj][q].x;
+                        part.y += v[jj][q].y;
+                        part.z += v[jj][q].z;
+                        part.w += v[jj][q].w;
+                    }
+                    const float wj = w_s[j0 + jj];
+                    acc.x = fmaf(wj, part.x, acc.x);
+                    acc.y = fmaf(wj, part.y, acc.y);
+                    acc.z = fmaf(wj, part.z, acc.z);
+                    acc.w = fmaf(wj, part.w, acc.w);
+                }
             }
             const long o = (long)tok * hidden + 4 * c4;
             if (y_dtype == VQ_F32) {
@@ -1162,8 +1212,14 @@ cudaError_t launch_swiglu(const float *G, const float *U, int slices, long slice
                           cudaStream_t s, bool pdl)
 {
     const long n = (long)slots * inter;
-    const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
-    return launch(vq_swiglu_kernel, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, s, pdl, G, U, slices, slice_stride, n, h);
+    const dim3 grid((unsigned)((n + 255) / 256 < 4096 ? (n > 0 ? (n + 255) / 256 : 1) : 4096));
+    switch (slices) {
+    case 1: return launch(vq_swiglu_kernel<1>, grid, dim3(256), 0, s, pdl, G, U, slices, slice_stride, n, h);
+    case 2: return launch(vq_swiglu_kernel<2>, grid, dim3(256), 0, s, pdl, G, U, slices, slice_stride, n, h);
+    case 3: return launch(vq_swiglu_kernel<3>, grid, dim3(256), 0, s, pdl, G, U, slices, slice_stride, n, h);
+    case 4: return launch(vq_swiglu_kernel<4>, grid, dim3(256), 0, s, pdl, G, U, slices, slice_stride, n, h);
+    default: return launch(vq_swiglu_kernel<0>, grid, dim3(256), 0, s, pdl, G, U, slices, slice_stride, n, h);
+    }
 }
 
 cudaError_t launch_combine(const float *D, int slices, long slice_stride, const float *w, const int32_t *pos, int T, int k,
@@ -1175,8 +1231,17 @@ cudaError_t launch_combine(const float *D, int slices, long slice_stride, const 
     int ysplit = 1;
     while (blocks * ysplit < 2 * num_sms() && ysplit * 256 < h4)
         ysplit *= 2;
-    return launch(vq_combine_kernel, dim3(blocks, ysplit), dim3(256), 0, s, pdl, D, slices, slice_stride, w, pos, T, k,
-                  hidden, y, y_dtype);
+    const dim3 grid(blocks, ysplit);
+#define VQ_COMBINE(S_) launch(vq_combine_kernel<S_>, grid, dim3(256), 0, s, pdl, D, slices, slice_stride, w, pos, T, k, \
+                              hidden, y, y_dtype)
+    switch (slices) {
+    case 1: return VQ_COMBINE(1);
+    case 2: return VQ_COMBINE(2);
+    case 3: return VQ_COMBINE(3);
+    case 4: return VQ_COMBINE(4);
+    default: return VQ_COMBINE(0);
+    }
+#undef VQ_COMBINE
 }
 
 cudaError_t launch_unpack(const ModDev &m, int expert, uint16_t *out, cudaStream_t s)
