@@ -67,10 +67,15 @@ __device__ __forceinline__ void route_token(const float *__restrict__ l, int E, 
     float my_l = 0.f, top = 0.f;
     uint64_t keys[PER_LANE > 0 ? PER_LANE : 1];
     if constexpr (PER_LANE > 0) {
+        // all loads first (a clamped index keeps them unconditional and independent)
+        float v[PER_LANE];
+#pragma unroll
+        for (int i = 0; i < PER_LANE; ++i)
+            v[i] = __ldg(l + min(lane + 32 * i, E - 1));
 #pragma unroll
         for (int i = 0; i < PER_LANE; ++i) {
             const int e = lane + 32 * i;
-            keys[i] = e < E ? expert_key(l[e], e) : 0ull;
+            keys[i] = e < E ? expert_key(v[i], e) : 0ull;
         }
     }
     uint64_t prev = ~0ull;
