@@ -60,18 +60,19 @@ __device__ __forceinline__ float key_value(uint32_t key)
 // kernel runs once per layer with a cold instruction cache, so short code
 // matters more than unrolling.
 template <int PER_LANE>
-__device__ __forceinline__ void route_token(const float *__restrict__ l, int E, int k, int renorm, int lane,
+__device__ __forceinline__ void route_token(const float *l, int E, int k, int renorm, int lane,
                                             int32_t *ids, float *w)
 {
     int my_id = 0;
     float my_l = 0.f, top = 0.f;
     uint64_t keys[PER_LANE > 0 ? PER_LANE : 1];
     if constexpr (PER_LANE > 0) {
-        // all loads first (a clamped index keeps them unconditional and independent)
+        // all loads first (a clamped index keeps them unconditional and independent);
+        // plain loads, since the warm-up pass reads its logits from shared memory
         float v[PER_LANE];
 #pragma unroll
         for (int i = 0; i < PER_LANE; ++i)
-            v[i] = __ldg(l + min(lane + 32 * i, E - 1));
+            v[i] = l[min(lane + 32 * i, E - 1)];
 #pragma unroll
         for (int i = 0; i < PER_LANE; ++i) {
             const int e = lane + 32 * i;
@@ -130,7 +131,9 @@ __device__ void route_tokens(const float *logits, int t_begin, int t_end, int E,
 }
 
 // Called by the warps [w0, w0 + nw) of the CTA.
-__device__ void route_range(const float *logits, int t_begin, int t_end, int E, int k, int renorm, int32_t *ids,
+// Not inlined: the routing kernel's warm-up pass and its real pass run the same code.
+__device__ __noinline__ void route_range(const float *logits, int t_begin, int t_end, int E, int k, int renorm,
+                                        int32_t *ids,
                             float *w, int w0, int nw)
 {
     if (E <= 128)
@@ -146,7 +149,8 @@ __device__ void route_range(const float *logits, int t_begin, int t_end, int E, 
 // slot; n_passes receives their number. Warp c of `chunks` handles pairs [c*P, (c+1)*P) with
 // its own histogram row, so the stable scatter runs in parallel. `ids` may point to global or shared memory; every
 // intermediate table lives in shared memory: hist [chunks][E] and base [E + 1] int32.
-__device__ void bucket(const int32_t *ids, int npairs, int E, int32_t *offsets, int32_t *perm, int32_t *pos,
+__device__ __noinline__ void bucket(const int32_t *ids, int npairs, int E, int32_t *offsets, int32_t *perm,
+                                    int32_t *pos,
                        int32_t *active, int32_t *n_active, int2 *passes, int32_t *n_passes, int32_t *hist,
                        int32_t *base, int chunks)
 {
@@ -318,10 +322,16 @@ __host__ __device__ __forceinline__ int bucket_chunks(int E, int npairs, int thr
     return c < 1 ? 1 : (c > threads / 32 ? threads / 32 : c);
 }
 
-// Shared memory of a bucketing CTA: hist, base and (fused kernel) the pair ids.
-__host__ __device__ __forceinline__ size_t bucket_smem_ints(int E, int npairs, bool with_ids, int threads)
+// Outputs of the fused kernel's warm-up pass (one token): ids and weights of k
+// slots, offsets [E + 1], perm and pos [k], active [E], counts, token tiles.
+__host__ __device__ __forceinline__ size_t warmup_smem_ints(int E, int k) { return 2 * (size_t)E + 8 * (size_t)k + 8; }
+
+// Shared memory of a bucketing CTA: hist, base and (fused kernel) the pair ids
+// and the warm-up scratch.
+__host__ __device__ __forceinline__ size_t bucket_smem_ints(int E, int npairs, bool fused, int threads, int k = 0)
 {
-    return (size_t)bucket_chunks(E, npairs, threads) * E + (size_t)E + 1 + (with_ids ? (size_t)npairs : 0);
+    return (size_t)bucket_chunks(E, npairs, threads) * E + (size_t)E + 1 +
+           (fused ? (size_t)npairs + warmup_smem_ints(E, k) : 0);
 }
 
 // Small T: one CTA routes every token and buckets the pairs.
@@ -336,6 +346,31 @@ __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_fused_kernel(const flo
     const int npairs = T * k, chunks = bucket_chunks(E, npairs, ROUTE_THREADS);
     int32_t *hist = sm, *base = sm + (size_t)chunks * E, *s_ids = base + E + 1;
     grid_dep_launch();   // the next kernel may start its prologue; it waits for this one's results
+
+    // Warm-up while the previous kernel on the stream finishes: one token of
+    // zero logits through the same routing and bucketing code, with every
+    // output in shared memory, so the real pass finds its instructions cached;
+    // and the logits prefetched into L2. Nothing global is read or written
+    // here except the prefetch hints.
+    {
+        int32_t *wu = s_ids + npairs;
+        int32_t *w_ids = wu, *w_off = w_ids + 2 * k, *w_perm = w_off + E + 1, *w_pos = w_perm + k;
+        int32_t *w_act = w_pos + k, *w_cnt = w_act + E;
+        int2 *w_tiles = reinterpret_cast<int2 *>(w_cnt + 2 + ((reinterpret_cast<uintptr_t>(w_cnt + 2) & 4) ? 1 : 0));
+        float *zeros = reinterpret_cast<float *>(hist);   // E zero logits in the histogram area
+        for (int e = threadIdx.x; e < E; e += blockDim.x)
+            zeros[e] = 0.f;
+        const long lbytes = (long)T * E * 4;
+        for (long o = (long)threadIdx.x * 128; o < lbytes; o += (long)blockDim.x * 128)
+            asm volatile("prefetch.L2 [%0];" ::"l"(reinterpret_cast<const char *>(logits) + o));   // generic address
+        __syncthreads();
+        if (threadIdx.x < 32)
+            route_range(zeros, 0, 1, E, k, renorm, w_ids, reinterpret_cast<float *>(w_ids + k), 0, 1);
+        __syncthreads();
+        bucket(w_ids, k, E, w_off, w_perm, w_pos, w_act, w_cnt, w_tiles, w_cnt + 1, hist, base,
+               bucket_chunks(E, k, ROUTE_THREADS));
+        __syncthreads();
+    }
     grid_dep_wait();
     if (err && threadIdx.x == 0)
         *err = 0;
@@ -409,9 +444,10 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
                          int2 *passes, int32_t *n_passes, const uint16_t *x, __half *x16, int H, int *errw,
                          cudaStream_t s, bool pdl)
 {
-    // dynamic shared memory of the bucketing CTA: at most 32 x 1024 histogram
-    // rows + bases + 8192 pair ids (T <= 256 tokens of k <= 32) = 168 KB; the
-    // kernels' static tables come on top
+    // dynamic shared memory of a bucketing CTA: at most 32 x 1024 histogram rows
+    // + bases (the 1024-thread bucketing CTA, 135 KB), or 16 x 1024 rows + bases
+    // + 8192 pair ids + the warm-up scratch (the fused CTA, 112 KB); the kernels'
+    // static tables come on top
     constexpr size_t ROUTE_SMEM_MAX = 170 * 1024;
     static bool attr_set = false;
     if (!attr_set) {
@@ -425,7 +461,7 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
         attr_set = true;
     }
     const bool fused = T <= ROUTE_TOKENS_PER_CTA;
-    const size_t smem = bucket_smem_ints(E, T * k, fused, fused ? ROUTE_THREADS : BUCKET_THREADS) * sizeof(int32_t);
+    const size_t smem = bucket_smem_ints(E, T * k, fused, fused ? ROUTE_THREADS : BUCKET_THREADS, k) * sizeof(int32_t);
     if (smem > ROUTE_SMEM_MAX)
         return cudaErrorInvalidValue;
     if (fused)
