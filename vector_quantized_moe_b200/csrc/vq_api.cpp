@@ -401,6 +401,11 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     const DecodePlan p = plan_decode(L, T, top_k);
     if (ws_bytes < p.total)
         return VQ_ERR_WORKSPACE;
+    // the GEMV kernels index their work (token tiles x modules x 256-row blocks x
+    // stages) with 32-bit integers
+    for (const vq_module *m : {&L->gate, &L->up, &L->down})
+        if ((double)max_passes(T, top_k, p.E) * 2.0 * ((m->rows + 255) / 256) * (m->cols / 64) >= 2147483647.0)
+            return VQ_ERR_UNSUPPORTED;
     cudaStream_t s = (cudaStream_t)stream;
     int32_t *ids = ws_at<int32_t>(workspace, p.r.ids);
     float *w = ws_at<float>(workspace, p.r.w);

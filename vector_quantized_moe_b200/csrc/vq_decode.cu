@@ -364,8 +364,10 @@ __global__ void __launch_bounds__(GEMV_THREADS, 2) vq_grouped_gemv_kernel(const 
 // shared-memory stages of 256 weight rows x CG scale groups. A CTA has 16
 // consumer warps in two halves and one producer warp whose lane 0 issues the
 // stage's tensor loads. Consumer warp w takes rows [32 (w % 8), +32) of the
-// stage and half w / 8 of its groups; the two halves' partial sums of a row
-// tile meet in shared memory when a piece of work ends. For d=2/8-bit codes a
+// stage (two m16 tiles, four rows per lane) and half w / 8 of its groups; the
+// two halves' partial sums of a row tile meet in shared memory when a piece of
+// work ends. (Measured: 8 warps of 64 rows are slower; 16 warps hide more
+// latency at 96 registers per thread.) For d=2/8-bit codes a
 // stage row is 128 bytes loaded with the 128-byte swizzle, and m16 row g of a
 // warp is weight row sigma(g) (even rows in the first half-warp, odd rows in
 // the second), so a warp's 8-byte code reads hit distinct banks. Each wait on
@@ -382,12 +384,15 @@ __global__ void __launch_bounds__(GEMV_THREADS, 2) vq_grouped_gemv_kernel(const 
 // order, so results do not depend on timing.
 
 constexpr int TG_HALVES = 2;                     // consumer warp sets splitting a stage's groups
+constexpr int TG_RT = 2;                         // m16 row tiles per consumer warp
+constexpr int TG_RL = 2 * TG_RT;                 // weight rows per lane
+constexpr int TG_WROWS = 16 * TG_RT;             // weight rows per consumer warp
 constexpr int TG_WPH = 8;                        // consumer warps per half
 constexpr int TG_CONSUMERS = TG_HALVES * TG_WPH;
 constexpr int TG_THREADS = 32 * (TG_CONSUMERS + 1);
-constexpr int TG_ROWS = 32 * TG_WPH;
-// per warp pair: 2 buffers of 8 floats per lane
-constexpr int TG_XCHG_BYTES = TG_HALVES > 1 ? TG_WPH * 2 * 8 * 32 * 4 : 0;
+constexpr int TG_ROWS = TG_WROWS * TG_WPH;
+// per warp pair: 2 buffers of 4 * TG_RT floats per lane
+constexpr int TG_XCHG_BYTES = TG_HALVES > 1 ? TG_WPH * 2 * (4 * TG_RT) * 32 * 4 : 0;
 constexpr int TG_BAR_BYTES = 1024;
 
 // Scale groups per stage: the codes of one row of a stage fill whole 16-byte
@@ -472,13 +477,15 @@ struct TgItem {
     int rb;   // 256-row block
 };
 
+// (32-bit index arithmetic: 64-bit division is a long instruction sequence)
 __device__ __forceinline__ TgItem tg_item(const GemvArgs &a, long item, int nrb, int cta_mods, bool fast)
 {
     TgItem r;
-    r.rb = (int)(item % nrb);
-    const long rest = item / nrb;
-    r.mi = fast ? (int)(rest % cta_mods) : (int)blockIdx.y;
-    const long tile = fast ? rest / cta_mods : rest;
+    const int it32 = (int)item;
+    const int rest = it32 / nrb;
+    r.rb = it32 - rest * nrb;
+    r.mi = fast ? (cta_mods == 2 ? (rest & 1) : 0) : (int)blockIdx.y;
+    const int tile = fast && cta_mods == 2 ? (rest >> 1) : rest;
     if (a.passes) {
         const int2 pt = a.passes[tile];
         r.e = pt.x & 0xFFFF;
@@ -614,28 +621,28 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
     uint32_t slot = 0, ph = 0, xk = 0;   // stage ring; pieces exchanged by this warp pair
     bool ok = true;
     TgItem it{};
-    int prow[4];
+    int prow[TG_RL];
     // Row b of a stage holds the codes of packed row prow0 + b. Without a live
     // bitmap this lane's rows are b = 32 wr + 8 i + sigma(g), so one base and
     // immediates address all four; with one, each row has its own offsets
     // (a dead row reads row 0: its sums are never stored, so the inner loop
     // has no branches).
-    const int bd = 32 * wr + sg;
+    const int bd = TG_WROWS * wr + sg;
     // 128-byte swizzled rows (d=2, 8-bit codes): 16-byte chunk c of row b sits at
     // chunk c ^ (b & 7); this lane reads chunk 2 gq + t/2, half t%2, and with the
     // group's bits kept apart that is koff ^ ((gq - first group of the half) << 5)
     const uint32_t koff = ((uint32_t)(((2 * half * TG::HG) | (t >> 1)) ^ sg) << 4) | ((uint32_t)(t & 1) << 3);
-    uint32_t roff[4], soff[4];
-    int swz[4];
+    uint32_t roff[TG_RL], soff[TG_RL];
+    int swz[TG_RL];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < TG_RL; ++i) {
         roff[i] = (uint32_t)((bd + 8 * i) * TG::SRB);
         soff[i] = A.off_sc + (uint32_t)((bd + 8 * i) * 16);
         swz[i] = sg;
     }
     int rows = 0, rep = 0, log_rep = 0, r0 = 0;
     uint32_t lane_sel = 0, aoff = 0;
-    float acc[2][4];
+    float acc[TG_RT][4];
     long item = u0 / spp;
     int j = (int)(u0 % spp);
     for (long u = u0; u < u1 && ok; ++u, j = (j + 1 == spp) ? 0 : j + 1, item += (j == 0)) {
@@ -649,8 +656,8 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
             r0 = it.rb * TG_ROWS;
             const int prow0 = tg_prow0(m, it.e, r0);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = r0 + 32 * wr + 8 * i + sg;
+            for (int i = 0; i < TG_RL; ++i) {
+                const int r = r0 + TG_WROWS * wr + 8 * i + sg;
                 if constexpr (DENSE) {
                     prow[i] = r < rows ? 0 : -1;
                 } else {
@@ -665,7 +672,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
             // no extra shared-memory traffic) and their output columns are never stored
             aoff = A.off_act + (uint32_t)((g < it.n ? g : 0) * TG::ACOLS * 2 + t * 32);
 #pragma unroll
-            for (int i = 0; i < 2; ++i)
+            for (int i = 0; i < TG_RT; ++i)
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
                     acc[i][q] = 0.f;
@@ -677,9 +684,9 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
         const uint8_t *ssc = sb + 2 * ((j * TG::CG) & 7);
 #pragma unroll
         for (int gh = 0; gh < TG::HG; gh += GP) {
-            uint32_t cw[GP][4][G::LW];
+            uint32_t cw[GP][TG_RL][G::LW];
             int co[GP];
-            float sv[GP][4];
+            float sv[GP][TG_RL];
             uint32_t bw[GP][8];
 #pragma unroll
             for (int uu = 0; uu < GP; ++uu) {
@@ -689,7 +696,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                     // rows bd + 8i share the swizzle key sigma(g): one offset, then immediates
                     const uint8_t *p = sb + roff[0] + (koff ^ (uint32_t)((gq - half * TG::HG) << 5));
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                    for (int i = 0; i < TG_RL; ++i) {
                         const uint2 v = *reinterpret_cast<const uint2 *>(p + i * 8 * TG::SRB);
                         cw[uu][i][0] = v.x;
                         cw[uu][i][1] = v.y;
@@ -697,7 +704,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                 } else if constexpr (TG::SWZ) {
                     const int c = 2 * gq + (t >> 1);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                    for (int i = 0; i < TG_RL; ++i) {
                         const uint2 v = *reinterpret_cast<const uint2 *>(
                             sb + roff[i] + ((uint32_t)((c ^ swz[i]) << 4) | ((uint32_t)(t & 1) << 3)));
                         cw[uu][i][0] = v.x;
@@ -708,7 +715,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                     co[uu] = bit & 31;
                     const uint32_t *p = reinterpret_cast<const uint32_t *>(sb + roff[0]) + (bit >> 5);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
+                    for (int i = 0; i < TG_RL; ++i)
 #pragma unroll
                         for (int q = 0; q < G::LW; ++q)
                             cw[uu][i][q] = p[i * 8 * TG::SRB / 4 + q];
@@ -718,7 +725,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                     const int bit = (4 * gq + t) * G::QB;
                     co[uu] = bit & 31;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                    for (int i = 0; i < TG_RL; ++i) {
                         const uint32_t *p = reinterpret_cast<const uint32_t *>(sb + roff[i]) + (bit >> 5);
 #pragma unroll
                         for (int q = 0; q < G::LW; ++q)
@@ -728,11 +735,11 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                 if constexpr (DENSE) {
                     const uint8_t *p = ssc + soff[0] + 2 * gq;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
+                    for (int i = 0; i < TG_RL; ++i)
                         sv[uu][i] = f16_to_f32(*reinterpret_cast<const uint16_t *>(p + i * 8 * 16));
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
+                    for (int i = 0; i < TG_RL; ++i)
                         sv[uu][i] = f16_to_f32(*reinterpret_cast<const uint16_t *>(ssc + soff[i] + 2 * gq));
                 }
                 const uint4 v0 = *reinterpret_cast<const uint4 *>(sb + aoff + gq * 128);
@@ -750,19 +757,19 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                 if (lane == 0)
                     mbar_arrive(&empty[slot]);
             }
-            uint32_t c[GP][4][G::CODES];
+            uint32_t c[GP][TG_RL][G::CODES];
             if constexpr (!FAST) {
 #pragma unroll
                 for (int uu = 0; uu < GP; ++uu)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
+                    for (int i = 0; i < TG_RL; ++i)
                         extract_codes<D, BITS>(cw[uu][i], co[uu], c[uu][i]);
             }
-            float tmp[GP][2][4];
+            float tmp[GP][TG_RT][4];
 #pragma unroll
             for (int uu = 0; uu < GP; ++uu)
 #pragma unroll
-                for (int i = 0; i < 2; ++i)
+                for (int i = 0; i < TG_RT; ++i)
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         tmp[uu][i][q] = 0.f;
@@ -771,7 +778,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
 #pragma unroll
                 for (int uu = 0; uu < GP; ++uu) {
 #pragma unroll
-                    for (int rt = 0; rt < 2; ++rt) {
+                    for (int rt = 0; rt < TG_RT; ++rt) {
                         uint32_t Aw[4];
                         if constexpr (FAST) {
                             const char *cbb = reinterpret_cast<const char *>(cbs);
@@ -794,7 +801,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
 #pragma unroll
             for (int uu = 0; uu < GP; ++uu)
 #pragma unroll
-                for (int rt = 0; rt < 2; ++rt) {
+                for (int rt = 0; rt < TG_RT; ++rt) {
                     const float slo = sv[uu][2 * rt], shi = sv[uu][2 * rt + 1];
                     acc[rt][0] = fmaf(tmp[uu][rt][0], slo, acc[rt][0]);
                     acc[rt][1] = fmaf(tmp[uu][rt][1], slo, acc[rt][1]);
@@ -815,14 +822,14 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
         const int xb = (int)(xk & 1);
         const uint32_t xph = (xk >> 1) & 1;
         ++xk;
-        float *xs = xchg + (size_t)(wr * 2 + xb) * 8 * 32;
+        float *xs = xchg + (size_t)(wr * 2 + xb) * (4 * TG_RT) * 32;
         if (TG_HALVES == 1) {
             // one warp set: the sums are complete
         } else if (half == 1) {
             if (!(ok = mbar_wait(&xempty[wr * 2 + xb], xph ^ 1, abort_flag, A.err, 14)))
                 break;
 #pragma unroll
-            for (int v = 0; v < 8; ++v)
+            for (int v = 0; v < 4 * TG_RT; ++v)
                 xs[v * 32 + lane] = acc[v >> 2][v & 3];
             mbar_arrive(&xfull[wr * 2 + xb]);
             continue;
@@ -830,21 +837,21 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
             if (!(ok = mbar_wait(&xfull[wr * 2 + xb], xph, abort_flag, A.err, 15)))
                 break;
 #pragma unroll
-            for (int v = 0; v < 8; ++v)
+            for (int v = 0; v < 4 * TG_RT; ++v)
                 acc[v >> 2][v & 3] += xs[v * 32 + lane];
             mbar_arrive(&xempty[wr * 2 + xb]);
         }
 
         void *const out = it.mi == 0 ? a.out[0] : a.out[1];
-        const int piece = (int)(blockIdx.x - (item * spp) / L);
+        const int piece = (int)blockIdx.x - (int)item * spp / (int)L;
         const int last = j == spp - 1 ? a.slices : piece + 1;   // zeros past the item's last piece
         // lane holds rows r0 + 32 wr + 8 i + sigma(g) for tile tokens 2t + {0, 1}
 #pragma unroll
-        for (int rt = 0; rt < 2; ++rt)
+        for (int rt = 0; rt < TG_RT; ++rt)
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 const int i = 2 * rt + hf;
-                const int r = r0 + 32 * wr + 8 * i + tg_sigma(g);
+                const int r = r0 + TG_WROWS * wr + 8 * i + tg_sigma(g);
                 if (r >= rows)
                     continue;
 #pragma unroll
