@@ -425,8 +425,17 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     trace_point(0, s);
     int2 *passes = ws_at<int2>(workspace, p.r.passes);
     int32_t *npass = ws_at<int32_t>(workspace, p.r.npass);
+    // the routing launch clears the partial-sum slices beyond the first; the GEMVs
+    // then store only the pieces they compute
+    ZeroSpans zs{};
+    zs.p[0] = G + tk * p.I;
+    zs.n[0] = (long)(p.sa - 1) * tk * p.I;
+    zs.p[1] = U + tk * p.I;
+    zs.n[1] = (long)(p.sa - 1) * tk * p.I;
+    zs.p[2] = D + tk * p.H;
+    zs.n[2] = (long)(p.sb - 1) * tk * p.H;
     cudaError_t err = launch_route(logits, T, p.E, top_k, renorm, ids, w, offsets, perm, pos, active, nact, passes,
-                                   npass, x, x16, p.H, errw, s, true);
+                                   npass, x, x16, p.H, errw, s, true, &zs);
     if (err != cudaSuccess)
         return VQ_ERR_CUDA;
     trace_point(1, s);
@@ -446,6 +455,7 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     a.n_passes = npass;
     a.slices = p.sa;
     a.min_units = p.pg.min_units;
+    a.slices_zeroed = 1;
     a.out_dtype = VQ_F32;
     a.out_slice_stride = tk * p.I;
     a.err = errw;

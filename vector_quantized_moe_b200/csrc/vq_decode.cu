@@ -844,7 +844,8 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
 
         void *const out = it.mi == 0 ? a.out[0] : a.out[1];
         const int piece = (int)blockIdx.x - (int)item * spp / (int)L;
-        const int last = j == spp - 1 ? a.slices : piece + 1;   // zeros past the item's last piece
+        // zeros past the item's last piece, unless the routing launch cleared those slices
+        const int last = (j == spp - 1 && !a.slices_zeroed) ? a.slices : piece + 1;
         // lane holds rows r0 + 32 wr + 8 i + sigma(g) for tile tokens 2t + {0, 1}
 #pragma unroll
         for (int rt = 0; rt < TG_RT; ++rt)

@@ -56,6 +56,7 @@ struct GemvArgs {
     int T;                  // single-expert mode: tokens
     int slices;             // partial-sum slices of the output (the reader sums them in order)
     int min_units;          // TMA kernel: least weight stages per CTA (bounds the pieces of a work item)
+    int slices_zeroed;      // slices beyond the first are zero on entry (cleared by the routing launch)
     void *out[2];           // per module: [slices][slots][rows]
     int out_dtype;          // VQ_F32 or VQ_BF16
     long out_slice_stride;  // elements between slices
@@ -79,11 +80,19 @@ size_t gemv_smem_bytes(const ModDev &m);
 // Routing + bucketing. pos = inverse of perm; active/n_active as above (may be NULL).
 // When x is not NULL the same launch also writes x16 = fp16(x) [T, H]; when
 // err is not NULL it is cleared.
+// Up to three device spans of 32-bit words that a routing launch clears (after
+// its grid-dependency wait): the partial-sum slices beyond the first, which a
+// GEMV launch with slices_zeroed set then leaves to the items that write them.
+struct ZeroSpans {
+    float *p[3];
+    long n[3];   // words
+};
+
 // passes / n_passes (may be NULL): the token tiles of the buckets, see VQ_PASS_TOKENS.
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int32_t *ids, float *w,
                          int32_t *offsets, int32_t *perm, int32_t *pos, int32_t *active, int32_t *n_active,
                          int2 *passes, int32_t *n_passes, const uint16_t *x, __half *x16, int H, int *err,
-                         cudaStream_t s, bool pdl);
+                         cudaStream_t s, bool pdl, const ZeroSpans *zero = nullptr);
 
 // h[q, c] = fp16( silu(sum_s G[s, q, c]) * sum_s U[s, q, c] )
 cudaError_t launch_swiglu(const float *G, const float *U, int slices, long slice_stride, int slots, int inter,

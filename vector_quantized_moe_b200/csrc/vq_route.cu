@@ -11,6 +11,8 @@
 // a bucket), its inverse (pos), and the ascending list of experts with
 // tokens. Every step is integer work or a fixed-order reduction, so the
 // tables are bit-identical from run to run.
+#include <algorithm>
+
 #include "vq_device.cuh"
 #include "vq_internal.h"
 
@@ -334,14 +336,31 @@ __host__ __device__ __forceinline__ size_t bucket_smem_ints(int E, int npairs, b
            (fused ? (size_t)npairs + warmup_smem_ints(E, k) : 0);
 }
 
-// Small T: one CTA routes every token and buckets the pairs.
+// Clears this CTA's share of the spans (32-bit words, coalesced).
+__device__ void zero_spans(const ZeroSpans &z, int cta, int nctas)
+{
+    const long stride = (long)nctas * blockDim.x;
+    for (int q = 0; q < 3; ++q)
+        for (long i = (long)cta * blockDim.x + threadIdx.x; i < z.n[q]; i += stride)
+            z.p[q][i] = 0.f;
+}
+
+// Small T: CTA 0 routes every token and buckets the pairs; CTAs 1.. clear the
+// zero spans.
 __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_fused_kernel(const float *logits, int T, int E, int k,
                                                                       int renorm, int32_t *ids, float *w,
                                                                       int32_t *offsets, int32_t *perm, int32_t *pos,
                                                                       int32_t *active, int32_t *n_active,
                                                                       int2 *passes, int32_t *n_passes,
-                                                                      const uint16_t *x, __half *x16, int H, int *err)
+                                                                      const uint16_t *x, __half *x16, int H, int *err,
+                                                                      const ZeroSpans zero)
 {
+    if (blockIdx.x > 0) {
+        grid_dep_launch();
+        grid_dep_wait();   // the previous call's readers of these slices have finished
+        zero_spans(zero, blockIdx.x - 1, gridDim.x - 1);
+        return;
+    }
     extern __shared__ int32_t sm[];
     const int npairs = T * k, chunks = bucket_chunks(E, npairs, ROUTE_THREADS);
     int32_t *hist = sm, *base = sm + (size_t)chunks * E, *s_ids = base + E + 1;
@@ -397,12 +416,14 @@ constexpr int ROUTE_TOKENS_PER_CTA = 256;
 
 __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_topk_kernel(const float *logits, int T, int E, int k,
                                                                      int renorm, int32_t *ids, float *w,
-                                                                     const uint16_t *x, __half *x16, int H, int *err)
+                                                                     const uint16_t *x, __half *x16, int H, int *err,
+                                                                     const ZeroSpans zero)
 {
     grid_dep_launch();   // the next kernel may start its prologue; it waits for this one's results
     grid_dep_wait();
     if (err && blockIdx.x == 0 && threadIdx.x == 0)
         *err = 0;
+    zero_spans(zero, blockIdx.x, gridDim.x);
     const int t0 = blockIdx.x * ROUTE_TOKENS_PER_CTA;
     convert_rows(x, x16, t0, min(T, t0 + ROUTE_TOKENS_PER_CTA), H, threadIdx.x, blockDim.x);
     route_range(logits, t0, min(T, t0 + ROUTE_TOKENS_PER_CTA), E, k, renorm, ids, w, 0, blockDim.x >> 5);
@@ -442,8 +463,14 @@ cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int32_t *ids, float *w,
                          int32_t *offsets, int32_t *perm, int32_t *pos, int32_t *active, int32_t *n_active,
                          int2 *passes, int32_t *n_passes, const uint16_t *x, __half *x16, int H, int *errw,
-                         cudaStream_t s, bool pdl)
+                         cudaStream_t s, bool pdl, const ZeroSpans *zero)
 {
+    ZeroSpans z{};
+    if (zero)
+        z = *zero;
+    const long zwords = z.n[0] + z.n[1] + z.n[2];
+    // clearing CTAs for the fused launch: about 16 words per thread
+    const int zctas = zwords > 0 ? (int)std::min<long>(64, (zwords + 16L * ROUTE_THREADS - 1) / (16L * ROUTE_THREADS)) : 0;
     // dynamic shared memory of a bucketing CTA: at most 32 x 1024 histogram rows
     // + bases (the 1024-thread bucketing CTA, 135 KB), or 16 x 1024 rows + bases
     // + 8192 pair ids + the warm-up scratch (the fused CTA, 112 KB); the kernels'
@@ -465,11 +492,11 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
     if (smem > ROUTE_SMEM_MAX)
         return cudaErrorInvalidValue;
     if (fused)
-        return launch_ex(vq_route_fused_kernel, dim3(1), dim3(ROUTE_THREADS), smem, s, pdl, logits, T, E, k, renorm,
-                         ids, w, offsets, perm, pos, active, n_active, passes, n_passes, x, x16, H, errw);
+        return launch_ex(vq_route_fused_kernel, dim3(1 + zctas), dim3(ROUTE_THREADS), smem, s, pdl, logits, T, E, k,
+                         renorm, ids, w, offsets, perm, pos, active, n_active, passes, n_passes, x, x16, H, errw, z);
     const int ctas = (T + ROUTE_TOKENS_PER_CTA - 1) / ROUTE_TOKENS_PER_CTA;
     cudaError_t err = launch_ex(vq_route_topk_kernel, dim3(ctas), dim3(ROUTE_THREADS), 0, s, pdl, logits, T, E, k,
-                                renorm, ids, w, x, x16, H, errw);
+                                renorm, ids, w, x, x16, H, errw, z);
     if (err != cudaSuccess)
         return err;
     return launch_ex(vq_bucket_kernel, dim3(1), dim3(BUCKET_THREADS), smem, s, pdl, (const int32_t *)ids, T * k, E,
