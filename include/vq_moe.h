@@ -174,7 +174,8 @@ enum { VQ_MODE_DECODE = 0, VQ_MODE_PREFILL = 1 };
  * (VQ_MODE_PREFILL) need for T tokens and top_k. 0 on invalid arguments. */
 size_t vq_moe_workspace_size(const vq_moe_layer *L, int32_t T, int32_t top_k, int32_t mode);
 
-/* MoE SwiGLU layer for decode-sized batches (a few tokens per expert):
+/* MoE SwiGLU layer for decode-sized batches (a few tokens per expert). T = 0
+ * launches nothing and returns VQ_OK; x, logits and y may then be NULL:
  *   y[t] = sum_j w[t, j] * W_down,e_j ( silu(W_gate,e_j x[t]) * (W_up,e_j x[t]) )
  * with (e_j, w[t, j]) from vq_route on `logits` (device fp32 [T, E]).
  * x: device bf16 [T, hidden], 16-byte aligned. y: device [T, hidden] of

@@ -380,8 +380,9 @@ static vq_status check_moe_args(const vq_moe_layer *L, const uint16_t *x, int32_
     vq_status st = check_layer(L);
     if (st != VQ_OK)
         return st;
-    if (!x || !logits || !y || T < 0 || top_k < 1 || top_k > std::min(L->gate.E, 32) || L->gate.E > 4096 ||
-        (y_dtype != VQ_F32 && y_dtype != VQ_BF16) || (long)T * top_k >= (1L << 31))
+    // an empty batch launches nothing, so its x, logits and y may be NULL
+    if ((T > 0 && (!x || !logits || !y)) || T < 0 || top_k < 1 || top_k > std::min(L->gate.E, 32) ||
+        L->gate.E > 4096 || (y_dtype != VQ_F32 && y_dtype != VQ_BF16) || (long)T * top_k >= (1L << 31))
         return VQ_ERR_ARG;
     if (!aligned(x, 16) || !aligned(y, 16))
         return VQ_ERR_ALIGN;
