@@ -397,12 +397,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                         break;
                     tc_fence_after();
                     const uint64_t bdesc = sw128_desc(smem_u32(sm_b + (size_t)st * B_TILE));
-                    for (int m = 0; m < nmod; ++m) {
-                        const uint32_t a_tmem = tmem + acc_cols + (st * nmod + m) * A_COLS;
+                    // the two modules' MMAs alternate: consecutive MMAs into one
+                    // accumulator depend on each other, the two accumulators do not
 #pragma unroll
-                        for (int k16 = 0; k16 < 4; ++k16)
+                    for (int k16 = 0; k16 < 4; ++k16)
+                        for (int m = 0; m < nmod; ++m) {
+                            const uint32_t a_tmem = tmem + acc_cols + (st * nmod + m) * A_COLS;
                             umma_ts(tmem + m * BN, a_tmem + 8 * k16, bdesc + 2 * k16, idesc, (k | k16) != 0);
-                    }
+                        }
                     umma_commit(&empty[st]);
                     if (++st == (uint32_t)a.sa) {
                         st = 0;
