@@ -316,15 +316,30 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
     grid_dep_wait();
 
     // tile prefix over the active experts: tiles[ai] = first global n-tile of expert active[ai]
+    // (warp 2 scans 32 experts per step, so the loads of a step are in flight together)
     const int n_act = *a.n_active;
-    if (threadIdx.x == 0) {
+    if (warp == 2) {
         int run = 0;
-        for (int ai = 0; ai < n_act; ++ai) {
-            tiles[ai] = run;
-            const int e = a.active[ai];
-            run += (a.offsets[e + 1] - a.offsets[e] + BN - 1) / BN;
+        for (int a0 = 0; a0 < n_act; a0 += 32) {
+            const int ai = a0 + lane;
+            int nt = 0;
+            if (ai < n_act) {
+                const int e = a.active[ai];
+                nt = (a.offsets[e + 1] - a.offsets[e] + BN - 1) / BN;
+            }
+            int incl = nt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                if (lane >= o)
+                    incl += v;
+            }
+            if (ai < n_act)
+                tiles[ai] = run + incl - nt;
+            run += __shfl_sync(0xFFFFFFFFu, incl, 31);
         }
-        tiles[n_act] = run;
+        if (lane == 0)
+            tiles[n_act] = run;
     }
     tc_fence_before();
     __syncthreads();
