@@ -28,7 +28,8 @@ def _bf16_of(y32):
 
 CASES = [
     # (E, k, H, I, geometries, dead rows)
-    (8, 3, 512, 320, ((2, 8), (2, 8), (2, 8)), (0, 0, 0)),          # ragged 128-row tile (320 = 2.5 tiles)
+    (8, 3, 512, 320, ((2, 8), (2, 8), (2, 8)), (0, 0, 0)),          # ragged gate/up tile (320 = 2.5 x 128 rows)
+    (8, 3, 320, 256, ((2, 8), (2, 8), (2, 8)), (0, 0, 0)),          # ragged down tile (320 = 2.5 x 128 rows)
     (8, 3, 512, 512, ((4, 9), (4, 9), (4, 9)), (0, 0, 0)),
     (8, 2, 512, 256, ((2, 10), (2, 10), (8, 12)), (21, 17, 0)),      # skipzero gate/up + d=8 down
     (6, 2, 1024, 512, ((4, 11), (4, 11), (4, 11)), (0, 0, 9)),
@@ -58,12 +59,13 @@ def test_prefill_small(case, T):
 
 
 def test_prefill_buckets_span_several_token_tiles():
-    # 4 experts, top-2 of 600 tokens: ~300 tokens per bucket -> 3 ragged 128-token tiles
+    # 4 experts, top-2 of 1200 tokens: ~600 tokens per bucket -> 5 ragged 128-token gate/up tiles
+    # and 3 ragged 256-token down tiles
     E, k, H, I = 4, 2, 512, 256
     oms, layer = _layer(E, H, I, ((2, 8), (2, 8), (2, 8)), seed=77)
     g = synth.rng(82)
-    x = synth.activations(600, H, g)
-    lg = synth.logits_normal(600, E, g)
+    x = synth.activations(1200, H, g)
+    lg = synth.logits_normal(1200, E, g)
     y = layer.prefill(torch.from_numpy(x.view(np.int16)).cuda(), torch.from_numpy(lg).cuda(), k)
     torch.cuda.synchronize()
     assert_close(y.cpu().numpy(), oracle.moe(*oms, x, lg, k), what="multi-tile buckets")

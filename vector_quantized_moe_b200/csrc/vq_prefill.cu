@@ -24,12 +24,15 @@
 // D[row, token] = sum_k W[row, k] X[token, k]: the weight tile is the
 // M=128 operand (in tensor memory), the tokens of the bucket the N operand
 // (16..128, shared memory), so small buckets waste no M rows. Tensor memory
-// holds the accumulators (nmod x 128 columns) and 4 stages of A tiles. Every mbarrier wait is bounded; on a timeout the
-// CTA records an error word, stops, and frees its tensor memory.
+// holds the accumulators (nmod x 128 columns) and 4 stages of A tiles; the MMAs of a
+// tile start once both warpgroups have read the previous tile's accumulators.
+// Every mbarrier wait is bounded; on a timeout the CTA records an error word,
+// stops, and frees its tensor memory.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <climits>
 #include <utility>
 
 #include "vq_device.cuh"
@@ -225,8 +228,8 @@ template <int BN>
 __device__ __forceinline__ Item item_of(long it, int MT, const int *tiles, int n_act, const int32_t *active,
                                         const int32_t *offsets)
 {
-    const int mt = (int)(it % MT);
-    const int ntg = (int)(it / MT);
+    const int mt = (int)it % MT;   // item counts fit 32 bits (a host check)
+    const int ntg = (int)it / MT;
     int lo = 0, hi = n_act;   // last ai with tiles[ai] <= ntg
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
@@ -274,9 +277,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
     int *tiles = reinterpret_cast<int *>(smem + a.off_tiles);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + a.off_bar);
     uint64_t *full_a = bars, *full_b = bars + a.sa, *empty = bars + 2 * a.sa;
-    uint64_t *full_c = bars + 3 * a.sa, *empty_c = full_c + a.sc, *acc_full = empty_c + a.sc;
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(acc_full + 1);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 2);
+    uint64_t *full_c = bars + 3 * a.sa, *empty_c = full_c + a.sc;
+    uint64_t *acc_full = empty_c + a.sc, *acc_empty = acc_full + 1;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(acc_empty + 1);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int nmod = NMOD;
@@ -301,6 +305,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
             mbar_init(&empty_c[s], 128 * NWG);
         }
         mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 128 * NWG);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -399,12 +404,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            uint32_t st = 0, ph = 0;
+            uint32_t st = 0, ph = 0, nacc = 0;
             bool ok = true;
             for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
                 const Item itm = item_of<BN>(it, MT, tiles, n_act, a.active, a.offsets);
                 const int n16 = (itm.n + 15) & ~15;
                 const uint32_t idesc = idesc_f16(BM, n16);
+                // both warpgroups' epilogues of the previous item have read the accumulators
+                if (!(ok = mbar_wait(acc_empty, (nacc & 1) ^ 1, abort_flag, a.err, 9)))
+                    break;
+                ++nacc;
+                tc_fence_after();
                 for (int k = 0; k < ksteps; ++k) {
                     if (!(ok = mbar_wait(&full_a[st], ph, abort_flag, a.err, 4)))
                         break;
@@ -540,6 +550,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                 }
             }
             tc_fence_before();
+            mbar_arrive(acc_empty);   // the next item's MMAs may overwrite the accumulators
         }
     }
 
@@ -627,7 +638,7 @@ SmemPlan smem_plan(int nmod, int d, int bits, int E)
         p.off_cb = p.off_c + p.sc * code_stage;
         p.off_tiles = p.off_cb + cb;
         p.off_bar = (uint32_t)align_up(p.off_tiles + tiles, 8);
-        p.total = p.off_bar + (3 * sa + 2 * p.sc + 1) * 8 + 16 + 1024;
+        p.total = p.off_bar + (3 * sa + 2 * p.sc + 2) * 8 + 16 + 1024;
         if (p.total <= limit + 1024)
             return p;
     }
@@ -723,6 +734,12 @@ vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const flo
     __half *hh = ws_at<__half>(ws, p.h);
     float *dp = ws_at<float>(ws, p.dp);
     const long tk = (long)T * k;
+    // the kernels count work items in 32 bits
+    for (int m = 0; m < 2; ++m) {
+        const long bn = bn_of(2 - m), rows = m ? H : I;
+        if (((tk + bn - 1) / bn + E) * ((rows + BM - 1) / BM) >= INT_MAX)
+            return VQ_ERR_UNSUPPORTED;
+    }
 
     trace_point(0, s);
     cudaError_t e = launch_route(logits, T, E, k, renorm, ids, w, offsets, perm, pos, active, nact, nullptr, nullptr,
