@@ -39,6 +39,9 @@ from synth import workloads as wl  # noqa: E402
 METRIC = "VQ expert decode HBM GB/s"
 UNIT = "GB/s"
 N_DRAWS = 16
+# the other decode workloads, reported under "extra": (layer, tokens)
+OTHER_DECODE = {"decode_d4k512_T16": (wl.DECODE_D4K512, 16), "decode_d4k2048_T16": (wl.DECODE_D4K2048, 16),
+                "decode_skipzero_T1": (wl.SKIPZERO_MIXED, 1)}
 
 
 def _peaks():
@@ -225,6 +228,22 @@ def run_ours(args):
             fn(i)
         torch.cuda.synchronize()
         return
+    if args.only in OTHER_DECODE:
+        # profiler runs of another decode workload: warm-up, then the steps
+        import dataclasses
+        spec_x, T_x = OTHER_DECODE[args.only]
+        if args.small:
+            spec_x = dataclasses.replace(spec_x, E=64, name=spec_x.name.replace(f"e{spec_x.E}", "e64"))
+        mds = wl.layer_modules(spec_x, raw=False, row_words=lambda c, g: vq.packed_words(1, c // g.d, g.bits))
+        layer = vq.MoELayer(*[lib_module(m, device=dev) for m in mds])
+        x, lg = wl.layer_inputs(spec_x, T_x, 200)
+        xt, lt = torch.from_numpy(x.view(np.int16)).to(dev), torch.from_numpy(lg).to(dev)
+        y = torch.empty((T_x, spec_x.hidden), dtype=torch.float32, device=dev)
+        wsp = layer.workspace(T_x, spec_x.top_k, vq.VQ_MODE_DECODE, dev)
+        for i in range(args.warmup + args.steps):
+            layer.decode(xt, lt, spec_x.top_k, out=y, workspace=wsp)
+        torch.cuda.synchronize()
+        return
 
     spec = wl.DECODE_D2K256
     if args.small:
@@ -353,6 +372,10 @@ def run_ours(args):
         del layer, mods
         torch.cuda.empty_cache()
         extra["prefill"] = measure_prefill(torch, vq, dev, min(args.steps, 20), args.warmup)
+        for key, (spec_x, T_x) in OTHER_DECODE.items():
+            extra[key] = measure_decode_layer(torch, vq, spec_x, T_x, dev, min(args.steps, 100), args.warmup)
+        extra["prefill_skipzero_T2048"] = measure_prefill(torch, vq, dev, min(args.steps, 20), args.warmup,
+                                                          spec=wl.SKIPZERO_MIXED, T=2048)
 
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
@@ -405,6 +428,49 @@ def _traced(torch, vq, fn, steps, n_events=6):
     return np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(n_events - 1)] for i in range(steps)])
 
 
+def measure_decode_layer(torch, vq, spec, T, dev, steps, warmup):
+    """Another decode workload (its own layer, 16 rotating routing draws): step GB/s and the gate+up
+    launch's fraction of the measured HBM bandwidth."""
+    from tests.helpers import lib_module
+    mds = wl.layer_modules(spec, raw=False, row_words=lambda c, g: vq.packed_words(1, c // g.d, g.bits))
+    per_expert = [_module_bytes(m) for m in mds]
+    cb_bytes = sum(m.codebook.nbytes for m in mds)
+    gu_cb = mds[0].codebook.nbytes + mds[1].codebook.nbytes
+    layer = vq.MoELayer(*[lib_module(m, device=dev) for m in mds])
+    del mds
+    draws = [wl.layer_inputs(spec, T, 200 + i) for i in range(N_DRAWS)]
+    xs = [torch.from_numpy(x.view(np.int16)).to(dev) for x, _ in draws]
+    lgs = [torch.from_numpy(lg).to(dev) for _, lg in draws]
+    y = torch.empty((T, spec.hidden), dtype=torch.float32, device=dev)
+    ws = layer.workspace(T, spec.top_k, vq.VQ_MODE_DECODE, dev)
+    io = T * spec.hidden * 2 + T * spec.E * 4 + T * spec.hidden * 4
+    step_bytes, gu_bytes = [], []
+    for lg in lgs:
+        _, _, off, _ = vq.route(lg, spec.top_k)
+        touched = np.nonzero(np.diff(off.cpu().numpy()) > 0)[0]
+        g, u, d = (float(p[touched].sum()) for p in per_expert)
+        step_bytes.append(g + u + d + cb_bytes + io)
+        gu_bytes.append(g + u + gu_cb + T * spec.hidden * 2)
+    fn = lambda i: layer.decode(xs[i % N_DRAWS], lgs[i % N_DRAWS], spec.top_k, out=y, workspace=ws)
+    for i in range(warmup):
+        fn(i)
+    ms = _time_steps(torch, fn, steps)
+    stage = _traced(torch, vq, fn, steps).mean(axis=0)
+    hbm, _, _, src = _peaks()
+    gu_ach = float(np.mean([gu_bytes[i % N_DRAWS] for i in range(steps)])) / (stage[1] * 1e-3) / 1e9
+    out = {"workload": spec.name, "T": T, "value": sum(step_bytes[i % N_DRAWS] for i in range(steps)) / (ms * 1e-3) / 1e9,
+           "unit": UNIT, "ms_per_step": ms / steps, "tokens_per_s": T * steps / (ms * 1e-3),
+           "stage_ms": {"route": float(stage[0]), "gate_up_gemv": float(stage[1]), "swiglu": float(stage[2]),
+                        "down_gemv": float(stage[3]), "combine": float(stage[4])},
+           "gate_up_stage": {"achieved": gu_ach, "peak": hbm, "unit": "GB/s", "frac": gu_ach / hbm,
+                       "peak_source": f"{src} hbm_gbs"},
+           "geometry": f"gate {spec.gate.d}/{spec.gate.bits}b, up {spec.up.d}/{spec.up.bits}b, "
+                       f"down {spec.down.d}/{spec.down.bits}b (d / code bits)"}
+    del layer, xs, lgs, y, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 def measure_decode_t1(torch, vq, layer, spec, per_expert, cb_bytes, dev, steps, warmup):
     """Same layer, one token per step (latency-bound case), 16 rotating routing draws."""
     draws = [wl.layer_inputs(spec, 1, 100 + i) for i in range(N_DRAWS)]
@@ -426,17 +492,21 @@ def measure_decode_t1(torch, vq, layer, spec, per_expert, cb_bytes, dev, steps, 
             "tokens_per_s": steps / (ms * 1e-3), "launches_per_step": 5}
 
 
-def measure_prefill(torch, vq, dev, steps, warmup, small=False, ncu_mode=False):
-    """MoE prefill layer, d=4/K=512, 4096 tokens, Zipf(1.1) routing: tcgen05 grouped GEMM path."""
+def measure_prefill(torch, vq, dev, steps, warmup, small=False, ncu_mode=False, spec=None, T=None):
+    """MoE prefill layer (default: d=4/K=512, 4096 tokens, Zipf(1.1) routing): tcgen05 grouped GEMM path.
+    FLOPs count live weights only; GB/s counts the touched experts' live codes and scales."""
     import dataclasses
     from tests.helpers import lib_module
-    spec = wl.PREFILL_D4K512
-    T = spec.batches[0]
+    default = spec is None
+    if default:
+        spec = wl.PREFILL_D4K512
+        T = spec.batches[0]
     if small:
         spec = dataclasses.replace(spec, E=64, name=spec.name.replace("e256", "e64"))
         T = 1024
     mds = wl.layer_modules(spec, raw=False, row_words=lambda c, g: vq.packed_words(1, c // g.d, g.bits))
     layer = vq.MoELayer(*[lib_module(m, device=dev) for m in mds])
+    per_expert = [_module_bytes(m) for m in mds]
     draws = [wl.layer_inputs(spec, T, i) for i in range(2)]
     xs = [torch.from_numpy(x.view(np.int16)).to(dev) for x, _ in draws]
     lgs = [torch.from_numpy(lg).to(dev) for _, lg in draws]
@@ -447,24 +517,38 @@ def measure_prefill(torch, vq, dev, steps, warmup, small=False, ncu_mode=False):
         fn(i)
     torch.cuda.synchronize()
     pairs = T * spec.top_k
-    flops_gu = 2.0 * pairs * 2 * spec.inter * spec.hidden
-    flops_dn = 2.0 * pairs * spec.hidden * spec.inter
+    # live weights only (skipzero rows are never multiplied)
+    flops_gu = 2.0 * pairs * (2 * spec.inter - spec.dead_gate - spec.dead_up) * spec.hidden
+    flops_dn = 2.0 * pairs * (spec.hidden - spec.dead_down) * spec.inter
     if ncu_mode:
         return layer, fn
+    # weight bytes streamed per step: live codes + scales of the experts the two draws touch
+    wbytes = []
+    for lg in lgs:
+        _, _, off, _ = vq.route(lg, spec.top_k)
+        touched = np.nonzero(np.diff(off.cpu().numpy()) > 0)[0]
+        wbytes.append([float(p[touched].sum()) for p in per_expert])
+    gu_w = float(np.mean([b[0] + b[1] for b in wbytes]))
+    step_w = float(np.mean([sum(b) for b in wbytes]))
     ms = _time_steps(torch, fn, steps)
     stage = _traced(torch, vq, fn, steps).mean(axis=0)
-    _, tf_burst, tf_sust, src = _peaks()
+    hbm, tf_burst, tf_sust, src = _peaks()
     gu_tflops = flops_gu / (stage[2] * 1e-3) / 1e12
+    gu_gbs = gu_w / (stage[2] * 1e-3) / 1e9
     out = {"workload": spec.name, "T": T, "metric": "prefill TFLOP/s", "unit": "TFLOP/s",
            "value": (flops_gu + flops_dn) / (ms / steps * 1e-3) / 1e12, "ms_per_step": ms / steps,
            "tokens_per_s": T * steps / (ms * 1e-3), "flops_per_step": flops_gu + flops_dn,
+           "weights_gbs": step_w / (ms / steps * 1e-3) / 1e9,
            "stage_ms": {"route": float(stage[0]), "gather": float(stage[1]), "gate_up_gemm": float(stage[2]),
                         "down_gemm": float(stage[3]), "combine": float(stage[4])},
            "roofline": {"bound": "tensor", "achieved": gu_tflops, "peak": tf_burst, "unit": "TFLOP/s",
-                        "frac": gu_tflops / tf_burst, "traffic": _traffic_per_launch("prefill_gemm_gate_up"),
-                        "kernel": "vq_prefill_gemm_kernel<4,9,2> (gate+up, SwiGLU epilogue)",
+                        "frac": gu_tflops / tf_burst,
+                        "traffic": _traffic_per_launch("prefill_gemm_gate_up") if default else None,
+                        "kernel": f"vq_prefill_gemm_kernel<{spec.gate.d},{spec.gate.bits},2> (gate+up, SwiGLU epilogue)",
                         "peak_source": f"{src} bf16_tflops (fp16 runs at the bf16 rate)",
                         "flops_per_launch": flops_gu, "ms_per_launch": float(stage[2])},
+           "gate_up_hbm": {"achieved": gu_gbs, "peak": hbm, "unit": "GB/s", "frac": gu_gbs / hbm,
+                           "bytes_per_launch": gu_w},
            "launches_per_step": 7}
     del layer
     torch.cuda.empty_cache()
@@ -502,9 +586,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ncu", action="store_true", help="only warmup + timed steps, for profiler captures")
     ap.add_argument("--small", action="store_true", help="64-expert variant of the workload (profiling)")
-    ap.add_argument("--only", choices=("decode", "prefill"), default="decode",
+    ap.add_argument("--only", choices=("decode", "prefill", *OTHER_DECODE), default="decode",
                     help="with --ncu: which path the profiler run exercises")
-    ap.add_argument("--no-extra", action="store_true", help="skip the 1-token decode and prefill lines")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' lines")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -27,8 +27,6 @@ int num_sms()
 
 namespace {
 
-constexpr size_t CODEBOOK_SMEM_BUDGET = 100 * 1024;   // replicated codebook per CTA
-
 bool geometry_ok(int d, int bits)
 {
 #define VQ_GEO_OK(D_, B_) \
@@ -148,15 +146,8 @@ ModDev make_moddev(const vq_module &m)
     d.ngroups = m.cols / 64;
     d.bm_words = (m.rows + 31) / 32;
     d.live_rows = m.live_bitmap ? m.live_rows : (int64_t)m.E * m.rows;
-    const size_t entry = std::max(4, 2 * m.d);
-    const int full = (int)(128 / entry);
-    int rep = full;
-    while (rep > 1 && ((size_t)1 << m.bits) * entry * rep > CODEBOOK_SMEM_BUDGET)
-        rep /= 2;
-    d.rep = rep;
-    d.log_rep = 0;
-    while ((1 << d.log_rep) < rep)
-        ++d.log_rep;
+    d.log_rep = codebook_log_rep(m.d, m.bits);
+    d.rep = 1 << d.log_rep;
     return d;
 }
 

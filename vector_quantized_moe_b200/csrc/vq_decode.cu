@@ -38,6 +38,9 @@ struct Geo {
     static constexpr int LW = ALIGNED ? NW : NW + 1;   // words loaded from the row
     static constexpr int EW = D <= 2 ? 1 : D / 2;      // shared-memory words per codebook entry
     static constexpr uint32_t MASK = (1u << BITS) - 1u;
+    static constexpr int LOG_REP = codebook_log_rep(D, BITS);   // replicas per entry (log2)
+    // code -> byte offset of its replica block: code << LSH (entries of 4 * EW bytes)
+    static constexpr int LSH = LOG_REP + (EW == 1 ? 2 : EW == 2 ? 3 : 4);
 };
 
 // Load the words holding lane-quarter j (= 4*group + t) of a packed row.
@@ -84,6 +87,55 @@ __device__ __forceinline__ void extract_codes(const uint32_t (&w)[Geo<D, BITS>::
             c[k] = (n[wi] >> sh) & G::MASK;
         else
             c[k] = __funnelshift_r(n[wi], n[wi + 1], sh) & G::MASK;
+    }
+}
+
+// The byte offsets (in the shared-memory codebook) of the lane's replica of
+// each of its CODES codes: code k sits at bit o + k * BITS of the loaded
+// words, and its offset (code << LSH) | rep_off takes one shift and one
+// mask-or.
+template <int D, int BITS>
+__device__ __forceinline__ void code_offsets(const uint32_t (&w)[Geo<D, BITS>::LW], int o, uint32_t rep_off,
+                                             uint32_t (&off)[Geo<D, BITS>::CODES])
+{
+    using G = Geo<D, BITS>;
+    static_assert(BITS + G::LSH <= 32, "offsets fit 32 bits");
+    uint32_t n[G::NW];
+#pragma unroll
+    for (int i = 0; i < G::NW; ++i)
+        n[i] = G::ALIGNED ? w[i] : __funnelshift_r(w[i], w[i + (G::ALIGNED ? 0 : 1)], o);
+#pragma unroll
+    for (int k = 0; k < G::CODES; ++k) {
+        const int p = k * BITS, wi = p >> 5, sh = p & 31;
+        uint32_t v;
+        int at;   // bit of v where the code starts
+        if (sh + BITS <= 32) {
+            v = n[wi];
+            at = sh;
+        } else {
+            v = __funnelshift_r(n[wi], n[wi + 1], sh);
+            at = 0;
+        }
+        const uint32_t x = at >= G::LSH ? v >> (at - G::LSH) : v << (G::LSH - at);
+        off[k] = (x & (G::MASK << G::LSH)) | rep_off;
+    }
+}
+
+// a_words from byte offsets formed by code_offsets (d >= 2).
+template <int D>
+__device__ __forceinline__ void a_words_off(const char *cbb, const uint32_t *off, int s, uint32_t &lo, uint32_t &hi)
+{
+    if constexpr (D == 2) {
+        lo = *reinterpret_cast<const uint32_t *>(cbb + off[2 * s]);
+        hi = *reinterpret_cast<const uint32_t *>(cbb + off[2 * s + 1]);
+    } else if constexpr (D == 4) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(cbb + off[s]);
+        lo = v.x;
+        hi = v.y;
+    } else {
+        const uint4 v = *reinterpret_cast<const uint4 *>(cbb + off[s >> 1]);
+        lo = (s & 1) ? v.z : v.x;
+        hi = (s & 1) ? v.w : v.y;
     }
 }
 
@@ -642,6 +694,8 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
     }
     int rows = 0, rep = 0, log_rep = 0, r0 = 0;
     uint32_t lane_sel = 0, aoff = 0;
+    // the lane's replica within an entry's block of replicas (d >= 2)
+    const uint32_t rep_off = (uint32_t)(lane & ((1 << G::LOG_REP) - 1)) * (4 * G::EW);
     float acc[TG_RT][4];
     long item = u0 / spp;
     int j = (int)(u0 % spp);
@@ -757,13 +811,18 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                 if (lane == 0)
                     mbar_arrive(&empty[slot]);
             }
+            // codes (d=1) or their codebook byte offsets (d >= 2)
             uint32_t c[GP][TG_RL][G::CODES];
             if constexpr (!FAST) {
 #pragma unroll
                 for (int uu = 0; uu < GP; ++uu)
 #pragma unroll
-                    for (int i = 0; i < TG_RL; ++i)
-                        extract_codes<D, BITS>(cw[uu][i], co[uu], c[uu][i]);
+                    for (int i = 0; i < TG_RL; ++i) {
+                        if constexpr (D == 1)
+                            extract_codes<D, BITS>(cw[uu][i], co[uu], c[uu][i]);
+                        else
+                            code_offsets<D, BITS>(cw[uu][i], co[uu], rep_off, c[uu][i]);
+                    }
             }
             float tmp[GP][TG_RT][4];
 #pragma unroll
@@ -790,9 +849,13 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                                 Aw[2 * h + 1] = *reinterpret_cast<const uint32_t *>(
                                     cbb + __byte_perm(cw[uu][2 * rt + 1][s >> 1], lane_sel, sel));
                             }
-                        } else {
+                        } else if constexpr (D == 1) {
                             a_words<D>(cbs, log_rep, rep, c[uu][2 * rt], s, Aw[0], Aw[2]);
                             a_words<D>(cbs, log_rep, rep, c[uu][2 * rt + 1], s, Aw[1], Aw[3]);
+                        } else {
+                            const char *cbb = reinterpret_cast<const char *>(cbs);
+                            a_words_off<D>(cbb, c[uu][2 * rt], s, Aw[0], Aw[2]);
+                            a_words_off<D>(cbb, c[uu][2 * rt + 1], s, Aw[1], Aw[3]);
                         }
                         mma_16816(tmp[uu][rt], Aw, bw[uu][2 * s], bw[uu][2 * s + 1]);
                     }

@@ -18,6 +18,22 @@
 
 namespace vq {
 
+constexpr size_t CODEBOOK_SMEM_BUDGET = 100 * 1024;   // replicated codebook per CTA (decode)
+
+// Decode codebook replicas in shared memory (log2): the per-lane count that
+// spreads a warp's lookups over all banks (128 bytes / entry; d=1 entries take
+// a 32-bit word), halved until the module's replicated codebook fits the budget.
+__host__ __device__ constexpr int codebook_log_rep(int d, int bits)
+{
+    const long entry = d <= 2 ? 4 : 2 * d;
+    int lr = 0;
+    while ((1L << (lr + 1)) <= 128 / entry)
+        ++lr;
+    while (lr > 0 && (1L << bits) * entry * (1L << lr) > (long)CODEBOOK_SMEM_BUDGET)
+        --lr;
+    return lr;
+}
+
 // A module as the kernels see it.
 struct ModDev {
     const uint32_t *codes;
