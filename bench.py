@@ -376,6 +376,7 @@ def run_ours(args):
             extra[key] = measure_decode_layer(torch, vq, spec_x, T_x, dev, min(args.steps, 100), args.warmup)
         extra["prefill_skipzero_T2048"] = measure_prefill(torch, vq, dev, min(args.steps, 20), args.warmup,
                                                           spec=wl.SKIPZERO_MIXED, T=2048)
+        extra["prefill_chunked_T8192"] = measure_prefill_chunked(torch, vq, dev, min(args.steps, 5), args.warmup)
 
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
@@ -549,8 +550,36 @@ def measure_prefill(torch, vq, dev, steps, warmup, small=False, ncu_mode=False, 
                         "flops_per_launch": flops_gu, "ms_per_launch": float(stage[2])},
            "gate_up_hbm": {"achieved": gu_gbs, "peak": hbm, "unit": "GB/s", "frac": gu_gbs / hbm,
                            "bytes_per_launch": gu_w},
-           "launches_per_step": 7}
+           "launches_per_step": 6}
     del layer
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_prefill_chunked(torch, vq, dev, steps, warmup, T=8192, chunk=2048):
+    """A long prompt of the Zipf prefill layer in `chunk`-token chunks through one chunk-sized
+    workspace (vq_moe_prefill_chunked): TFLOP/s and the workspace it needs against one call's."""
+    from tests.helpers import lib_module
+    spec = wl.PREFILL_D4K512
+    mds = wl.layer_modules(spec, raw=False, row_words=lambda c, g: vq.packed_words(1, c // g.d, g.bits))
+    layer = vq.MoELayer(*[lib_module(m, device=dev) for m in mds])
+    del mds
+    x, lg = wl.layer_inputs(spec, T, 300)
+    xt, lt = torch.from_numpy(x.view(np.int16)).to(dev), torch.from_numpy(lg).to(dev)
+    y = torch.empty((T, spec.hidden), dtype=torch.float32, device=dev)
+    ws = layer.workspace(chunk, spec.top_k, vq.VQ_MODE_PREFILL, dev)
+    fn = lambda i: layer.prefill_chunked(xt, lt, spec.top_k, chunk=chunk, out=y, workspace=ws)
+    for i in range(warmup):
+        fn(i)
+    ms = _time_steps(torch, fn, steps)
+    flops = 2.0 * T * spec.top_k * 3 * spec.inter * spec.hidden
+    out = {"workload": spec.name, "T": T, "chunk": chunk, "metric": "prefill TFLOP/s", "unit": "TFLOP/s",
+           "value": flops / (ms / steps * 1e-3) / 1e12, "ms_per_step": ms / steps,
+           "tokens_per_s": T * steps / (ms * 1e-3),
+           "workspace_bytes": layer.workspace_size(chunk, spec.top_k, vq.VQ_MODE_PREFILL),
+           "workspace_bytes_one_call": layer.workspace_size(T, spec.top_k, vq.VQ_MODE_PREFILL),
+           "launches_per_step": 6 * ((T + chunk - 1) // chunk)}
+    del layer, xt, lt, y, ws
     torch.cuda.empty_cache()
     return out
 

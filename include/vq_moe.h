@@ -200,6 +200,21 @@ vq_status vq_moe_prefill(const vq_moe_layer *L, const uint16_t *x, int32_t T, co
                          int32_t top_k, int32_t renorm, void *y, int32_t y_dtype, void *workspace,
                          size_t ws_bytes, void *stream);
 
+/* Prefill of a long prompt in chunks, so that scratch memory is bounded by
+ * the chunk rather than the prompt (the gemma-4 and Qwen3.5 VQ model cards
+ * run prefill in 2048-token chunks). Tokens [c0, c0 + chunk) of x and logits
+ * go through vq_moe_prefill into rows [c0, c0 + chunk) of y, one chunk after
+ * another on `stream`; the last chunk takes the remaining tokens. Each
+ * token's output depends only on its own x row and logits, so the result is
+ * vq_moe_prefill's over all T tokens. The workspace is sized for one chunk:
+ * vq_moe_workspace_size(L, min(T, chunk), top_k, VQ_MODE_PREFILL) bytes, and
+ * is reused by every chunk. chunk < 1 returns VQ_ERR_ARG; other errors as
+ * vq_moe_prefill (a chunk that fails stops the loop; earlier chunks stay
+ * queued). */
+vq_status vq_moe_prefill_chunked(const vq_moe_layer *L, const uint16_t *x, int32_t T, const float *logits,
+                                 int32_t top_k, int32_t renorm, int32_t chunk, void *y, int32_t y_dtype,
+                                 void *workspace, size_t ws_bytes, void *stream);
+
 /* Diagnostic (synchronises `stream`). Every wait of the library's pipelined
  * kernels on an on-chip barrier is bounded; a kernel that gives up records a
  * nonzero word at offset 0 of the MoE workspace it ran with (the routing

@@ -103,3 +103,14 @@ def test_workspace_size_monotone():
     b = vq._L().vq_moe_workspace_size(ctypes.byref(L), 64, 1, 0)
     assert 0 < a < b
     assert vq._L().vq_moe_workspace_size(ctypes.byref(L), 4, 3, 0) == 0   # top_k > E
+
+
+def test_prefill_chunked_validates_before_launch():
+    # fake (never dereferenced) pointers: chunk < 1 fails validation, an empty prompt queues nothing
+    m = _null_module()
+    down = _null_module(rows=128, cols=64)
+    L = vq.vq_moe_layer(m, m, down)
+    f = vq._L().vq_moe_prefill_chunked
+    assert f(ctypes.byref(L), 4096, 4, 8192, 1, 1, 0, 16384, 0, 65536, 1 << 20, None) == 1
+    assert f(ctypes.byref(L), 4096, 4, 8192, 1, 1, -3, 16384, 0, 65536, 1 << 20, None) == 1
+    assert f(ctypes.byref(L), None, 0, None, 1, 1, 5, None, 0, 65536, 1 << 20, None) == 0

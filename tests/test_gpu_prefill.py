@@ -71,6 +71,29 @@ def test_prefill_buckets_span_several_token_tiles():
     assert_close(y.cpu().numpy(), oracle.moe(*oms, x, lg, k), what="multi-tile buckets")
 
 
+@pytest.mark.parametrize("T,chunk", [(600, 256), (700, 700), (1000, 333), (5, 2)])
+def test_prefill_chunked_matches_one_call(T, chunk):
+    # chunk after chunk through one chunk-sized workspace: every token's output equals the
+    # one-call prefill bit for bit (it depends only on its own row), and the oracle on samples
+    E, k, H, I = 8, 3, 512, 256
+    oms, layer = _layer(E, H, I, ((2, 8), (2, 8), (2, 8)), seed=91)
+    g = synth.rng(83, T, chunk)
+    x = synth.activations(T, H, g)
+    lg = synth.logits_normal(T, E, g)
+    xt = torch.from_numpy(x.view(np.int16)).cuda()
+    lt = torch.from_numpy(lg).cuda()
+    y = layer.prefill(xt, lt, k)
+    ws = torch.empty(layer.workspace_size(min(T, chunk), k, vq.VQ_MODE_PREFILL) + 256, dtype=torch.uint8,
+                     device="cuda")
+    yc = layer.prefill_chunked(xt, lt, k, chunk=chunk, workspace=ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(yc.cpu().numpy().view(np.uint32), y.cpu().numpy().view(np.uint32))
+    tok = np.unique(np.array([0, chunk - 1, chunk % T, T // 2, T - 1]) % T)
+    assert_close(yc.cpu().numpy()[tok], oracle.moe(*oms, x, lg, k, tokens=tok), what=f"chunked T{T} c{chunk}")
+    if T > chunk:
+        assert layer.workspace_size(chunk, k, vq.VQ_MODE_PREFILL) < layer.workspace_size(T, k, vq.VQ_MODE_PREFILL)
+
+
 def test_prefill_rejects_unaligned_geometry():
     # d=4 / 9-bit needs cols to be a multiple of 512 for whole 16-byte code chunks
     E, H, I = 4, 256, 512
@@ -97,6 +120,11 @@ def test_prefill_full_size(spec, T, sample):
     tok = np.array(sample)
     ref = oracle.moe(*oms, x, lg, spec.top_k, tokens=tok)
     assert_close(y.cpu().numpy()[tok], ref, what=f"{spec.name} T{T}")
+    # in ragged chunks through a chunk-sized workspace: the same outputs bit for bit
+    yc = layer.prefill_chunked(xt, lt, spec.top_k, chunk=T // 2 + 7)
+    torch.cuda.synchronize()
+    assert np.array_equal(yc.cpu().numpy().view(np.uint32), y.cpu().numpy().view(np.uint32))
+    del yc
     # every token: decode path and prefill path agree
     yd = layer.decode(xt, lt, spec.top_k)
     torch.cuda.synchronize()

@@ -63,6 +63,7 @@ def _load():
         "vq_moe_workspace_size": (SZ, [LP, I32, I32, I32]),
         "vq_moe_decode": (ctypes.c_int, [LP, P, I32, P, I32, I32, P, I32, P, SZ, P]),
         "vq_moe_prefill": (ctypes.c_int, [LP, P, I32, P, I32, I32, P, I32, P, SZ, P]),
+        "vq_moe_prefill_chunked": (ctypes.c_int, [LP, P, I32, P, I32, I32, I32, P, I32, P, SZ, P]),
         "vq_set_trace_events": (ctypes.c_int, [P, I32]),
         "vq_moe_check": (ctypes.c_int, [P, P]),
         "vq_moe_decode_noalloc": (ctypes.c_int, [LP, P, I32, P, I32, I32, P, I32, P]),
@@ -315,3 +316,21 @@ class MoELayer:
         """y [T, hidden] for prefill-sized batches (vq_moe_prefill, tcgen05 grouped GEMM)."""
         return self._run(_L().vq_moe_prefill, "vq_moe_prefill", VQ_MODE_PREFILL, x, logits, top_k, renorm, out,
                          out_dtype, workspace, stream)
+
+    def prefill_chunked(self, x, logits, top_k: int, chunk: int = 2048, renorm: bool = True, out=None,
+                        out_dtype=None, workspace=None, stream=None):
+        """y [T, hidden] for a long prompt, `chunk` tokens at a time through one chunk-sized
+        workspace (vq_moe_prefill_chunked)."""
+        torch = _torch()
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty((T, self.hidden), dtype=out_dtype or torch.float32, device=x.device)
+        ws = workspace if workspace is not None else self.workspace(max(1, min(T, chunk)), top_k, VQ_MODE_PREFILL,
+                                                                     x.device)
+        base = ws.data_ptr()
+        aligned = (base + 255) // 256 * 256
+        nbytes = ws.numel() - (aligned - base)
+        _check(_L().vq_moe_prefill_chunked(ctypes.byref(self._s), x.data_ptr(), T, logits.data_ptr(), top_k,
+                                            int(bool(renorm)), int(chunk), out.data_ptr(), _dt(out.dtype), aligned,
+                                            nbytes, _stream(stream)), "vq_moe_prefill_chunked")
+        return out

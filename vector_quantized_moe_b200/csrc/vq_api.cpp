@@ -525,4 +525,26 @@ vq_status vq_moe_prefill(const vq_moe_layer *L, const uint16_t *x, int32_t T, co
     return run_prefill(L, x, T, logits, top_k, renorm, y, y_dtype, workspace, ws_bytes, (cudaStream_t)stream);
 }
 
+vq_status vq_moe_prefill_chunked(const vq_moe_layer *L, const uint16_t *x, int32_t T, const float *logits,
+                                 int32_t top_k, int32_t renorm, int32_t chunk, void *y, int32_t y_dtype,
+                                 void *workspace, size_t ws_bytes, void *stream)
+{
+    vq_status st = check_moe_args(L, x, T, logits, top_k, y, y_dtype, workspace);
+    if (st != VQ_OK)
+        return st;
+    if (chunk < 1)
+        return VQ_ERR_ARG;
+    const int H = L->gate.cols, E = L->gate.E;
+    const size_t ybytes = y_dtype == VQ_F32 ? 4 : 2;
+    for (int32_t c0 = 0; c0 < T; c0 += chunk) {
+        const int32_t n = std::min(chunk, T - c0);
+        st = run_prefill(L, x + (size_t)c0 * H, n, logits + (size_t)c0 * E, top_k, renorm,
+                         static_cast<char *>(y) + (size_t)c0 * H * ybytes, y_dtype, workspace, ws_bytes,
+                         (cudaStream_t)stream);
+        if (st != VQ_OK)
+            return st;
+    }
+    return VQ_OK;
+}
+
 }  // extern "C"
