@@ -5,7 +5,8 @@ legs may import this package. The CUDA library never does, and nothing here
 imports the library: the two share no code.
 
 The arithmetic lives in vq_oracle.c (plain C, double precision); this file
-builds it with gcc and marshals numpy arrays through ctypes. Each function
+builds it with gcc and marshals numpy arrays through ctypes. The data-free
+VQ fit (k-means over weight subvectors) is oracle/fit.py, plain numpy. Each function
 says which passage of the VQ model cards it follows; the readings of silent
 points are listed in vq_oracle.c's header and in the design doc.
 

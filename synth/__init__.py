@@ -13,7 +13,10 @@ Distributions follow the workloads of the VQ-MoE model cards:
   * codes uniform over the K = 2**bits codebook entries,
   * activations N(0, 1) stored as bf16,
   * router logits N(0, 1) fp32, or Zipf(s)-skewed: -s*ln(rank_e) + Gumbel(0, 1),
-  * skipzero: a seeded random set of dead output rows per (expert, module).
+  * skipzero: a seeded random set of dead output rows per (expert, module),
+  * expert weights for the data-free fit: N(0, 0.02) stored as bf16 (a bf16
+    checkpoint), the k-means subsample and its initial centroids drawn as
+    subvector indices.
 """
 from __future__ import annotations
 
@@ -22,6 +25,7 @@ import numpy as np
 __all__ = [
     "rng", "bf16_bits", "f16_bits", "codebook", "scales", "raw_codes",
     "live_bitmap", "random_words", "activations", "logits_normal", "logits_zipf",
+    "weights", "fit_draw",
 ]
 
 
@@ -109,3 +113,16 @@ def logits_zipf(T: int, E: int, s: float, g: np.random.Generator) -> np.ndarray:
     base = -s * np.log(rank)
     gum = g.gumbel(0.0, 1.0, size=(T, E))
     return (base[None, :] + gum).astype(np.float32)
+
+
+def weights(rows: int, cols: int, g: np.random.Generator, sigma: float = 0.02) -> np.ndarray:
+    """A bf16 weight tensor [rows, cols] (bit patterns), entries N(0, sigma)."""
+    return bf16_bits(g.normal(0.0, sigma, size=(rows, cols)))
+
+
+def fit_draw(n_sub: int, n_sample: int, K: int, g: np.random.Generator):
+    """The k-means subsample (n_sample distinct subvector indices, sorted) and
+    K distinct initial centroids drawn from it (subvector indices), int32."""
+    sample = np.sort(g.choice(n_sub, size=n_sample, replace=False)).astype(np.int32)
+    init = sample[g.choice(n_sample, size=K, replace=False)].astype(np.int32)
+    return sample, init
