@@ -34,6 +34,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+import synth  # noqa: E402
 from synth import workloads as wl  # noqa: E402
 
 METRIC = "VQ expert decode HBM GB/s"
@@ -377,6 +378,7 @@ def run_ours(args):
         extra["prefill_skipzero_T2048"] = measure_prefill(torch, vq, dev, min(args.steps, 20), args.warmup,
                                                           spec=wl.SKIPZERO_MIXED, T=2048)
         extra["prefill_chunked_T8192"] = measure_prefill_chunked(torch, vq, dev, min(args.steps, 5), args.warmup)
+        extra["fit_d4k512"] = measure_fit(torch, vq, dev, min(args.steps, 5), args.warmup)
 
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
@@ -582,6 +584,32 @@ def measure_prefill_chunked(torch, vq, dev, steps, warmup, T=8192, chunk=2048):
     del layer, xt, lt, y, ws
     torch.cuda.empty_cache()
     return out
+
+
+def measure_fit(torch, vq, dev, steps, warmup, rows=2048, cols=6144, d=4, K=512, n_sample=65536, iters=10):
+    """Data-free VQ fit of one expert tensor (vq_fit): Lloyd steps on a subsample, then the codes
+    of every subvector. Work = squared-distance evaluations (point x centroid); each takes 3d
+    fp32 operations on the CUDA cores, so the roofline is the fp32 issue rate (148 SMs x 128
+    lanes x the SM clock) / 3d."""
+    g = synth.rng(900)
+    w = torch.from_numpy(synth.weights(rows, cols, g).view(np.int16)).to(dev)
+    sample, init = synth.fit_draw(rows * cols // d, n_sample, K, g)
+    st, it = torch.from_numpy(sample).to(dev), torch.from_numpy(init).to(dev)
+    _, _, _, ws = vq.fit(w, d, K, st, it, iters)
+    fn = lambda i: vq.fit(w, d, K, st, it, iters, workspace=ws)
+    for i in range(warmup):
+        fn(i)
+    ms = _time_steps(torch, fn, steps) / steps
+    n_sub = rows * cols // d
+    evals = float(n_sample * iters + n_sub) * K
+    clocks = 1965e6
+    peak = 148 * 128 * clocks / (3 * d)
+    ach = evals / (ms * 1e-3)
+    return {"workload": f"vq_fit d{d}K{K} {rows}x{cols} (one expert tensor), {n_sample} sample points, {iters} Lloyd steps",
+            "value": ms, "unit": "ms", "subvectors_per_s": n_sub / (ms * 1e-3),
+            "roofline": {"bound": "alu", "achieved": ach, "peak": peak, "unit": "distance evaluations/s",
+                         "frac": ach / peak, "peak_source": "148 SMs x 128 fp32 lanes x 1965 MHz / (3 d)"},
+            "launches_per_step": 4 + 2 * iters}
 
 
 def cpu_baseline(mds, draws, spec, T, per_expert, cb_bytes, budget_s=10.0):

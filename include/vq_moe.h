@@ -47,7 +47,8 @@ typedef enum vq_status {
     VQ_ERR_UNSUPPORTED = 3,   /* geometry (d, bits) or size the kernels do not implement */
     VQ_ERR_WORKSPACE = 4,     /* workspace NULL, misaligned or smaller than required */
     VQ_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
-    VQ_ERR_DEVICE_CHECK = 6   /* a kernel gave up a bounded wait (see vq_moe_check) */
+    VQ_ERR_DEVICE_CHECK = 6   /* a kernel recorded an error: it gave up a bounded wait, or
+                                 vq_fit met an index out of range (see vq_moe_check) */
 } vq_status;
 
 /* Output element types. */
@@ -215,11 +216,47 @@ vq_status vq_moe_prefill_chunked(const vq_moe_layer *L, const uint16_t *x, int32
                                  int32_t top_k, int32_t renorm, int32_t chunk, void *y, int32_t y_dtype,
                                  void *workspace, size_t ws_bytes, void *stream);
 
+/* ---- Data-free VQ fit: the step that makes a module's codebook, codes and
+ * scales from a bf16 weight tensor ----
+ * The VQ model cards ("Methodology" of Qwen3.5-397B-A17B-VQ-2.6bpw,
+ * Qwen3.8-Flash-Next-VQ-4.4bpw, GLM-5.1-VQ-2.7bpw) fit each tensor's codebook
+ * in pure weight space: k-means / Lloyd over the weight subvectors of a drawn
+ * subsample, no Hessian, activation statistics or calibration data; an fp16
+ * scale per (row, 64 weights). For one tensor W (bf16, row-major
+ * [rows, cols]; subvector i = row i / (cols/d), weights d*(i % (cols/d)) ..)
+ * vq_fit computes:
+ *   scales   fp16 [rows, cols/64]: the group's largest |w| (the cards give the
+ *            scale's shape only; this is the reading taken),
+ *   v        = w / scale per subvector, fp32 (0 where the scale is 0),
+ *   `iters`  Lloyd steps over the subvectors sample[0..n_sample) from the
+ *            centroids v[init[k]]: each point goes to its nearest centroid
+ *            (fp32 squared distance, components summed in order with no fused
+ *            multiply-add, ties to the lower index); a centroid with points
+ *            becomes their exact mean rounded to fp32, one with none keeps its
+ *            value,
+ *   codebook fp16 [K, d]: the final centroids rounded to fp16,
+ *   codes    uint16 [rows, cols/d]: every subvector's nearest codebook entry.
+ * Pack codes with vq_pack for the expert path. All arrays are device memory;
+ * sample and init hold subvector indices drawn by the caller. Requirements:
+ * d in {1, 2, 4, 8}; cols a multiple of 64; 2 <= K <= 65536 and K*d <= 32768
+ * (the centroids sit in shared memory); K <= n_sample <= 2^22; iters >= 0;
+ * rows*cols/d < 2^31 (VQ_ERR_ARG otherwise); w, scales, codebook and codes
+ * 16-byte aligned (VQ_ERR_ALIGN). An index outside [0, rows*cols/d) is
+ * skipped and sets the workspace's error word (see vq_moe_check). Results are
+ * deterministic: centroid sums are exact integers. Workspace:
+ * vq_fit_workspace_size(K, d) bytes (0 for invalid K or d), 256-byte aligned,
+ * owned by the caller. Asynchronous on `stream`. */
+size_t vq_fit_workspace_size(int32_t K, int32_t d);
+vq_status vq_fit(const uint16_t *w, int32_t rows, int32_t cols, int32_t d, int32_t K, const int32_t *sample,
+                 int32_t n_sample, const int32_t *init, int32_t iters, uint16_t *scales, uint16_t *codebook,
+                 uint16_t *codes, void *workspace, size_t ws_bytes, void *stream);
+
 /* Diagnostic (synchronises `stream`). Every wait of the library's pipelined
  * kernels on an on-chip barrier is bounded; a kernel that gives up records a
  * nonzero word at offset 0 of the MoE workspace it ran with (the routing
  * kernel of each vq_moe_decode / vq_moe_prefill call clears it) and stops
- * without completing its outputs. Returns VQ_ERR_DEVICE_CHECK when the word
+ * without completing its outputs. vq_fit records the same word in its own
+ * workspace for a sample or init index out of range (each call clears it). Returns VQ_ERR_DEVICE_CHECK when the word
  * of `workspace` is set after the work queued on `stream`, VQ_OK when not,
  * VQ_ERR_WORKSPACE for a NULL or misaligned workspace. */
 vq_status vq_moe_check(const void *workspace, void *stream);

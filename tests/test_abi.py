@@ -114,3 +114,35 @@ def test_prefill_chunked_validates_before_launch():
     assert f(ctypes.byref(L), 4096, 4, 8192, 1, 1, 0, 16384, 0, 65536, 1 << 20, None) == 1
     assert f(ctypes.byref(L), 4096, 4, 8192, 1, 1, -3, 16384, 0, 65536, 1 << 20, None) == 1
     assert f(ctypes.byref(L), None, 0, None, 1, 1, 5, None, 0, 65536, 1 << 20, None) == 0
+
+
+def test_fit_argument_errors_before_launch():
+    # fake (never dereferenced) pointers: every check fails before any CUDA call
+    f = vq._L().vq_fit
+    ok = dict(w=4096, rows=8, cols=256, d=4, K=8, sample=8192, n=64, init=12288, iters=2, sc=16384, cb=20480,
+              codes=24576, ws=65536, nws=1 << 20)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["w"], a["rows"], a["cols"], a["d"], a["K"], a["sample"], a["n"], a["init"], a["iters"], a["sc"],
+                 a["cb"], a["codes"], a["ws"], a["nws"], None)
+    assert call(d=3) == 1
+    assert call(cols=100) == 1
+    assert call(K=1) == 1                          # VQ_ERR_ARG
+    assert call(K=128) == 1                        # K > n_sample
+    assert call(K=8192, n=1 << 14, d=8) == 1       # K * d beyond the shared-memory table
+    assert call(w=4098) == 2                       # VQ_ERR_ALIGN
+    assert call(ws=65600) == 4                     # VQ_ERR_WORKSPACE (misaligned)
+    assert call(nws=16) == 4                       # too small
+    assert vq._L().vq_fit_workspace_size(8, 3) == 0
+    assert vq._L().vq_fit_workspace_size(512, 4) > 512 * 4 * 12
+
+
+def test_status_constants_match_header():
+    import os
+    import re
+    text = open(os.path.join(os.path.dirname(vq.__file__), "..", "include", "vq_moe.h")).read()
+    enum = dict((n, int(v)) for n, v in re.findall(r"(VQ_(?:OK|ERR_[A-Z_]+)) = (\d+)", text))
+    assert len(enum) == 7
+    for name, value in enum.items():
+        assert getattr(vq, name) == value, name

@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libvqmoe.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "vq_moe.h")
 
 VQ_OK = 0
+VQ_ERR_ARG, VQ_ERR_ALIGN, VQ_ERR_UNSUPPORTED, VQ_ERR_WORKSPACE, VQ_ERR_CUDA, VQ_ERR_DEVICE_CHECK = 1, 2, 3, 4, 5, 6
 VQ_F32, VQ_BF16 = 0, 1
 VQ_MODE_DECODE, VQ_MODE_PREFILL = 0, 1
 
@@ -67,6 +68,8 @@ def _load():
         "vq_set_trace_events": (ctypes.c_int, [P, I32]),
         "vq_moe_check": (ctypes.c_int, [P, P]),
         "vq_moe_decode_noalloc": (ctypes.c_int, [LP, P, I32, P, I32, I32, P, I32, P]),
+        "vq_fit_workspace_size": (SZ, [I32, I32]),
+        "vq_fit": (ctypes.c_int, [P, I32, I32, I32, I32, P, I32, P, I32, P, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -239,6 +242,35 @@ def route(logits, top_k: int, renorm: bool = True, stream=None):
     _check(_L().vq_route(logits.data_ptr(), T, E, top_k, int(bool(renorm)), ids.data_ptr(), w.data_ptr(),
                          offsets.data_ptr(), perm.data_ptr(), _stream(stream)), "vq_route")
     return ids, w, offsets, perm
+
+
+def fit(w, d: int, K: int, sample, init, iters: int, workspace=None, stream=None):
+    """Data-free VQ fit of one bf16 tensor w [rows, cols] (16-bit bit patterns on the device):
+    (scales fp16 bits [rows, cols/64], codebook fp16 bits [K, d], codes uint16 [rows, cols/d] as
+    int16 tensors) from `iters` Lloyd steps over the subvectors `sample` starting at the
+    subvectors `init` (int32 device tensors) (vq_fit)."""
+    torch = _torch()
+    rows, cols = w.shape
+    dev = w.device
+    scales = torch.empty((rows, cols // 64), dtype=torch.int16, device=dev)
+    codebook = torch.empty((K, d), dtype=torch.int16, device=dev)
+    codes = torch.empty((rows, cols // d), dtype=torch.int16, device=dev)
+    n = int(_L().vq_fit_workspace_size(K, d))
+    if n == 0:
+        raise VQError(1, "vq_fit_workspace_size")
+    ws = workspace if workspace is not None else torch.empty(n + 256, dtype=torch.uint8, device=dev)
+    base = ws.data_ptr()
+    aligned = (base + 255) // 256 * 256
+    _check(_L().vq_fit(w.data_ptr(), rows, cols, d, K, sample.data_ptr(), sample.numel(), init.data_ptr(), iters,
+                       scales.data_ptr(), codebook.data_ptr(), codes.data_ptr(), aligned, ws.numel() - (aligned - base),
+                       _stream(stream)), "vq_fit")
+    return scales, codebook, codes, ws
+
+
+def fit_check(workspace, stream=None) -> int:
+    """Status of the error word of a vq_fit workspace returned by fit() (vq_moe_check)."""
+    base = (workspace.data_ptr() + 255) // 256 * 256
+    return int(_L().vq_moe_check(base, _stream(stream)))
 
 
 def set_trace_events(events) -> None:

@@ -502,6 +502,29 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     return cuda_status(err);
 }
 
+size_t vq_fit_workspace_size(int32_t K, int32_t d)
+{
+    if (K < 2 || K > 65536 || (d != 1 && d != 2 && d != 4 && d != 8))
+        return 0;
+    return fit_workspace_size(K, d);
+}
+
+vq_status vq_fit(const uint16_t *w, int32_t rows, int32_t cols, int32_t d, int32_t K, const int32_t *sample,
+                 int32_t n_sample, const int32_t *init, int32_t iters, uint16_t *scales, uint16_t *codebook,
+                 uint16_t *codes, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (!w || !sample || !init || !scales || !codebook || !codes || rows < 1 || cols < 64 || cols % 64 ||
+        (d != 1 && d != 2 && d != 4 && d != 8) || n_sample > (1 << 22) || (long)rows * (cols / d) >= (1L << 31))
+        return VQ_ERR_ARG;
+    if (!aligned(w, 16) || !aligned(scales, 16) || !aligned(codebook, 16) || !aligned(codes, 16) ||
+        !aligned(sample, 4) || !aligned(init, 4))
+        return VQ_ERR_ALIGN;
+    if (!workspace || !aligned(workspace, 256))
+        return VQ_ERR_WORKSPACE;
+    return run_fit(w, rows, cols, d, K, sample, n_sample, init, iters, scales, codebook, codes, workspace, ws_bytes,
+                   (cudaStream_t)stream);
+}
+
 vq_status vq_moe_check(const void *workspace, void *stream)
 {
     if (!workspace || !aligned(workspace, 256))

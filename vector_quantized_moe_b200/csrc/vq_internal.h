@@ -170,4 +170,10 @@ size_t prefill_workspace_size(const vq_moe_layer *L, int T, int k);
 vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const float *logits, int k, int renorm,
                       void *y, int y_dtype, void *ws, size_t ws_bytes, cudaStream_t s);
 
+// Data-free VQ fit (vq_fit.cu).
+size_t fit_workspace_size(int K, int d);
+vq_status run_fit(const uint16_t *w, int rows, int cols, int d, int K, const int32_t *sample, int n_sample,
+                  const int32_t *init, int iters, uint16_t *scales, uint16_t *codebook, uint16_t *codes, void *ws,
+                  size_t ws_bytes, cudaStream_t s);
+
 }  // namespace vq
