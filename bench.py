@@ -229,6 +229,16 @@ def run_ours(args):
             fn(i)
         torch.cuda.synchronize()
         return
+    if args.only == "fit":
+        # profiler runs of the data-free fit of one d4K512 expert tensor: warm-up, then the steps
+        g = synth.rng(900)
+        w = torch.from_numpy(synth.weights(2048, 6144, g).view(np.int16)).to(dev)
+        sample, init = synth.fit_draw(2048 * 6144 // 4, 65536, 512, g)
+        st, itx = torch.from_numpy(sample).to(dev), torch.from_numpy(init).to(dev)
+        for i in range(args.warmup + args.steps):
+            vq.fit(w, 4, 512, st, itx, 10)
+        torch.cuda.synchronize()
+        return
     if args.only in OTHER_DECODE:
         # profiler runs of another decode workload: warm-up, then the steps
         import dataclasses
@@ -643,7 +653,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ncu", action="store_true", help="only warmup + timed steps, for profiler captures")
     ap.add_argument("--small", action="store_true", help="64-expert variant of the workload (profiling)")
-    ap.add_argument("--only", choices=("decode", "prefill", *OTHER_DECODE), default="decode",
+    ap.add_argument("--only", choices=("decode", "prefill", "fit", *OTHER_DECODE), default="decode",
                     help="with --ncu: which path the profiler run exercises")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' lines")
     args = ap.parse_args()
