@@ -92,3 +92,30 @@ def test_fit_index_out_of_range_sets_error_word():
     _, _, _, ws = vq.fit(wt, d, K, torch.from_numpy(sample).cuda(), torch.from_numpy(init).cuda(), 2)
     torch.cuda.synchronize()
     assert vq.fit_check(ws) == vq.VQ_ERR_DEVICE_CHECK
+
+
+def test_fit_duplicate_start_and_empty_centroids():
+    # two identical initial centroids: in the first step the second loses every tie, gets no
+    # point and keeps its value (later steps move the first, and the second may then win points)
+    rows, cols, d, K = 32, 512, 4, 16
+    g = synth.rng(704)
+    w = synth.weights(rows, cols, g)
+    sample, init = synth.fit_draw(rows * cols // d, 1024, K, g)
+    init[3] = init[1]
+    for iters in (1, 4):
+        sc, cb, codes = _run(w, d, K, sample, init, iters)
+        osc, ocb, ocodes, hist = ofit.fit(w, d, K, sample, init, iters)
+        assert np.array_equal(cb, ocb) and np.array_equal(codes, ocodes) and np.array_equal(sc, osc)
+        if iters == 1:
+            assert np.array_equal(cb[3], hist[0][3].astype(np.float16).view(np.uint16))
+            assert not np.array_equal(cb[1], cb[3])
+
+
+def test_fit_all_zero_tensor():
+    # every scale 0, every subvector 0: all codes go to entry 0, the codebook stays the start
+    rows, cols, d, K = 8, 256, 2, 8
+    w = np.zeros((rows, cols), dtype=np.uint16)
+    sample = np.arange(0, rows * cols // d, 2, dtype=np.int32)
+    init = sample[:K].copy()
+    sc, cb, codes = _run(w, d, K, sample, init, 3)
+    assert not sc.any() and not cb.any() and not codes.any()
