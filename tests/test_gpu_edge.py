@@ -73,3 +73,36 @@ def test_decode_bitwise_repeatable():
     lg = torch.from_numpy(synth.logits_normal(T, layer.E, g)).cuda()
     ys = [layer.decode(x, lg, k).cpu().numpy() for _ in range(3)]
     assert all(np.array_equal(ys[0], y) for y in ys[1:])
+
+
+def test_decode_step_replays_from_a_cuda_graph():
+    # the decode step allocates nothing and only launches on its stream: it can be captured
+    # once into a CUDA graph and replayed, with outputs bit-identical to eager calls
+    E, k, H, I = 16, 4, 512, 256
+    oms, layer = _layer(E, H, I, seed=31)
+    g = synth.rng(93)
+    xs, lgs = [], []
+    for _ in range(3):
+        x = synth.activations(5, H, g)
+        xs.append(torch.from_numpy(x.view(np.int16)).cuda())
+        lgs.append(torch.from_numpy(synth.logits_normal(5, E, g)).cuda())
+    ws = layer.workspace(5, k, vq.VQ_MODE_DECODE, "cuda")
+    outs = [torch.empty((5, H), dtype=torch.float32, device="cuda") for _ in range(3)]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        layer.decode(xs[0], lgs[0], k, out=outs[0], workspace=ws, stream=s)   # warm-up outside capture
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=s):
+            for i in range(3):
+                layer.decode(xs[i], lgs[i], k, out=outs[i], workspace=ws, stream=s)
+    for o in outs:
+        o.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    for i in range(3):
+        want = layer.decode(xs[i], lgs[i], k)
+        torch.cuda.synchronize()
+        assert torch.equal(outs[i], want)
+    del graph
