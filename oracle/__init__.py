@@ -8,7 +8,7 @@ The arithmetic lives in vq_oracle.c (plain C, double precision); this file
 builds it with gcc and marshals numpy arrays through ctypes. The data-free
 VQ fit (k-means over weight subvectors) is oracle/fit.py, plain numpy. Each function
 says which passage of the VQ model cards it follows; the readings of silent
-points are listed in vq_oracle.c's header and in the design doc.
+points are listed in vq_oracle.c's header and in fit.py's.
 
 Parity status: every function below is pinned by tests/test_oracle.py against
 closed forms, library routines, hand-worked fixtures or brute force, except

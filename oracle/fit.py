@@ -10,7 +10,7 @@ k-means runs on a drawn subsample; each subvector stores the index of one
 entry of a per-tensor fp16 codebook of K entries, and each (row, 64 weights)
 group has an fp16 scale.
 
-Readings of what the cards leave open (each listed in the design doc):
+Readings of what the cards leave open:
   F1 scale: s[r, g] = fp16(max |w| over the group's 64 weights); the
      subvector the codebook sees is v = w / s (fp32), v = 0 where s = 0.
   F2 distance: squared Euclidean in fp32, sum over components in order,

@@ -21,7 +21,7 @@
  *   - Qwen3.8-Flash-Next and gemma-4 cards: MoE experts selected top-k from
  *     router logits (10-of-512, 128 experts top-8).
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent:
  *   R3  bit order: code j of a row occupies bits [j*b, j*b + b) of the row's
  *       bit string; bit i of that string is bit (i % 32) of word i / 32
  *       (least significant bit first). A 32-code block is then exactly b
