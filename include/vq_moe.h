@@ -219,7 +219,7 @@ vq_status vq_moe_prefill_chunked(const vq_moe_layer *L, const uint16_t *x, int32
 /* ---- Data-free VQ fit: the step that makes a module's codebook, codes and
  * scales from a bf16 weight tensor ----
  * The VQ model cards ("Methodology" of Qwen3.5-397B-A17B-VQ-2.6bpw,
- * Qwen3.8-Flash-Next-VQ-4.4bpw, GLM-5.1-VQ-2.7bpw) fit each tensor's codebook
+ * Qwen3.8-Flash-Next-VQ-4.4bpw, GLM-5.3-Flash-VQ-2.7bpw) fit each tensor's codebook
  * in pure weight space: k-means / Lloyd over the weight subvectors of a drawn
  * subsample, no Hessian, activation statistics or calibration data; an fp16
  * scale per (row, 64 weights). For one tensor W (bf16, row-major

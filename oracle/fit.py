@@ -3,7 +3,7 @@ for who may use it). Plain numpy, float32 where the method decides an integer
 (a code), float64 / exact integers elsewhere.
 
 What the VQ model cards state ("Methodology" of Qwen3.5-397B-A17B-VQ-2.6bpw,
-Qwen3.8-Flash-Next-VQ-4.4bpw and GLM-5.1-VQ-2.7bpw): codebooks are fit in pure
+Qwen3.8-Flash-Next-VQ-4.4bpw and GLM-5.3-Flash-VQ-2.7bpw): codebooks are fit in pure
 weight space by k-means / Lloyd over the weight subvectors (d consecutive
 weights of a row), with no Hessian, activation statistics or calibration data;
 k-means runs on a drawn subsample; each subvector stores the index of one

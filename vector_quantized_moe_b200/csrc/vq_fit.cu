@@ -2,7 +2,7 @@
 // scales the expert path consumes, fit in pure weight space by k-means /
 // Lloyd over the weight subvectors of a drawn subsample (VQ model cards,
 // "Methodology": Qwen3.5-397B-A17B-VQ-2.6bpw, Qwen3.8-Flash-Next-VQ-4.4bpw,
-// GLM-5.1-VQ-2.7bpw). The cards give the scale's shape (fp16 per row and 64
+// GLM-5.3-Flash-VQ-2.7bpw). The cards give the scale's shape (fp16 per row and 64
 // weights), not its derivation; here it is the group's largest |w|.
 //
 // Kernels (one launch each, stream-ordered):
