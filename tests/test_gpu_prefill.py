@@ -86,8 +86,10 @@ def test_prefill_chunked_matches_one_call(T, chunk):
     ws = torch.empty(layer.workspace_size(min(T, chunk), k, vq.VQ_MODE_PREFILL) + 256, dtype=torch.uint8,
                      device="cuda")
     yc = layer.prefill_chunked(xt, lt, k, chunk=chunk, workspace=ws)
+    yb = layer.prefill_chunked(xt, lt, k, chunk=chunk, out_dtype=torch.bfloat16, workspace=ws)
     torch.cuda.synchronize()
     assert np.array_equal(yc.cpu().numpy().view(np.uint32), y.cpu().numpy().view(np.uint32))
+    assert np.array_equal(yb.view(torch.int16).cpu().numpy().view(np.uint16), _bf16_of(y))   # bf16 rows offset right
     tok = np.unique(np.array([0, chunk - 1, chunk % T, T // 2, T - 1]) % T)
     assert_close(yc.cpu().numpy()[tok], oracle.moe(*oms, x, lg, k, tokens=tok), what=f"chunked T{T} c{chunk}")
     if T > chunk:
