@@ -736,6 +736,15 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
             break;
         const uint8_t *sb = stages + (size_t)slot * A.stage_bytes;
         const uint8_t *ssc = sb + 2 * ((j * TG::CG) & 7);
+        // dense rows with two groups per half: both groups' fp16 scales of a row in one 4-byte load
+        constexpr bool PAIR_SC = DENSE && TG::HG == 2 && GP == 1;
+        uint32_t sc2[TG_RL];
+        if constexpr (PAIR_SC) {
+            const uint8_t *p = ssc + soff[0] + 2 * half * TG::HG;
+#pragma unroll
+            for (int i = 0; i < TG_RL; ++i)
+                sc2[i] = *reinterpret_cast<const uint32_t *>(p + i * 8 * 16);
+        }
 #pragma unroll
         for (int gh = 0; gh < TG::HG; gh += GP) {
             uint32_t cw[GP][TG_RL][G::LW];
@@ -786,7 +795,11 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                             cw[uu][i][q] = p[q];
                     }
                 }
-                if constexpr (DENSE) {
+                if constexpr (PAIR_SC) {
+#pragma unroll
+                    for (int i = 0; i < TG_RL; ++i)
+                        sv[uu][i] = f16_to_f32((uint16_t)(gh == 0 ? sc2[i] : sc2[i] >> 16));
+                } else if constexpr (DENSE) {
                     const uint8_t *p = ssc + soff[0] + 2 * gq;
 #pragma unroll
                     for (int i = 0; i < TG_RL; ++i)
