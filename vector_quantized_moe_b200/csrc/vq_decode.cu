@@ -736,14 +736,20 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
             break;
         const uint8_t *sb = stages + (size_t)slot * A.stage_bytes;
         const uint8_t *ssc = sb + 2 * ((j * TG::CG) & 7);
-        // dense rows with two groups per half: both groups' fp16 scales of a row in one 4-byte load
-        constexpr bool PAIR_SC = DENSE && TG::HG == 2 && GP == 1;
-        uint32_t sc2[TG_RL];
+        // with 2 or 4 groups per half, the fp16 scales of a row's groups in this half are adjacent:
+        // one 4- or 8-byte load per row and stage (4- or 8-byte aligned: the scale box rows are 16 bytes
+        // and a half starts at byte 2 * HG * half of the stage's groups)
+        constexpr bool PAIR_SC = (TG::HG == 2 || TG::HG == 4) && GP == 1;
+        uint2 sc2[TG_RL];
         if constexpr (PAIR_SC) {
-            const uint8_t *p = ssc + soff[0] + 2 * half * TG::HG;
 #pragma unroll
-            for (int i = 0; i < TG_RL; ++i)
-                sc2[i] = *reinterpret_cast<const uint32_t *>(p + i * 8 * 16);
+            for (int i = 0; i < TG_RL; ++i) {
+                const uint8_t *p = ssc + (DENSE ? soff[0] + i * 8 * 16 : soff[i]) + 2 * half * TG::HG;
+                if constexpr (TG::HG == 2)
+                    sc2[i] = make_uint2(*reinterpret_cast<const uint32_t *>(p), 0u);
+                else
+                    sc2[i] = *reinterpret_cast<const uint2 *>(p);
+            }
         }
 #pragma unroll
         for (int gh = 0; gh < TG::HG; gh += GP) {
@@ -797,8 +803,10 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                 }
                 if constexpr (PAIR_SC) {
 #pragma unroll
-                    for (int i = 0; i < TG_RL; ++i)
-                        sv[uu][i] = f16_to_f32((uint16_t)(gh == 0 ? sc2[i] : sc2[i] >> 16));
+                    for (int i = 0; i < TG_RL; ++i) {
+                        const uint32_t wv = gh < 2 ? sc2[i].x : sc2[i].y;
+                        sv[uu][i] = f16_to_f32((uint16_t)((gh & 1) ? wv >> 16 : wv));
+                    }
                 } else if constexpr (DENSE) {
                     const uint8_t *p = ssc + soff[0] + 2 * gq;
 #pragma unroll
