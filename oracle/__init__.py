@@ -47,7 +47,7 @@ class _Module(ctypes.Structure):
     _fields_ = [("E", ctypes.c_int32), ("rows", ctypes.c_int32), ("cols", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("bits", ctypes.c_int32),
                 ("words", ctypes.c_void_p), ("scales", ctypes.c_void_p),
-                ("codebook", ctypes.c_void_p), ("bitmap", ctypes.c_void_p)]
+                ("codebook", ctypes.c_void_p), ("bitmap", ctypes.c_void_p), ("biases", ctypes.c_void_p)]
 
 
 _lib = None
@@ -171,6 +171,7 @@ class Module:
     scales: fp16 bits [n_live, cols // 64]
     codebook: fp16 bits [2**bits, d]
     bitmap: uint32 [E, ceil(rows / 32)] or None (all rows live)
+    biases: fp16 bits [n_live, cols // 64] or None: an affine offset per group (w = s * C[q] + b)
     """
     E: int
     rows: int
@@ -181,12 +182,14 @@ class Module:
     scales: np.ndarray
     codebook: np.ndarray
     bitmap: Optional[np.ndarray] = None
+    biases: Optional[np.ndarray] = None
 
     def _struct(self):
         self._keep = (_c(self.words, np.uint32), _c(self.scales, np.uint16), _c(self.codebook, np.uint16),
-                      None if self.bitmap is None else _c(self.bitmap, np.uint32))
-        w, s, cb, bm = self._keep
-        return _Module(self.E, self.rows, self.cols, self.d, self.bits, _p(w), _p(s), _p(cb), _p(bm))
+                      None if self.bitmap is None else _c(self.bitmap, np.uint32),
+                      None if self.biases is None else _c(self.biases, np.uint16))
+        w, s, cb, bm, b = self._keep
+        return _Module(self.E, self.rows, self.cols, self.d, self.bits, _p(w), _p(s), _p(cb), _p(bm), _p(b))
 
 
 def dequant(m: Module, e: int) -> np.ndarray:

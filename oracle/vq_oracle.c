@@ -207,6 +207,7 @@ typedef struct {
     const uint16_t *scales;    /* fp16 [live rows, cols/64] */
     const uint16_t *codebook;  /* fp16 [2^bits, d] */
     const uint32_t *bitmap;    /* [E, ceil(rows/32)], bit set = live; NULL = all live */
+    const uint16_t *biases;    /* fp16 [live rows, cols/64]: an affine offset per group; NULL = none */
 } vqo_module;
 
 /* Packed-row index of every row of expert e (-1 for dead rows). */
@@ -220,8 +221,11 @@ static void live_rows(const vqo_module *m, int e, long *idx)
         idx[r] = is_live(m->bitmap, m->rows, e, r) ? base++ : -1;
 }
 
-/* Dequantise expert e of a module: W[r, c] = C[code(r, c/d)][c % d] * s[r, c/64];
- * dead rows are all zero. W is [rows, cols] row-major. */
+/* Dequantise expert e of a module: W[r, c] = C[code(r, c/d)][c % d] * s[r, c/64]
+ * (+ b[r, c/64] for a module with biases: the affine form s * q + b of the
+ * "affine 3-bit, group 64" modules, Qwen3.5-397B-A17B-VQ-2.4bpw "2026-09-20
+ * correction", with the identity codebook C[q] = q); dead rows are all zero.
+ * W is [rows, cols] row-major. */
 void vqo_dequant(const vqo_module *m, int e, double *W)
 {
     int ncode = m->cols / m->d;
@@ -242,7 +246,8 @@ void vqo_dequant(const vqo_module *m, int e, double *W)
         for (int c = 0; c < m->cols; ++c) {
             double centroid = vqo_f16_to_f64(m->codebook[(size_t)codes[c / m->d] * m->d + c % m->d]);
             double scale = vqo_f16_to_f64(m->scales[(size_t)idx[r] * ngroup + c / 64]);
-            w[c] = centroid * scale;
+            double bias = m->biases ? vqo_f16_to_f64(m->biases[(size_t)idx[r] * ngroup + c / 64]) : 0.0;
+            w[c] = centroid * scale + bias;
         }
         free(codes);
     }

@@ -165,6 +165,78 @@ def test_dequant_d1_affine(oracle_lib):
     assert np.array_equal(W, affine)
 
 
+def _golden_affine_cases():
+    rows = []
+    with open(os.path.join(os.path.dirname(__file__), "golden", "affine_3bit_group64.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            sc, b, ws = (x.strip() for x in line.split("|"))
+            rows.append((float(sc), float(b), [float(v) for v in ws.split()]))
+    return rows
+
+
+def test_dequant_affine_biases_golden(oracle_lib):
+    # one row per fixture line: its 64 weights cycle q = 0..7 in group 0 (scale and bias of the line);
+    # a second group of each row checks that the bias is taken per group
+    cases = _golden_affine_cases()
+    assert len(cases) == 4
+    rows, cols, bits = len(cases), 128, 3
+    q = np.tile(np.arange(8, dtype=np.uint16), cols // 8)[None, None, :].repeat(rows, axis=1)
+    cb = synth.f16_bits(np.arange(8, dtype=np.float32)).reshape(8, 1)           # identity codebook
+    sc = synth.f16_bits(np.array([[c[0], 1.0] for c in cases], dtype=np.float32))
+    bi = synth.f16_bits(np.array([[c[1], 0.0] for c in cases], dtype=np.float32))
+    m = _module(oracle_lib, q, bits, 1, cb, sc[None])
+    m.biases = bi
+    W = oracle_lib.dequant(m, 0)
+    for r, (_, _, want) in enumerate(cases):
+        assert list(W[r, :8]) == want and list(W[r, 56:64]) == want
+        assert list(W[r, 64:72]) == [float(v) for v in range(8)]                # group 1: s = 1, b = 0
+
+
+def test_dequant_affine_biases_equal_zero_point_form(oracle_lib):
+    # with b = -s * z (exact in fp16) the biased identity codebook equals the zero-point codebook
+    # c_q = q - z without biases, the form pinned by test_dequant_d1_affine
+    g = synth.rng(24)
+    rows, cols, bits, z = 5, 192, 3, 3
+    q = synth.raw_codes((1, rows, cols), bits, g)
+    s_bits = synth.f16_bits(2.0 ** g.integers(-6, 2, size=(rows, cols // 64)).astype(np.float32))
+    s = s_bits.view(np.float16).astype(np.float32)
+    ident = synth.f16_bits(np.arange(8, dtype=np.float32)).reshape(8, 1)
+    zp = synth.f16_bits(np.arange(8, dtype=np.float32) - z).reshape(8, 1)
+    m_b = _module(oracle_lib, q, bits, 1, ident, s_bits[None])
+    m_b.biases = synth.f16_bits(-s * z)
+    m_z = _module(oracle_lib, q, bits, 1, zp, s_bits[None])
+    assert np.array_equal(oracle_lib.dequant(m_b, 0), oracle_lib.dequant(m_z, 0))
+
+
+def test_affine_biases_dead_rows_and_gemv_linearity(oracle_lib):
+    # dead rows stay exactly zero with biases; the GEMV of a biased module is the unbiased GEMV
+    # plus b times each group's activation sum (linearity of the dot product)
+    g = synth.rng(25)
+    E, rows, cols, bits = 2, 40, 192, 3
+    q = synth.raw_codes((E, rows, cols), bits, g)
+    bm = synth.live_bitmap(E, rows, 6, g)
+    cb = synth.f16_bits(np.arange(8, dtype=np.float32)).reshape(8, 1)
+    sc = synth.scales(E * rows, cols // 64, g).reshape(E, rows, cols // 64)
+    m0 = _module(oracle_lib, q, bits, 1, cb, sc, bm)
+    m1 = _module(oracle_lib, q, bits, 1, cb, sc, bm)
+    b = synth.f16_bits(g.normal(0, 0.5, size=(len(m1.scales), cols // 64)))
+    m1.biases = b
+    W1 = oracle_lib.dequant(m1, 1)
+    dead = [r for r in range(rows) if not (bm[1, r // 32] >> (r % 32)) & 1]
+    assert dead and all(np.all(W1[r] == 0) for r in dead)
+    x = synth.activations(3, cols, g)
+    y0, y1 = oracle_lib.gemv(m0, 1, x), oracle_lib.gemv(m1, 1, x)
+    xs = oracle_lib.bf16_to_f64(x).reshape(3, cols // 64, 64).sum(axis=2)          # [T, groups]
+    live = [r for r in range(rows) if r not in dead]
+    bl = b.view(np.float16).astype(np.float64)[sum(1 for rr in range(rows)
+                                                     if (bm[0, rr // 32] >> (rr % 32)) & 1):]
+    for i, r in enumerate(live):
+        assert np.allclose(y1[:, r], y0[:, r] + xs @ bl[i], rtol=0, atol=1e-12)
+
+
 def test_dequant_column_mapping(oracle_lib):
     # closed form: codebook entry k = (k, -k, 2k, -2k) (exact in fp16),
     # scales 2^(group index) per row r times (r + 1): W[r, c] is fixed by
