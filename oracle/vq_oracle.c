@@ -246,8 +246,9 @@ void vqo_dequant(const vqo_module *m, int e, double *W)
         for (int c = 0; c < m->cols; ++c) {
             double centroid = vqo_f16_to_f64(m->codebook[(size_t)codes[c / m->d] * m->d + c % m->d]);
             double scale = vqo_f16_to_f64(m->scales[(size_t)idx[r] * ngroup + c / 64]);
-            double bias = m->biases ? vqo_f16_to_f64(m->biases[(size_t)idx[r] * ngroup + c / 64]) : 0.0;
-            w[c] = centroid * scale + bias;
+            /* without biases the product alone (adding +0.0 would turn a -0.0 product into +0.0) */
+            w[c] = m->biases ? centroid * scale + vqo_f16_to_f64(m->biases[(size_t)idx[r] * ngroup + c / 64])
+                             : centroid * scale;
         }
         free(codes);
     }
