@@ -202,8 +202,9 @@ vq_status vq_moe_prefill(const vq_moe_layer *L, const uint16_t *x, int32_t T, co
                          size_t ws_bytes, void *stream);
 
 /* Prefill of a long prompt in chunks, so that scratch memory is bounded by
- * the chunk rather than the prompt (the gemma-4 and Qwen3.5 VQ model cards
- * run prefill in 2048-token chunks). Tokens [c0, c0 + chunk) of x and logits
+ * the chunk rather than the prompt (the Qwen3.8-Flash-Next-VQ-4.4bpw card
+ * chunks its speculative prefill in 2048 tokens, and the GLM-5.3-Flash-VQ-2.7bpw
+ * card tells serving loops to chunk the prefill at 2048). Tokens [c0, c0 + chunk) of x and logits
  * go through vq_moe_prefill into rows [c0, c0 + chunk) of y, one chunk after
  * another on `stream`; the last chunk takes the remaining tokens. Each
  * token's output depends only on its own x row and logits, so the result is
