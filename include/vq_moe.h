@@ -149,13 +149,44 @@ vq_status vq_dequant(const vq_module *m, int32_t expert, float *w_out, void *str
 /* y[t, r] = sum_c W_expert[r, c] * x[t, c] for t < T, accumulated in fp32.
  * x: device bf16 [T, cols], 16-byte aligned. y: device [T, rows] of y_dtype
  * (VQ_F32 or VQ_BF16, round to nearest even). Dead rows give +0.
- * The contraction runs on tensor cores with the codebook entries and the
- * activations in fp16 (bf16 -> fp16 is exact for |x| in [2^-14, 65504]) and
- * the group scale applied in fp32 to each 64-column partial sum. */
+ * The contraction runs on tensor cores (the decode GEMV) with the codebook
+ * entries and the activations in fp16. Every 64-column group of a token's
+ * activations is multiplied by a power of two 2^k that puts its largest |x|
+ * in [2^14, 2^15) before the fp16 rounding, so any finite bf16 input keeps
+ * fp16's full precision (down to 2^-28 of the group's largest value) and
+ * nothing overflows; the group's fp32 partial sum is multiplied by its fp32
+ * scale and by 2^-k (exact). Results are accurate wherever y is a normal fp32
+ * number. */
 vq_status vq_gemv(const vq_module *m, int32_t expert, const uint16_t *x, int32_t T, void *y,
                   int32_t y_dtype, void *stream);
 
-/* Top-k routing and expert bucketing of T tokens.
+/* Bytes of workspace vq_gemm needs for T tokens of module m's shape; 0 on
+ * invalid arguments. */
+size_t vq_gemm_workspace_size(const vq_module *m, int32_t T);
+
+/* The prefill path's tcgen05 GEMM for one expert (a dense building block with
+ * the same arithmetic as vq_moe_prefill's expert GEMMs): for t < T,
+ *   y0[t, r] = sum_c W0_expert[r, c] * x[t, c]     (module m0)
+ *   y1[t, r] = sum_c W1_expert[r, c] * x[t, c]     (module m1, when not NULL)
+ * m1, when given, must have m0's E, rows, cols, d and bits: the two share
+ * each weight-tile pass, as a layer's gate and up projections do. The weight
+ * tiles are decoded on chip to fp16 (fp16(centroid) x fp16(group scale),
+ * rounded to nearest even) and contracted with the tokens' activations in
+ * fp16 on the tensor cores, accumulated in fp32. Each token's activations are
+ * multiplied by 2^k (largest |x| in [2^14, 2^15)) before their fp16 rounding
+ * and the fp32 result by 2^-k. x: device bf16 [T, cols], 16-byte aligned.
+ * y0, y1: device fp32 [T, rows], 16-byte aligned. workspace: device,
+ * 256-byte aligned, vq_gemm_workspace_size(m0, T) bytes (its first word is the
+ * error word that vq_moe_check reads). Requirements as vq_moe_prefill's for
+ * each module (VQ_ERR_UNSUPPORTED otherwise). Errors: VQ_ERR_ARG (bad sizes,
+ * expert out of range, m1 of another shape), VQ_ERR_ALIGN, VQ_ERR_WORKSPACE. */
+vq_status vq_gemm(const vq_module *m0, const vq_module *m1, int32_t expert, const uint16_t *x, int32_t T,
+                  float *y0, float *y1, void *workspace, size_t ws_bytes, void *stream);
+
+/* Top-k routing and expert bucketing of T tokens: the MoE router of the VQ
+ * model cards' layers (Qwen3.8-Flash-Next-VQ-4.4bpw card: 10 of 512 experts
+ * per token; gemma-4-26b-a4b-it-VQ-6.2bpw card: 128 experts, top 8). The
+ * cards print no tie or normalisation rule; the readings taken here follow.
  * logits: device fp32 [T, E]. Per token the top_k experts are taken in order
  * of larger logit first, ties to the smaller expert index, NaN last.
  * weights: renorm != 0 -> softmax over the selected logits; renorm == 0 ->
@@ -179,6 +210,13 @@ size_t vq_moe_workspace_size(const vq_moe_layer *L, int32_t T, int32_t top_k, in
  * launches nothing and returns VQ_OK; x, logits and y may then be NULL:
  *   y[t] = sum_j w[t, j] * W_down,e_j ( silu(W_gate,e_j x[t]) * (W_up,e_j x[t]) )
  * with (e_j, w[t, j]) from vq_route on `logits` (device fp32 [T, E]).
+ * Range: the tensor cores take 16-bit fp16 operands, so each token's
+ * activation row, and each (token, expert) row of the SwiGLU output h, is
+ * multiplied by a power of two that puts its largest magnitude in
+ * [2^14, 2^15) before its fp16 rounding; the fp32 results are multiplied back
+ * exactly. Any finite bf16 input is therefore taken at fp16's full precision
+ * (down to 2^-28 of its row's largest value) without overflow; g, u, h and y
+ * are fp32, and results are accurate wherever those are normal fp32 numbers.
  * x: device bf16 [T, hidden], 16-byte aligned. y: device [T, hidden] of
  * y_dtype, 16-byte aligned. workspace: device, 256-byte aligned, at least
  * vq_moe_workspace_size(L, T, top_k, VQ_MODE_DECODE) bytes; it holds the
@@ -191,7 +229,8 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
 
 /* The same layer for prefill-sized batches (many tokens per expert): per
  * expert bucket a grouped GEMM on the tcgen05 tensor cores with the weight
- * tiles decoded on chip. Same arguments and result definition as
+ * tiles decoded on chip to fp16 (fp16(centroid) x fp16(group scale), rounded
+ * to nearest even). Same arguments, result definition and range handling as
  * vq_moe_decode; workspace sized with VQ_MODE_PREFILL. Additionally requires,
  * for every module, a packed row that is a multiple of 16 bytes
  * ((cols / d / 32) * bits divisible by 4) and cols a multiple of 64 * CH,
@@ -275,7 +314,9 @@ vq_status vq_moe_check(const void *workspace, void *stream);
  * VQ_ERR_WORKSPACE and launch nothing.
  * Set-up: the first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.
+ * before any stream capture. The address is kept per device and looked up
+ * again when the calling thread's context is not the one it was found in
+ * (for instance after cudaDeviceReset).
  * Sharing: all calls on a device use the same array and it keeps the last
  * call's contents (no call needs it zeroed: each writes what it reads).
  * Calls that overlap on the GPU (other streams, other host threads) race on
@@ -283,13 +324,24 @@ vq_status vq_moe_check(const void *workspace, void *stream);
 vq_status vq_moe_decode_noalloc(const vq_moe_layer *L, const uint16_t *x, int32_t T, const float *logits,
                                 int32_t top_k, int32_t renorm, void *y, int32_t y_dtype, void *stream);
 
+/* Bound on the polls of every barrier wait in the pipelined kernels that the
+ * calling thread launches from now on (no counterpart on the pages; a
+ * failure-detection hook). polls < 0 restores the default, 2^22 polls (each
+ * may suspend the waiting thread briefly); 0 makes every wait give up at
+ * once. A wait that gives up makes its CTA stop: it lets
+ * the copies and tensor-core operations it issued complete, frees its tensor
+ * memory, records a nonzero word in the workspace (see vq_moe_check) and
+ * returns without completing its outputs. Nothing faults or hangs. Errors:
+ * VQ_ERR_ARG when polls > 2^32 - 1. */
+vq_status vq_set_wait_limit(int64_t polls);
+
 /* Tracing (no counterpart on the pages; an observability hook for timing
  * each kernel stage with the caller's CUDA events). events: host array of
  * n_events cudaEvent_t handles (as void*) created by the caller, or NULL to
  * switch tracing off. While set, the calling thread's vq_moe_decode and
  * vq_moe_prefill record events[i] on their stream at stage boundary i:
  *   decode:  0 | route | 1 | gate/up GEMV | 2 | SwiGLU | 3 | down GEMV | 4 | combine | 5
- *   prefill: 0 | route | 1 | gather | 2 | gate/up GEMM | 3 | down GEMM | 4 | combine | 5
+ *   prefill: 0 | route | 1 | gather | 2 | gate/up GEMM | 3 | h scales + down GEMM | 4 | combine | 5
  * Boundaries beyond n_events are not recorded. The library does not own
  * the events. Errors: VQ_ERR_ARG when n_events < 0. */
 vq_status vq_set_trace_events(void *const *events, int32_t n_events);

@@ -24,7 +24,7 @@ import numpy as np
 
 __all__ = [
     "rng", "bf16_bits", "f16_bits", "codebook", "scales", "raw_codes",
-    "live_bitmap", "random_words", "activations", "logits_normal", "logits_zipf",
+    "live_bitmap", "random_words", "activations", "activations_scaled", "logits_normal", "logits_zipf",
     "weights", "fit_draw",
 ]
 
@@ -96,6 +96,22 @@ def random_words(n_rows: int, words_per_row: int, g: np.random.Generator) -> np.
 def activations(T: int, H: int, g: np.random.Generator) -> np.ndarray:
     """bf16 activations [T, H] drawn N(0, 1)."""
     return bf16_bits(g.standard_normal((T, H), dtype=np.float32))
+
+
+def activations_scaled(T: int, H: int, g: np.random.Generator, log2_token=None, log2_group=None,
+                       outliers=()) -> np.ndarray:
+    """bf16 activations [T, H] over bf16's range (the bf16 I/O of the cards'
+    runtime): N(0, 1) times 2**log2_token[t] times 2**log2_group[t, c // 64]
+    (integer exponents; each factor is exact), then each (t, c, value) of
+    `outliers` written over its element, all rounded to bf16."""
+    x = g.standard_normal((T, H)).astype(np.float32).astype(np.float64)
+    if log2_token is not None:
+        x = x * np.exp2(np.asarray(log2_token, dtype=np.float64))[:, None]
+    if log2_group is not None:
+        x = x * np.repeat(np.exp2(np.asarray(log2_group, dtype=np.float64)), 64, axis=1)
+    for t, c, v in outliers:
+        x[t, c] = v
+    return bf16_bits(x.astype(np.float32))
 
 
 def logits_normal(T: int, E: int, g: np.random.Generator) -> np.ndarray:

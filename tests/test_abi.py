@@ -146,3 +146,25 @@ def test_status_constants_match_header():
     assert len(enum) == 7
     for name, value in enum.items():
         assert getattr(vq, name) == value, name
+
+
+def test_wait_limit_argument_checked():
+    with pytest.raises(vq.VQError):
+        vq.set_wait_limit(1 << 33)
+    vq.set_wait_limit(0)
+    vq.set_wait_limit(None)
+
+
+def test_gemm_argument_errors_before_launch():
+    # fake (never dereferenced) pointers: validation fails before any CUDA call
+    f = vq._L().vq_gemm
+    m = _null_module()
+    other = _null_module(rows=128)
+    assert f(ctypes.byref(m), None, 2, 4096, 4, 8192, None, 65536, 1 << 20, None) == 1      # expert out of range
+    assert f(ctypes.byref(m), ctypes.byref(other), 0, 4096, 4, 8192, 16384, 65536, 1 << 20, None) == 1   # shapes
+    assert f(ctypes.byref(m), ctypes.byref(m), 0, 4096, 4, 8192, None, 65536, 1 << 20, None) == 1   # y1 missing
+    assert f(ctypes.byref(m), None, 0, 4098, 4, 8192, None, 65536, 1 << 20, None) == 2      # misaligned x
+    assert f(ctypes.byref(m), None, 0, 4096, 4, 8192, None, 65600, 1 << 20, None) == 4      # misaligned workspace
+    assert vq._L().vq_gemm_workspace_size(ctypes.byref(m), 4) > 4 * 128 * 2
+    assert vq._L().vq_gemm_workspace_size(ctypes.byref(_null_module(d=3)), 4) == 0
+

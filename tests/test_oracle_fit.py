@@ -117,3 +117,51 @@ def test_fit_recovers_planted_clusters(d, K):
     cbf = cb.view(np.float16).astype(np.float32)
     assert np.abs(cbf - centres).max() < 3e-3          # means of centre + noise, in fp16
     assert np.array_equal(hist[2], hist[3])            # converged: a further step changes nothing
+
+
+def _f32_of_fraction(fr: Fraction) -> np.float32:
+    """The fp32 number nearest the rational fr (ties to even), by exact integer arithmetic."""
+    if fr == 0:
+        return np.float32(0.0)
+    sign = -1 if fr < 0 else 1
+    a = abs(fr)
+    e = a.numerator.bit_length() - a.denominator.bit_length()   # 2^e <= a < 2^(e+2)
+    if Fraction(2) ** e > a:
+        e -= 1
+    if Fraction(2) ** (e + 1) <= a:
+        e += 1
+    q = max(e, -126) - 23                       # spacing of fp32 numbers near a
+    n = a / (Fraction(2) ** q)
+    fl = n.numerator // n.denominator
+    rem = n - fl
+    r = fl + (1 if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1) else 0)
+    return np.float32(sign * float(Fraction(r) * Fraction(2) ** q))
+
+
+def test_lloyd_update_is_the_exact_mean_on_realistic_points():
+    # the points a real fit sees: bf16 N(0, 0.02) weights over their fp16 group maxima (F1), so full
+    # fp32 significands and magnitudes down to the smallest bf16 weights of a group. Each centroid
+    # the step moves must be the fp32 rounding (to nearest even) of the exact rational mean of its
+    # points as they are, without any fixed-point rounding of the points before the sum.
+    g = synth.rng(505)
+    w = synth.weights(128, 1024, g)
+    sc = fit.fit_scales(w)
+    for d, K in ((4, 64), (2, 32), (8, 16)):
+        v_all = fit.subvectors(w, sc, d)
+        # every subvector with a component that is not a multiple of 2^-40 joins the sample
+        v64 = v_all.astype(np.float64)
+        fine = np.nonzero((np.rint(v64 * 2.0 ** 40) * 2.0 ** -40 != v64).any(axis=1))[0]
+        assert len(fine) > 0
+        sample = np.union1d(g.choice(v_all.shape[0], size=4096, replace=False), fine)
+        v = v_all[sample]
+        c = v[g.choice(len(v), size=K, replace=False)].copy()
+        new, a = fit.lloyd_step(v, c)
+        small = len(fine)
+        for k in range(K):
+            pts = v[a == k]
+            if len(pts) == 0:
+                assert np.array_equal(new[k], c[k])
+                continue
+            for t in range(d):
+                exact = sum(Fraction(float(x)) for x in pts[:, t]) / len(pts)
+                assert new[k, t] == _f32_of_fraction(exact), (d, K, k, t, small)

@@ -60,12 +60,15 @@ def _load():
         "vq_unpack": (ctypes.c_int, [MP, I32, P, P]),
         "vq_dequant": (ctypes.c_int, [MP, I32, P, P]),
         "vq_gemv": (ctypes.c_int, [MP, I32, P, I32, P, I32, P]),
+        "vq_gemm_workspace_size": (SZ, [MP, I32]),
+        "vq_gemm": (ctypes.c_int, [MP, MP, I32, P, I32, P, P, P, SZ, P]),
         "vq_route": (ctypes.c_int, [P, I32, I32, I32, I32, P, P, P, P, P]),
         "vq_moe_workspace_size": (SZ, [LP, I32, I32, I32]),
         "vq_moe_decode": (ctypes.c_int, [LP, P, I32, P, I32, I32, P, I32, P, SZ, P]),
         "vq_moe_prefill": (ctypes.c_int, [LP, P, I32, P, I32, I32, P, I32, P, SZ, P]),
         "vq_moe_prefill_chunked": (ctypes.c_int, [LP, P, I32, P, I32, I32, I32, P, I32, P, SZ, P]),
         "vq_set_trace_events": (ctypes.c_int, [P, I32]),
+        "vq_set_wait_limit": (ctypes.c_int, [I64]),
         "vq_moe_check": (ctypes.c_int, [P, P]),
         "vq_moe_decode_noalloc": (ctypes.c_int, [LP, P, I32, P, I32, I32, P, I32, P]),
         "vq_fit_workspace_size": (SZ, [I32, I32]),
@@ -230,6 +233,26 @@ def gemv(m: Module, expert: int, x, out_dtype=None, out=None, stream=None):
     return out
 
 
+def gemm(m0: Module, expert: int, x, m1: Optional[Module] = None, workspace=None, stream=None):
+    """The prefill path's tcgen05 GEMM for one expert (vq_gemm): y0 [T, rows] = x . W0_expert^T and,
+    with m1, y1 = x . W1_expert^T (fp32). Returns (y0, y1 or None, workspace)."""
+    torch = _torch()
+    T = x.shape[0]
+    y0 = torch.empty((T, m0.rows), dtype=torch.float32, device=x.device)
+    y1 = torch.empty((T, m0.rows), dtype=torch.float32, device=x.device) if m1 is not None else None
+    s0 = m0.struct()
+    s1 = m1.struct() if m1 is not None else None
+    n = int(_L().vq_gemm_workspace_size(ctypes.byref(s0), T))
+    if n == 0:
+        raise VQError(VQ_ERR_ARG, "vq_gemm_workspace_size")
+    ws = workspace if workspace is not None else torch.empty(n + 256, dtype=torch.uint8, device=x.device)
+    base = ws.data_ptr()
+    aligned = (base + 255) // 256 * 256
+    _check(_L().vq_gemm(ctypes.byref(s0), None if s1 is None else ctypes.byref(s1), expert, x.data_ptr(), T,
+                        y0.data_ptr(), _ptr(y1), aligned, ws.numel() - (aligned - base), _stream(stream)), "vq_gemm")
+    return y0, y1, ws
+
+
 def route(logits, top_k: int, renorm: bool = True, stream=None):
     """(ids [T,k] int32, weights [T,k] fp32, offsets [E+1] int32, perm [T*k] int32) (vq_route)."""
     torch = _torch()
@@ -290,6 +313,12 @@ def set_trace_events(events) -> None:
 
 
 _trace_keep = None
+
+
+def set_wait_limit(polls: Optional[int]) -> None:
+    """Bound the barrier waits of the kernels this thread launches (vq_set_wait_limit);
+    None restores the default."""
+    _check(_L().vq_set_wait_limit(-1 if polls is None else int(polls)), "vq_set_wait_limit")
 
 
 class MoELayer:

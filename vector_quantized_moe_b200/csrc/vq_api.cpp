@@ -8,6 +8,9 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "vq_internal.h"
 
@@ -72,7 +75,7 @@ struct DecodePlan {
     GemvPlan pg, pu, pd;         // GEMV plans of gate, up (pg covers both when they share a launch) and down
     bool gu_shared;              // gate and up in one launch
     RoutingLayout r;
-    size_t off_x16, off_G, off_U, off_h, off_D;
+    size_t off_x16, off_xinv, off_G, off_U, off_h, off_wh, off_D;
     size_t total;
 };
 
@@ -119,9 +122,11 @@ DecodePlan plan_decode(const vq_moe_layer *L, int T, int k)
     p.r = plan_routing(o, T, k, p.E);
     const size_t tk = (size_t)T * k;
     p.off_x16 = o; o = align_up(o + (size_t)T * p.H * 2, 256);
+    p.off_xinv = o; o = align_up(o + (size_t)T * 4, 256);
     p.off_G = o; o = align_up(o + (size_t)p.sa * tk * p.I * 4, 256);
     p.off_U = o; o = align_up(o + (size_t)p.sa * tk * p.I * 4, 256);
     p.off_h = o; o = align_up(o + tk * p.I * 2, 256);
+    p.off_wh = o; o = align_up(o + tk * 4, 256);
     p.off_D = o; o = align_up(o + (size_t)p.sb * tk * p.H * 4, 256);
     p.total = o;
     return p;
@@ -154,12 +159,34 @@ ModDev make_moddev(const vq_module &m)
 namespace {
 thread_local cudaEvent_t *g_trace = nullptr;
 thread_local int g_trace_n = 0;
+thread_local uint32_t g_wait_limit = 1u << 22;
+
+std::mutex g_attr_mu;
+std::map<std::pair<const void *, int>, int> g_attr_set;   // (kernel, device) -> shared-memory limit set
 }  // namespace
 
 void trace_point(int i, cudaStream_t s)
 {
     if (g_trace && i < g_trace_n)
         cudaEventRecord(g_trace[i], s);
+}
+
+uint32_t current_wait_limit() { return g_wait_limit; }
+
+cudaError_t set_smem_limit_once(const void *kernel, int bytes)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    std::lock_guard<std::mutex> lock(g_attr_mu);
+    int &cur = g_attr_set[{kernel, dev}];
+    if (cur >= bytes)
+        return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess)
+        cur = bytes;
+    return e;
 }
 
 }  // namespace vq
@@ -190,6 +217,14 @@ vq_status vq_set_trace_events(void *const *events, int32_t n_events)
         return VQ_ERR_ARG;
     g_trace = events ? (cudaEvent_t *)events : nullptr;
     g_trace_n = events ? n_events : 0;
+    return VQ_OK;
+}
+
+vq_status vq_set_wait_limit(int64_t polls)
+{
+    if (polls > 0xFFFFFFFFll)
+        return VQ_ERR_ARG;
+    g_wait_limit = polls < 0 ? (1u << 22) : (uint32_t)polls;
     return VQ_OK;
 }
 
@@ -343,6 +378,31 @@ vq_status vq_gemv(const vq_module *m, int32_t expert, const uint16_t *x, int32_t
     return cuda_status(launch_gemv(a, (cudaStream_t)stream, false));
 }
 
+size_t vq_gemm_workspace_size(const vq_module *m, int32_t T)
+{
+    if (check_module(m) != VQ_OK || T < 0)
+        return 0;
+    return gemm_workspace_size(m, T);
+}
+
+vq_status vq_gemm(const vq_module *m0, const vq_module *m1, int32_t expert, const uint16_t *x, int32_t T, float *y0,
+                  float *y1, void *workspace, size_t ws_bytes, void *stream)
+{
+    vq_status st = check_module(m0);
+    if (st != VQ_OK || (m1 && (st = check_module(m1)) != VQ_OK))
+        return st;
+    if (T < 0 || expert < 0 || expert >= m0->E || (T > 0 && (!x || !y0 || (m1 && !y1))))
+        return VQ_ERR_ARG;
+    if (m1 && (m1->E != m0->E || m1->rows != m0->rows || m1->cols != m0->cols || m1->d != m0->d ||
+               m1->bits != m0->bits))
+        return VQ_ERR_ARG;
+    if (!aligned(x, 16) || !aligned(y0, 16) || !aligned(y1, 16))
+        return VQ_ERR_ALIGN;
+    if (!workspace || !aligned(workspace, 256))
+        return VQ_ERR_WORKSPACE;
+    return run_gemm(m0, m1, expert, x, T, y0, y1, workspace, ws_bytes, (cudaStream_t)stream);
+}
+
 vq_status vq_route(const float *logits, int32_t T, int32_t E, int32_t top_k, int32_t renorm, int32_t *ids,
                    float *weights, int32_t *offsets, int32_t *perm, void *stream)
 {
@@ -350,8 +410,8 @@ vq_status vq_route(const float *logits, int32_t T, int32_t E, int32_t top_k, int
         top_k > std::min(E, 32) || (long)T * top_k >= (1L << 31))
         return VQ_ERR_ARG;
     return cuda_status(launch_route(logits, T, E, top_k, renorm, ids, weights, offsets, perm, nullptr, nullptr,
-                                    nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr, (cudaStream_t)stream,
-                                    false));
+                                    nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 0, nullptr,
+                                    (cudaStream_t)stream, false));
 }
 
 size_t vq_moe_workspace_size(const vq_moe_layer *L, int32_t T, int32_t top_k, int32_t mode)
@@ -408,9 +468,11 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     int32_t *nact = ws_at<int32_t>(workspace, p.r.nact);
     int *errw = ws_at<int>(workspace, p.r.err);
     __half *x16 = ws_at<__half>(workspace, p.off_x16);
+    float *xinv = ws_at<float>(workspace, p.off_xinv);
     float *G = ws_at<float>(workspace, p.off_G);
     float *U = ws_at<float>(workspace, p.off_U);
     __half *h = ws_at<__half>(workspace, p.off_h);
+    float *wh = ws_at<float>(workspace, p.off_wh);
     float *D = ws_at<float>(workspace, p.off_D);
     const long tk = (long)T * top_k;
 
@@ -427,7 +489,7 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
     zs.p[2] = D + tk * p.H;
     zs.n[2] = (long)(p.sb - 1) * tk * p.H;
     cudaError_t err = launch_route(logits, T, p.E, top_k, renorm, ids, w, offsets, perm, pos, active, nact, passes,
-                                   npass, x, x16, p.H, errw, s, true, &zs);
+                                   npass, x, x16, xinv, p.H, errw, s, true, &zs);
     if (err != cudaSuccess)
         return VQ_ERR_CUDA;
     trace_point(1, s);
@@ -475,7 +537,7 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
         return VQ_ERR_CUDA;
 
     trace_point(2, s);
-    err = launch_swiglu(G, U, p.sa, tk * p.I, (int)tk, p.I, h, s, true);
+    err = launch_swiglu(G, U, p.sa, tk * p.I, (int)tk, p.I, perm, top_k, xinv, w, h, wh, s, true);
     if (err != cudaSuccess)
         return VQ_ERR_CUDA;
     trace_point(3, s);
@@ -497,7 +559,7 @@ vq_status vq_moe_decode(const vq_moe_layer *L, const uint16_t *x, int32_t T, con
         return VQ_ERR_CUDA;
 
     trace_point(4, s);
-    err = launch_combine(D, p.sb, tk * p.H, w, pos, T, top_k, p.H, y, y_dtype, s, true);
+    err = launch_combine(D, p.sb, tk * p.H, wh, pos, T, top_k, p.H, y, y_dtype, s, true);
     trace_point(5, s);
     return cuda_status(err);
 }
@@ -559,8 +621,8 @@ vq_status vq_moe_prefill_chunked(const vq_moe_layer *L, const uint16_t *x, int32
         return VQ_ERR_ARG;
     const int H = L->gate.cols, E = L->gate.E;
     const size_t ybytes = y_dtype == VQ_F32 ? 4 : 2;
-    for (int32_t c0 = 0; c0 < T; c0 += chunk) {
-        const int32_t n = std::min(chunk, T - c0);
+    for (int64_t c0 = 0; c0 < T; c0 += chunk) {
+        const int32_t n = (int32_t)std::min<int64_t>(chunk, T - c0);
         st = run_prefill(L, x + (size_t)c0 * H, n, logits + (size_t)c0 * E, top_k, renorm,
                          static_cast<char *>(y) + (size_t)c0 * H * ybytes, y_dtype, workspace, ws_bytes,
                          (cudaStream_t)stream);

@@ -195,6 +195,31 @@ __device__ __forceinline__ void store_out(void *out, int dtype, long idx, float 
         reinterpret_cast<uint16_t *>(out)[idx] = f32_to_bf16_bits(v);
 }
 
+// bf16 activations of one 64-column group, as lane (g, t) holds them: 16
+// values of token g, columns [16t, 16t + 16) (the quad of lanes 4g..4g+3
+// holds the token's group). They are converted to fp16 in place after a
+// multiplication by 2^k, k putting the token's largest |x| in the group in
+// [2^14, 2^15) (scale_exp), so every bf16 value keeps its precision and none
+// overflows. f0 and f1 receive 2^-k of tokens 2t and 2t + 1, the columns of
+// the lane's accumulator fragment, which undo the scale of the group's sums
+// exactly. Every lane of the warp must call this.
+__device__ __forceinline__ void scale_group_bf16(uint32_t (&bw)[8], float &f0, float &f1)
+{
+    uint32_t m = max(bf16x8_max_mag(make_uint4(bw[0], bw[1], bw[2], bw[3])),
+                     bf16x8_max_mag(make_uint4(bw[4], bw[5], bw[6], bw[7])));
+    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+    const int k = scale_exp(m << 16);
+    const float s = pow2f_normal(k);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        bw[i] = bf16x2_to_f16x2_scaled(bw[i], s);
+    const float inv = pow2f(-k);
+    const int t = threadIdx.x & 3;
+    f0 = __shfl_sync(0xFFFFFFFFu, inv, 8 * t);
+    f1 = __shfl_sync(0xFFFFFFFFu, inv, 8 * t + 4);
+}
+
 constexpr int GEMV_THREADS = 256;
 constexpr int GEMV_PD = 3;   // groups of loads in flight per warp
 
@@ -317,11 +342,9 @@ __global__ void __launch_bounds__(GEMV_THREADS, 2) vq_grouped_gemv_kernel(const 
                     av1 = ldg_u128(arow + (long)grp * 64 + 8);
                 }
                 uint32_t bw[8] = {av0.x, av0.y, av0.z, av0.w, av1.x, av1.y, av1.z, av1.w};
-                if (a.act_bf16) {
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        bw[i] = bf16x2_to_f16x2(bw[i]);
-                }
+                float f0 = 1.f, f1 = 1.f;   // inverse activation scales of the fragment's token columns
+                if (a.act_bf16)
+                    scale_group_bf16(bw, f0, f1);
                 float tmp[2][4];
 #pragma unroll
                 for (int i = 0; i < 2; ++i)
@@ -365,10 +388,17 @@ __global__ void __launch_bounds__(GEMV_THREADS, 2) vq_grouped_gemv_kernel(const 
                 for (int rt = 0; rt < 2; ++rt) {
                     const float slo = f16_to_f32(L.sv[2 * rt]);
                     const float shi = f16_to_f32(L.sv[2 * rt + 1]);
-                    acc[rt][0] = fmaf(tmp[rt][0], slo, acc[rt][0]);
-                    acc[rt][1] = fmaf(tmp[rt][1], slo, acc[rt][1]);
-                    acc[rt][2] = fmaf(tmp[rt][2], shi, acc[rt][2]);
-                    acc[rt][3] = fmaf(tmp[rt][3], shi, acc[rt][3]);
+                    if (a.act_bf16) {   // (sum * scale) * 2^-k: the power of two is exact
+                        acc[rt][0] = fmaf(tmp[rt][0] * slo, f0, acc[rt][0]);
+                        acc[rt][1] = fmaf(tmp[rt][1] * slo, f1, acc[rt][1]);
+                        acc[rt][2] = fmaf(tmp[rt][2] * shi, f0, acc[rt][2]);
+                        acc[rt][3] = fmaf(tmp[rt][3] * shi, f1, acc[rt][3]);
+                    } else {
+                        acc[rt][0] = fmaf(tmp[rt][0], slo, acc[rt][0]);
+                        acc[rt][1] = fmaf(tmp[rt][1], slo, acc[rt][1]);
+                        acc[rt][2] = fmaf(tmp[rt][2], shi, acc[rt][2]);
+                        acc[rt][3] = fmaf(tmp[rt][3], shi, acc[rt][3]);
+                    }
                 }
             };
 
@@ -639,7 +669,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                     }
                     tx = stage_bytes_codes + (uint32_t)TG_ROWS * 16 + (uint32_t)it.n * TG::ACOLS * 2;
                 }
-                if (!(ok = mbar_wait(&empty[slot], ph ^ 1, abort_flag, A.err, 11)))
+                if (!(ok = mbar_wait(&empty[slot], ph ^ 1, abort_flag, A.err, 11, a.wait_limit)))
                     break;
                 uint8_t *sb = stages + (size_t)slot * A.stage_bytes;
                 mbar_expect_tx(&full[slot], tx);
@@ -656,11 +686,11 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                     ph ^= 1;
                 }
             }
-            if (!ok) {   // let the copies in flight land before the CTA exits
-                for (uint32_t s = 0; s < (uint32_t)A.ns && s < k; ++s) {
-                    const uint32_t kk = k - 1 - s;
-                    mbar_wait(&full[kk % A.ns], (kk / A.ns) & 1, abort_flag, A.err, 12);
-                }
+            // the copies issued have landed before this thread leaves (the last use of each slot):
+            // after a give-up the consumers may have left without waiting for them
+            for (uint32_t s = 0; s < (uint32_t)A.ns && s < k; ++s) {
+                const uint32_t kk = k - 1 - s;
+                mbar_drain(&full[kk % A.ns], (kk / A.ns) & 1);
             }
         }
         return;
@@ -732,7 +762,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                     acc[i][q] = 0.f;
         }
 
-        if (!(ok = mbar_wait(&full[slot], ph, abort_flag, A.err, 13)))
+        if (!(ok = mbar_wait(&full[slot], ph, abort_flag, A.err, 13, a.wait_limit)))
             break;
         const uint8_t *sb = stages + (size_t)slot * A.stage_bytes;
         const uint8_t *ssc = sb + 2 * ((j * TG::CG) & 7);
@@ -757,6 +787,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
             int co[GP];
             float sv[GP][TG_RL];
             uint32_t bw[GP][8];
+            float fa[GP][2];   // bf16 activations: inverse scales of the fragment's token columns
 #pragma unroll
             for (int uu = 0; uu < GP; ++uu) {
                 const int gq = half * TG::HG + gh + uu;   // group within the stage
@@ -821,11 +852,8 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                 const uint4 v1 = *reinterpret_cast<const uint4 *>(sb + aoff + gq * 128 + 16);
                 bw[uu][0] = v0.x; bw[uu][1] = v0.y; bw[uu][2] = v0.z; bw[uu][3] = v0.w;
                 bw[uu][4] = v1.x; bw[uu][5] = v1.y; bw[uu][6] = v1.z; bw[uu][7] = v1.w;
-                if constexpr (ABF16) {
-#pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        bw[uu][q] = bf16x2_to_f16x2(bw[uu][q]);
-                }
+                if constexpr (ABF16)
+                    scale_group_bf16(bw[uu], fa[uu][0], fa[uu][1]);
             }
             if (gh + GP >= TG::HG) {   // every read of this stage by the warp is done
                 __syncwarp();
@@ -887,10 +915,17 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
 #pragma unroll
                 for (int rt = 0; rt < TG_RT; ++rt) {
                     const float slo = sv[uu][2 * rt], shi = sv[uu][2 * rt + 1];
-                    acc[rt][0] = fmaf(tmp[uu][rt][0], slo, acc[rt][0]);
-                    acc[rt][1] = fmaf(tmp[uu][rt][1], slo, acc[rt][1]);
-                    acc[rt][2] = fmaf(tmp[uu][rt][2], shi, acc[rt][2]);
-                    acc[rt][3] = fmaf(tmp[uu][rt][3], shi, acc[rt][3]);
+                    if constexpr (ABF16) {   // (sum * scale) * 2^-k: the power of two is exact
+                        acc[rt][0] = fmaf(tmp[uu][rt][0] * slo, fa[uu][0], acc[rt][0]);
+                        acc[rt][1] = fmaf(tmp[uu][rt][1] * slo, fa[uu][1], acc[rt][1]);
+                        acc[rt][2] = fmaf(tmp[uu][rt][2] * shi, fa[uu][0], acc[rt][2]);
+                        acc[rt][3] = fmaf(tmp[uu][rt][3] * shi, fa[uu][1], acc[rt][3]);
+                    } else {
+                        acc[rt][0] = fmaf(tmp[uu][rt][0], slo, acc[rt][0]);
+                        acc[rt][1] = fmaf(tmp[uu][rt][1], slo, acc[rt][1]);
+                        acc[rt][2] = fmaf(tmp[uu][rt][2], shi, acc[rt][2]);
+                        acc[rt][3] = fmaf(tmp[uu][rt][3], shi, acc[rt][3]);
+                    }
                 }
         }
         if (++slot == (uint32_t)A.ns) {
@@ -910,7 +945,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
         if (TG_HALVES == 1) {
             // one warp set: the sums are complete
         } else if (half == 1) {
-            if (!(ok = mbar_wait(&xempty[wr * 2 + xb], xph ^ 1, abort_flag, A.err, 14)))
+            if (!(ok = mbar_wait(&xempty[wr * 2 + xb], xph ^ 1, abort_flag, A.err, 14, a.wait_limit)))
                 break;
 #pragma unroll
             for (int v = 0; v < 4 * TG_RT; ++v)
@@ -918,7 +953,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
             mbar_arrive(&xfull[wr * 2 + xb]);
             continue;
         } else {
-            if (!(ok = mbar_wait(&xfull[wr * 2 + xb], xph, abort_flag, A.err, 15)))
+            if (!(ok = mbar_wait(&xfull[wr * 2 + xb], xph, abort_flag, A.err, 15, a.wait_limit)))
                 break;
 #pragma unroll
             for (int v = 0; v < 4 * TG_RT; ++v)
@@ -956,43 +991,99 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
 
 // ------------------------------------------------------------ SwiGLU and combine
 
-// h = fp16(silu(sum_s G[s]) * sum_s U[s]), slices summed in order. S > 0: the
-// slice count is a compile-time constant, so every load is issued before the
-// first add; S == 0: any slice count.
+// SwiGLU of bucket slot q. The GEMVs read the slot's token t = perm[q] / top_k
+// scaled by 2^k_t, so g = xinv[t] * sum_s G[s, q, :] and u = xinv[t] *
+// sum_s U[s, q, :] (xinv[t] = 2^-k_t, exact), with the slices summed in order;
+// h = silu(g) * u in fp32. The down GEMV takes h as an fp16 operand, so the
+// slot's row is stored as hs[q, :] = fp16(h * 2^e_q), e_q putting the slot's
+// largest |h| in [2^14, 2^15) (scale_exp): no overflow for any finite h and
+// fp16's full precision for the values that matter. The inverse scale goes
+// into the routing weight of the slot's pair p = perm[q]: wh[p] = w[p] *
+// 2^-e_q (exact), which the combine applies to the down projection. One block
+// per slot (grid-stride); up to 8 elements per thread stay in registers
+// between the row's maximum and the stores (longer rows are computed again,
+// with the same arithmetic). S > 0: the slice count is a compile-time
+// constant, so every load of an element is issued before the first add;
+// S == 0: any count.
+constexpr int SWIGLU_THREADS = 256;
+constexpr int SWIGLU_KEEP = 8;
+
 template <int S>
-__global__ void vq_swiglu_kernel(const float *__restrict__ G, const float *__restrict__ U, int slices, long slice_stride,
-                                 long n, __half *__restrict__ h)
+__global__ void __launch_bounds__(SWIGLU_THREADS) vq_swiglu_kernel(
+    const float *__restrict__ G, const float *__restrict__ U, int slices, long slice_stride, int slots, int inter,
+    const int32_t *__restrict__ perm, int top_k, const float *__restrict__ xinv, const float *__restrict__ w,
+    __half *__restrict__ h, float *__restrict__ wh)
 {
+    __shared__ uint32_t red[SWIGLU_THREADS / 32];
     grid_dep_launch();   // the next kernel may start its prologue; it waits for this one's results
     grid_dep_wait();
-    for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
-        float gs = 0.f, us = 0.f;
-        if constexpr (S > 0) {
-            float gv[S], uv[S];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int q = blockIdx.x; q < slots; q += gridDim.x) {
+        const int p = perm[q];
+        const float f = xinv[p / top_k];
+        const long row = (long)q * inter;
+        auto h_at = [&](int c) {
+            float gs = 0.f, us = 0.f;
+            if constexpr (S > 0) {
+                float gv[S], uv[S];
 #pragma unroll
-            for (int q = 0; q < S; ++q) {
-                gv[q] = G[q * slice_stride + i];
-                uv[q] = U[q * slice_stride + i];
-            }
+                for (int i = 0; i < S; ++i) {
+                    gv[i] = G[i * slice_stride + row + c];
+                    uv[i] = U[i * slice_stride + row + c];
+                }
 #pragma unroll
-            for (int q = 0; q < S; ++q) {
-                gs += gv[q];
-                us += uv[q];
+                for (int i = 0; i < S; ++i) {
+                    gs += gv[i];
+                    us += uv[i];
+                }
+            } else {
+                for (int i = 0; i < slices; ++i) {
+                    gs += G[i * slice_stride + row + c];
+                    us += U[i * slice_stride + row + c];
+                }
             }
-        } else {
-            for (int q = 0; q < slices; ++q) {
-                gs += G[q * slice_stride + i];
-                us += U[q * slice_stride + i];
-            }
+            const float g = gs * f, u = us * f;
+            return __fdividef(g, 1.f + __expf(-g)) * u;
+        };
+        float hv[SWIGLU_KEEP];
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < SWIGLU_KEEP; ++i) {
+            const int c = threadIdx.x + i * SWIGLU_THREADS;
+            hv[i] = c < inter ? h_at(c) : 0.f;
+            m = max(m, __float_as_uint(hv[i]) & 0x7FFFFFFFu);
         }
-        const float silu = gs / (1.f + __expf(-gs));
-        h[i] = __float2half_rn(silu * us);
+        for (int c = threadIdx.x + SWIGLU_KEEP * SWIGLU_THREADS; c < inter; c += SWIGLU_THREADS)
+            m = max(m, __float_as_uint(h_at(c)) & 0x7FFFFFFFu);
+        m = __reduce_max_sync(0xFFFFFFFFu, m);
+        if (lane == 0)
+            red[warp] = m;
+        __syncthreads();
+        m = red[0];
+#pragma unroll
+        for (int i = 1; i < SWIGLU_THREADS / 32; ++i)
+            m = max(m, red[i]);
+        const int e = scale_exp(m);
+        const float sc = pow2f_normal(e);
+        if (threadIdx.x == 0)
+            wh[p] = w[p] * pow2f(-e);
+#pragma unroll
+        for (int i = 0; i < SWIGLU_KEEP; ++i) {
+            const int c = threadIdx.x + i * SWIGLU_THREADS;
+            if (c < inter)
+                h[row + c] = __float2half_rn(hv[i] * sc);
+        }
+        for (int c = threadIdx.x + SWIGLU_KEEP * SWIGLU_THREADS; c < inter; c += SWIGLU_THREADS)
+            h[row + c] = __float2half_rn(h_at(c) * sc);
+        __syncthreads();   // red is reused by the next slot
     }
 }
 
 // y[t, :] = sum_j w[t, j] * sum_s D[s, pos[t*k + j], :], slots in order j and
-// slices in order s; a block per token (and column range), four columns per
-// thread. The loads of 8 slots x S slices are issued before any is used.
+// slices in order s (w carries the inverse of the power-of-two scale of the
+// pair's down-projection operand); a block per token (and column range), four
+// columns per thread. The loads of 8 slots x S slices are issued before any
+// is used.
 template <int S>
 __global__ void __launch_bounds__(256) vq_combine_kernel(const float *__restrict__ D, int slices, long slice_stride,
                                                          const float *__restrict__ w, const int32_t *__restrict__ pos,
@@ -1135,13 +1226,9 @@ template <int D, int BITS>
 cudaError_t gemv_dispatch(const GemvArgs &a, cudaStream_t s, bool pdl)
 {
     auto k = vq_grouped_gemv_kernel<D, BITS, GEMV_PD>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (err != cudaSuccess)
-            return err;
-        attr_set = true;
-    }
+    cudaError_t err = set_smem_limit_once((const void *)k, 227 * 1024);
+    if (err != cudaSuccess)
+        return err;
     const size_t smem = gemv_smem_bytes(a.mod[0]);
     int occ = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, GEMV_THREADS, smem) != cudaSuccess || occ < 1)
@@ -1225,7 +1312,8 @@ cudaError_t gemv_tma_dispatch(const GemvArgs &a, cudaStream_t s, bool pdl)
         dense = dense && !a.mod[i].bitmap;
     auto k = a.act_bf16 ? (dense ? vq_gemv_tma_kernel<D, BITS, true, true> : vq_gemv_tma_kernel<D, BITS, true, false>)
                         : (dense ? vq_gemv_tma_kernel<D, BITS, false, true> : vq_gemv_tma_kernel<D, BITS, false, false>);
-    cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.total);
+    // the layout of every module of a geometry is the same, so its size is fixed per kernel
+    cudaError_t err = set_smem_limit_once((const void *)k, (int)p.total);
     if (err != cudaSuccess)
         return err;
     const bool both = FastByteCodes<D, BITS>::value;
@@ -1288,8 +1376,10 @@ GemvPlan gemv_plan(const ModDev *mods, int nmod, double n_tiles_expected, int sl
     return p;
 }
 
-cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, bool pdl)
+cudaError_t launch_gemv(const GemvArgs &args, cudaStream_t s, bool pdl)
 {
+    GemvArgs a = args;
+    a.wait_limit = current_wait_limit();
     const ModDev &m = a.mod[0];
     const bool tma = tma_for(a.mod, a.nmod);
 #define VQ_GEMV(D_, B_)                                                        \
@@ -1300,22 +1390,25 @@ cudaError_t launch_gemv(const GemvArgs &a, cudaStream_t s, bool pdl)
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_swiglu(const float *G, const float *U, int slices, long slice_stride, int slots, int inter, __half *h,
+cudaError_t launch_swiglu(const float *G, const float *U, int slices, long slice_stride, int slots, int inter,
+                          const int32_t *perm, int top_k, const float *xinv, const float *w, __half *h, float *wh,
                           cudaStream_t s, bool pdl)
 {
-    const long n = (long)slots * inter;
-    const dim3 grid((unsigned)((n + 255) / 256 < 4096 ? (n > 0 ? (n + 255) / 256 : 1) : 4096));
+    const dim3 grid((unsigned)std::max(1, std::min(slots, 8192)));
+#define VQ_SWIGLU(S_) launch(vq_swiglu_kernel<S_>, grid, dim3(SWIGLU_THREADS), 0, s, pdl, G, U, slices, slice_stride, \
+                             slots, inter, perm, top_k, xinv, w, h, wh)
     switch (slices) {
-    case 1: return launch(vq_swiglu_kernel<1>, grid, dim3(256), 0, s, pdl, G, U, slices, slice_stride, n, h);
-    case 2: return launch(vq_swiglu_kernel<2>, grid, dim3(256), 0, s, pdl, G, U, slices, slice_stride, n, h);
-    case 3: return launch(vq_swiglu_kernel<3>, grid, dim3(256), 0, s, pdl, G, U, slices, slice_stride, n, h);
-    case 4: return launch(vq_swiglu_kernel<4>, grid, dim3(256), 0, s, pdl, G, U, slices, slice_stride, n, h);
-    default: return launch(vq_swiglu_kernel<0>, grid, dim3(256), 0, s, pdl, G, U, slices, slice_stride, n, h);
+    case 1: return VQ_SWIGLU(1);
+    case 2: return VQ_SWIGLU(2);
+    case 3: return VQ_SWIGLU(3);
+    case 4: return VQ_SWIGLU(4);
+    default: return VQ_SWIGLU(0);
     }
+#undef VQ_SWIGLU
 }
 
-cudaError_t launch_combine(const float *D, int slices, long slice_stride, const float *w, const int32_t *pos, int T, int k,
-                           int hidden, void *y, int y_dtype, cudaStream_t s, bool pdl)
+cudaError_t launch_combine(const float *D, int slices, long slice_stride, const float *w, const int32_t *pos, int T,
+                           int k, int hidden, void *y, int y_dtype, cudaStream_t s, bool pdl)
 {
     const int blocks = T < 8192 ? (T > 0 ? T : 1) : 8192;
     // few tokens: spread each token's columns over several blocks

@@ -80,6 +80,60 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float v)
     return *reinterpret_cast<uint16_t *>(&b);
 }
 
+// ---------------------------------------------------------------- power-of-two operand scaling
+//
+// The tensor-core operands are fp16, whose range ([2^-24, 65504]) is far
+// narrower than bf16's. Every 16-bit operand row (a token's activations, a
+// slot's SwiGLU output) is therefore multiplied by 2^k before its fp16
+// rounding, with k chosen so that the row's largest magnitude lands in
+// [2^14, 2^15), and the fp32 results are multiplied by 2^-k. Both steps are
+// exact (a power of two), so the only rounding is the fp16 rounding of the
+// scaled operand, at fp16's full 11-bit precision for every element within
+// 2^-28 of the row's largest.
+
+// 2^e as an fp32 value, for e in [-149, 127] (subnormal below -126).
+__device__ __forceinline__ float pow2f(int e)
+{
+    return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(1u << (e + 149));
+}
+
+// The scale exponent k for a row whose largest magnitude has the fp32 bit
+// pattern `mag` (sign bit clear): 14 - floor(log2 max), capped at 127 so that
+// 2^k and 2^-k are fp32 numbers, read off the exponent field (for a normal
+// max with biased exponent E, floor(log2 max) = E - 127, so k = 141 - E; a
+// zero or subnormal max has E = 0 and takes the cap: any scale leaves such a
+// row's fp16 image within fp16's range). A row holding Inf or NaN (E = 255)
+// gets 0 (no scaling). The result lies in [-113, 127].
+__device__ __forceinline__ int scale_exp(uint32_t mag)
+{
+    const int E = (int)(mag >> 23);
+    return E == 255 ? 0 : min(141 - E, 127);
+}
+
+// 2^e for e in [-126, 127] (a normal fp32 number), e.g. a scale_exp result.
+__device__ __forceinline__ float pow2f_normal(int e)
+{
+    return __uint_as_float((uint32_t)(e + 127) << 23);
+}
+
+// Two bf16 values packed in a word, times 2^k (as the fp32 value s = 2^k),
+// -> fp16x2 (round to nearest even).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t w, float s)
+{
+    const float lo = __uint_as_float(w << 16) * s;
+    const float hi = __uint_as_float(w & 0xFFFF0000u) * s;
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Largest magnitude of the four bf16 pairs of a 16-byte load, as bf16
+// magnitude bits in the low half (NaN patterns compare above Inf).
+__device__ __forceinline__ uint32_t bf16x8_max_mag(uint4 v)
+{
+    uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu), __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+    return max(m & 0xFFFFu, m >> 16);
+}
+
 // ---------------------------------------------------------------- tensor cores
 
 // D = A * B + C for one m16n8k16 tile, fp16 inputs, fp32 accumulate.

@@ -77,6 +77,7 @@ struct GemvArgs {
     int out_dtype;          // VQ_F32 or VQ_BF16
     long out_slice_stride;  // elements between slices
     int *err;               // device error word for bounded waits (may be NULL)
+    uint32_t wait_limit;    // polls of a bounded wait before it gives up (current_wait_limit())
 };
 
 // Launches the TMA-fed kernel when the modules allow it (16-byte packed rows,
@@ -94,8 +95,9 @@ GemvPlan gemv_plan(const ModDev *mods, int nmod, double n_tiles_expected, int sl
 size_t gemv_smem_bytes(const ModDev &m);
 
 // Routing + bucketing. pos = inverse of perm; active/n_active as above (may be NULL).
-// When x is not NULL the same launch also writes x16 = fp16(x) [T, H]; when
-// err is not NULL it is cleared.
+// When x is not NULL the same launch also writes, per token t, x16[t] =
+// fp16(x[t] * 2^k_t) [T, H] and xinv[t] = 2^-k_t (k_t puts the token's largest
+// |x| in [2^14, 2^15)); when err is not NULL it is cleared.
 // Up to three device spans of 32-bit words that a routing launch clears (after
 // its grid-dependency wait): the partial-sum slices beyond the first, which a
 // GEMV launch with slices_zeroed set then leaves to the items that write them.
@@ -107,16 +109,23 @@ struct ZeroSpans {
 // passes / n_passes (may be NULL): the token tiles of the buckets, see VQ_PASS_TOKENS.
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int32_t *ids, float *w,
                          int32_t *offsets, int32_t *perm, int32_t *pos, int32_t *active, int32_t *n_active,
-                         int2 *passes, int32_t *n_passes, const uint16_t *x, __half *x16, int H, int *err,
-                         cudaStream_t s, bool pdl, const ZeroSpans *zero = nullptr);
+                         int2 *passes, int32_t *n_passes, const uint16_t *x, __half *x16, float *xinv, int H,
+                         int *err, cudaStream_t s, bool pdl, const ZeroSpans *zero = nullptr);
 
-// h[q, c] = fp16( silu(sum_s G[s, q, c]) * sum_s U[s, q, c] )
+// x16[t] = fp16(x[t] * 2^k_t), xinv[t] = 2^-k_t for t < T (as the routing launch does).
+cudaError_t launch_convert(const uint16_t *x, __half *x16, float *xinv, int T, int H, cudaStream_t s, bool pdl);
+
+// Per bucket slot q (pair p = perm[q], token t = p / top_k): g = xinv[t] *
+// sum_s G[s, q, :], u = xinv[t] * sum_s U[s, q, :], h = silu(g) * u;
+// h16[q, :] = fp16(h * 2^e_q) and wh[p] = w[p] * 2^-e_q, e_q putting the
+// slot's largest |h| in [2^14, 2^15).
 cudaError_t launch_swiglu(const float *G, const float *U, int slices, long slice_stride, int slots, int inter,
-                          __half *h, cudaStream_t s, bool pdl);
+                          const int32_t *perm, int top_k, const float *xinv, const float *w, __half *h, float *wh,
+                          cudaStream_t s, bool pdl);
 
 // y[t, r] = sum_j w[t*k + j] * sum_s D[s, pos[t*k + j], r]
-cudaError_t launch_combine(const float *D, int slices, long slice_stride, const float *w, const int32_t *pos,
-                           int T, int k, int hidden, void *y, int y_dtype, cudaStream_t s, bool pdl);
+cudaError_t launch_combine(const float *D, int slices, long slice_stride, const float *w, const int32_t *pos, int T,
+                           int k, int hidden, void *y, int y_dtype, cudaStream_t s, bool pdl);
 
 cudaError_t launch_unpack(const ModDev &m, int expert, uint16_t *out, cudaStream_t s);
 cudaError_t launch_dequant(const ModDev &m, int expert, float *out, cudaStream_t s);
@@ -165,10 +174,22 @@ T *ws_at(void *ws, size_t off) { return reinterpret_cast<T *>(reinterpret_cast<c
 // Stage-boundary tracing (vq_set_trace_events): records event i on stream s if set.
 void trace_point(int i, cudaStream_t s);
 
+// Polls of a bounded barrier wait in the kernels launched by this thread
+// (vq_set_wait_limit; 2^22 by default).
+uint32_t current_wait_limit();
+
+// Sets a kernel's dynamic shared-memory limit once per (kernel, device).
+cudaError_t set_smem_limit_once(const void *kernel, int bytes);
+
 // Prefill path (vq_prefill.cu).
 size_t prefill_workspace_size(const vq_moe_layer *L, int T, int k);
 vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const float *logits, int k, int renorm,
                       void *y, int y_dtype, void *ws, size_t ws_bytes, cudaStream_t s);
+
+// One expert's tcgen05 GEMM of one or two modules (vq_prefill.cu).
+size_t gemm_workspace_size(const vq_module *m, int T);
+vq_status run_gemm(const vq_module *m0, const vq_module *m1, int expert, const uint16_t *x, int T, float *y0,
+                   float *y1, void *ws, size_t ws_bytes, cudaStream_t s);
 
 // Data-free VQ fit (vq_fit.cu).
 size_t fit_workspace_size(int K, int d);

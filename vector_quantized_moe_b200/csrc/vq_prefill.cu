@@ -108,9 +108,14 @@ struct PrefillArgs {
     int sa, sc;               // operand stages, code stages
     uint32_t off_a, off_b, off_c, off_cb, off_tiles, off_bar;
     int scale_tma;            // scales staged by TMA with the code chunks (else read per thread)
-    void *out;                // SwiGLU: fp16 [slots, rows]; else fp32 [slots, rows]
+    void *out;                // SwiGLU: fp16 [slots, rows]; else fp32 [slots, rows] (module 0)
+    void *out2;               // not SwiGLU, two modules: module 1's fp32 [slots, rows]
     int swiglu;
+    const float *sxinv;       // per slot, 2^-k of its activation row's scale (NULL: the caller applies it)
+    int8_t *hexp;             // SwiGLU: per (slot, 32-row block), the exponent its fp16 h values carry
+    int nblk32;               // SwiGLU: rows / 32
     int *err;
+    uint32_t wait_limit;      // polls of a bounded wait before it gives up
 };
 
 __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b)
@@ -278,9 +283,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + a.off_bar);
     uint64_t *full_a = bars, *full_b = bars + a.sa, *empty = bars + 2 * a.sa;
     uint64_t *full_c = bars + 3 * a.sa, *empty_c = full_c + a.sc;
-    uint64_t *acc_full = empty_c + a.sc, *acc_empty = acc_full + 1;
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(acc_empty + 1);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    uint64_t *acc_full = empty_c + a.sc, *acc_empty = acc_full + 1, *drain_bar = acc_empty + 1;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(drain_bar + 1);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int nmod = NMOD;
@@ -306,6 +311,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 128 * NWG);
+        mbar_init(drain_bar, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -359,7 +365,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
         if (lane == 0) {
-            uint32_t ks = 0, st = 0, ph = 0, cst = 0, cph = 0;   // operand / code stage counters
+            uint32_t ks = 0, st = 0, ph = 0, cks = 0, cst = 0, cph = 0;   // operand / code stage counters
             bool ok = true;
             for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
                 const Item itm = item_of<BN>(it, MT, tiles, n_act, a.active, a.offsets);
@@ -367,7 +373,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                 for (int m = 0; m < nmod; ++m)
                     prow0[m] = tile_prow0(a.mod[m], itm.e, itm.m0);
                 for (int c = 0; c < nchunks && ok; ++c) {
-                    if (!(ok = mbar_wait(&empty_c[cst], cph ^ 1, abort_flag, a.err, 1)))
+                    if (!(ok = mbar_wait(&empty_c[cst], cph ^ 1, abort_flag, a.err, 1, a.wait_limit)))
                         break;
                     mbar_expect_tx(&full_c[cst], (uint32_t)(nmod * (a.scale_tma ? CODE_STAGE : BM * P::CHW * 4)));
                     for (int m = 0; m < nmod; ++m) {
@@ -377,12 +383,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                             tma_load_2d(stg + BM * P::CHW * 4, &a.tmap_s[m], (c * P::CH) & ~7, prow0[m],
                                         &full_c[cst]);
                     }
+                    ++cks;
                     if (++cst == (uint32_t)a.sc) {
                         cst = 0;
                         cph ^= 1;
                     }
                     for (int j = 0; j < P::CH; ++j) {
-                        if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag, a.err, 2)))
+                        if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag, a.err, 2, a.wait_limit)))
                             break;
                         mbar_expect_tx(&full_b[st], (uint32_t)B_TILE);
                         tma_load_2d(sm_b + (size_t)st * B_TILE, &a.tmap_b, (c * P::CH + j) * 64, itm.q0, &full_b[st]);
@@ -394,31 +401,31 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                     }
                 }
             }
-            if (!ok) {
-                // let the loads already issued land before the CTA leaves
-                for (uint32_t s = 0; s < (uint32_t)a.sa; ++s)
-                    if (ks > s)
-                        mbar_wait(&full_b[(ks - 1 - s) % a.sa], ((ks - 1 - s) / a.sa) & 1, abort_flag, a.err, 3);
-            }
+            // the loads issued have landed before the CTA leaves (the last use of each stage): after
+            // a give-up the other warps may not have waited for them
+            for (uint32_t s = 0; s < (uint32_t)a.sa && s < ks; ++s)
+                mbar_drain(&full_b[(ks - 1 - s) % a.sa], ((ks - 1 - s) / a.sa) & 1);
+            for (uint32_t s = 0; s < (uint32_t)a.sc && s < cks; ++s)
+                mbar_drain(&full_c[(cks - 1 - s) % a.sc], ((cks - 1 - s) / a.sc) & 1);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
             uint32_t st = 0, ph = 0, nacc = 0;
-            bool ok = true;
+            bool ok = true, issued = false;
             for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
                 const Item itm = item_of<BN>(it, MT, tiles, n_act, a.active, a.offsets);
                 const int n16 = (itm.n + 15) & ~15;
                 const uint32_t idesc = idesc_f16(BM, n16);
                 // both warpgroups' epilogues of the previous item have read the accumulators
-                if (!(ok = mbar_wait(acc_empty, (nacc & 1) ^ 1, abort_flag, a.err, 9)))
+                if (!(ok = mbar_wait(acc_empty, (nacc & 1) ^ 1, abort_flag, a.err, 9, a.wait_limit)))
                     break;
                 ++nacc;
                 tc_fence_after();
                 for (int k = 0; k < ksteps; ++k) {
-                    if (!(ok = mbar_wait(&full_a[st], ph, abort_flag, a.err, 4)))
+                    if (!(ok = mbar_wait(&full_a[st], ph, abort_flag, a.err, 4, a.wait_limit)))
                         break;
-                    if (!(ok = mbar_wait(&full_b[st], ph, abort_flag, a.err, 5)))
+                    if (!(ok = mbar_wait(&full_b[st], ph, abort_flag, a.err, 5, a.wait_limit)))
                         break;
                     tc_fence_after();
                     const uint64_t bdesc = sw128_desc(smem_u32(sm_b + (size_t)st * B_TILE));
@@ -431,6 +438,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                             umma_ts(tmem + m * BN, a_tmem + 8 * k16, bdesc + 2 * k16, idesc, (k | k16) != 0);
                         }
                     umma_commit(&empty[st]);
+                    issued = true;
                     if (++st == (uint32_t)a.sa) {
                         st = 0;
                         ph ^= 1;
@@ -438,6 +446,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                 }
                 if (ok)
                     umma_commit(acc_full);
+            }
+            if (issued) {
+                // every MMA has completed before the tensor memory is freed (after a give-up
+                // elsewhere in the CTA, the last ones may still run)
+                umma_commit(drain_bar);
+                mbar_drain(drain_bar, 0);
             }
         }
     } else {
@@ -459,7 +473,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                 lrow[m] = prow[m] >= 0 ? (int)(prow[m] - tile_prow0(md, itm.e, itm.m0)) : -1;
             }
             for (int c = 0; c < nchunks && ok; ++c) {
-                if (!(ok = mbar_wait(&full_c[cst], cph, abort_flag, a.err, 6)))
+                if (!(ok = mbar_wait(&full_c[cst], cph, abort_flag, a.err, 6, a.wait_limit)))
                     break;
                 const uint8_t *crow[2];
                 const uint16_t *srow[2];
@@ -494,7 +508,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                         if constexpr (NMOD == 2)
                             dequant_step<D, BITS, P::L, JJ>(crow[1], sm_cb + cb_bytes, rep_off, sfetch(1, JJ),
                                                             lrow[1] >= 0, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
-                        if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag, a.err, 7)))
+                        if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag, a.err, 7, a.wait_limit)))
                             return;
                         tc_fence_after();   // the stage's previous MMA has read it
                         if constexpr (NMOD == 2)
@@ -523,7 +537,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                 break;
             // epilogue: accumulators of this tile are complete; the warpgroups
             // take alternate 32-column blocks
-            if (!(ok = mbar_wait(acc_full, nit & 1, abort_flag, a.err, 8)))
+            if (!(ok = mbar_wait(acc_full, nit & 1, abort_flag, a.err, 8, a.wait_limit)))
                 break;
             ++nit;
             tc_fence_after();
@@ -533,19 +547,48 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                 if (nmod == 2)
                     tmem_ld32(tmem + lane_addr + BN + cb0, u);
                 tmem_wait_ld();
-                if (r < a.rows) {
+                if (a.swiglu) {
+                    // the tile's 32 token columns j: the accumulators carry each token's activation
+                    // scale 2^k, undone exactly; h = silu(g) u in fp32. The down GEMM reads h as fp16, so
+                    // each (slot, 32-row block) is stored times 2^e, e putting the block's largest |h| in
+                    // [2^14, 2^15), and e is recorded (the slot's blocks are brought to one exponent
+                    // before the down GEMM). The warp's rows lie inside the module or outside it whole
+                    // (rows is a multiple of 32).
+                    const int wrow0 = itm.m0 + 32 * (warp & 3);
+                    if (wrow0 < a.rows) {
+                        // lane j holds the inverse activation scale of column j
+                        const float fl = cb0 + lane < itm.n ? a.sxinv[itm.q0 + cb0 + lane] : 0.f;
+                        int my_e = 0;   // lane j: the exponent of column j
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int n = cb0 + j;
+                            const float f = __shfl_sync(0xFFFFFFFFu, fl, j);
+                            const float gv = __uint_as_float(g[j]) * f, uv = __uint_as_float(u[j]) * f;
+                            const float hv = __fdividef(gv, 1.f + __expf(-gv)) * uv;
+                            // the column's largest |h| over the warp's 32 rows, in every lane
+                            const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(hv) & 0x7FFFFFFFu);
+                            const int e = scale_exp(m);
+                            my_e = lane == j ? e : my_e;
+                            if (n < itm.n)
+                                reinterpret_cast<__half *>(a.out)[(long)(itm.q0 + n) * a.rows + r] =
+                                    __float2half_rn(hv * pow2f_normal(e));
+                        }
+                        if (cb0 + lane < itm.n)
+                            a.hexp[(long)(itm.q0 + cb0 + lane) * a.nblk32 + (wrow0 >> 5)] = (int8_t)my_e;
+                    }
+                } else if (r < a.rows) {
+                    // fp32 accumulators of one module, or of both (then u holds module 1's), times the
+                    // inverse activation scale when the kernel applies it
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int n = cb0 + j;
                         if (n >= itm.n)
                             break;
                         const long o = (long)(itm.q0 + n) * a.rows + r;
-                        if (a.swiglu) {
-                            const float gv = __uint_as_float(g[j]), uv = __uint_as_float(u[j]);
-                            reinterpret_cast<__half *>(a.out)[o] = __float2half_rn(gv / (1.f + __expf(-gv)) * uv);
-                        } else {
-                            reinterpret_cast<float *>(a.out)[o] = __uint_as_float(g[j]);
-                        }
+                        const float f = a.sxinv ? a.sxinv[itm.q0 + n] : 1.f;
+                        reinterpret_cast<float *>(a.out)[o] = __uint_as_float(g[j]) * f;
+                        if (nmod == 2)
+                            reinterpret_cast<float *>(a.out2)[o] = __uint_as_float(u[j]) * f;
                     }
                 }
             }
@@ -562,9 +605,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
     }
 }
 
-// gathered activations: Xg[q, :] = fp16(x[perm[q] / k, :])
-__global__ void vq_gather_kernel(const uint16_t *__restrict__ x, const int32_t *__restrict__ perm, int k, long slots,
-                                 int H, __half *__restrict__ xg)
+// gathered activations: Xg[q, :] = x16[perm[q] / k, :] (the token's scaled fp16
+// row) and sxinv[q] = xinv[perm[q] / k] (its inverse scale)
+__global__ void vq_gather_kernel(const __half *__restrict__ x16, const float *__restrict__ xinv,
+                                 const int32_t *__restrict__ perm, int k, long slots, int H, __half *__restrict__ xg,
+                                 float *__restrict__ sxinv)
 {
     grid_dep_launch();   // the next kernel may start its prologue; it waits for this one's results
     grid_dep_wait();
@@ -573,13 +618,54 @@ __global__ void vq_gather_kernel(const uint16_t *__restrict__ x, const int32_t *
         const long q = i / per_row;
         const int c = (int)(i % per_row) * 8;
         const long t = perm[q] / k;
-        const uint4 v = ldg_u128(x + t * H + c);
-        uint4 o;
-        o.x = bf16x2_to_f16x2(v.x);
-        o.y = bf16x2_to_f16x2(v.y);
-        o.z = bf16x2_to_f16x2(v.z);
-        o.w = bf16x2_to_f16x2(v.w);
-        *reinterpret_cast<uint4 *>(xg + q * H + c) = o;
+        *reinterpret_cast<uint4 *>(xg + q * H + c) = ldg_u128(x16 + t * H + c);
+        if (c == 0)
+            sxinv[q] = xinv[t];
+    }
+}
+
+// The gate/up epilogue stored each (slot, 32-row block) of h with its own
+// exponent e_b (hexp). Per slot q, every block is brought to the slot's
+// exponent E = min_b e_b (the one of its largest |h|): hs *= 2^(E - e_b), a
+// power of two <= 1, exact unless a value falls into fp16's subnormal range;
+// and the slot's pair p = perm[q] gets wh[p] = w[p] * 2^-E, the routing weight
+// that the combine applies to the down projection. One warp per slot; a lane
+// rescales whole 64-byte blocks.
+__global__ void vq_hnorm_kernel(__half *__restrict__ h, const int8_t *__restrict__ hexp, long slots, int nblk,
+                                const int32_t *__restrict__ perm, const float *__restrict__ w, float *__restrict__ wh)
+{
+    grid_dep_launch();   // the next kernel may start its prologue; it waits for this one's results
+    grid_dep_wait();
+    const int lane = threadIdx.x & 31;
+    const long nwarps = (long)gridDim.x * (blockDim.x >> 5);
+    for (long q = blockIdx.x * (long)(blockDim.x >> 5) + (threadIdx.x >> 5); q < slots; q += nwarps) {
+        const int8_t *eq = hexp + q * nblk;
+        int E = 127;
+        for (int b = lane; b < nblk; b += 32)
+            E = min(E, (int)eq[b]);
+        E = max(__reduce_min_sync(0xFFFFFFFFu, E), -126);
+        if (lane == 0) {
+            const int p = perm[q];
+            wh[p] = w[p] * pow2f(-E);
+        }
+        for (int b = lane; b < nblk; b += 32) {
+            const int d = max(E - (int)eq[b], -64);   // beyond 2^-64 every fp16 value becomes 0
+            if (d >= 0)
+                continue;
+            const float sc = pow2f(d);
+            uint4 *p = reinterpret_cast<uint4 *>(h + (q * nblk + b) * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                uint4 x = p[v];
+                __half2 *hw = reinterpret_cast<__half2 *>(&x);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = __half22float2(hw[i]);   // exact; the product too, then one rounding
+                    hw[i] = __floats2half2_rn(f.x * sc, f.y * sc);
+                }
+                p[v] = x;
+            }
+        }
     }
 }
 
@@ -638,7 +724,7 @@ SmemPlan smem_plan(int nmod, int d, int bits, int E)
         p.off_cb = p.off_c + p.sc * code_stage;
         p.off_tiles = p.off_cb + cb;
         p.off_bar = (uint32_t)align_up(p.off_tiles + tiles, 8);
-        p.total = p.off_bar + (3 * sa + 2 * p.sc + 2) * 8 + 16 + 1024;
+        p.total = p.off_bar + (3 * sa + 2 * p.sc + 3) * 8 + 16 + 1024;
         if (p.total <= limit + 1024)
             return p;
     }
@@ -650,7 +736,7 @@ template <int D, int BITS, int NMOD>
 cudaError_t launch_gemm(const PrefillArgs &a, int ctas, uint32_t smem, cudaStream_t s)
 {
     auto k = vq_prefill_gemm_kernel<D, BITS, NMOD>;
-    cudaError_t err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t err = set_smem_limit_once((const void *)k, (int)smem);
     if (err != cudaSuccess)
         return err;
     cudaLaunchConfig_t cfg = {};
@@ -678,7 +764,7 @@ cudaError_t dispatch_gemm(const PrefillArgs &a, int d, int bits, int ctas, uint3
 
 struct PrefillPlan {
     RoutingLayout r;
-    size_t xg, h, dp, total;
+    size_t x16, xinv, xg, sxinv, h, hexp, wh, dp, total;
 };
 
 PrefillPlan plan_prefill(const vq_moe_layer *L, int T, int k)
@@ -687,11 +773,48 @@ PrefillPlan plan_prefill(const vq_moe_layer *L, int T, int k)
     size_t o = 0;
     p.r = plan_routing(o, T, k, L->gate.E);
     const size_t tk = (size_t)T * k;
-    p.xg = o; o = align_up(o + tk * L->gate.cols * 2, 256);
-    p.h = o; o = align_up(o + tk * L->gate.rows * 2, 256);
-    p.dp = o; o = align_up(o + tk * L->down.rows * 4, 256);
+    const size_t H = L->gate.cols, I = L->gate.rows;
+    p.x16 = o; o = align_up(o + (size_t)T * H * 2, 256);     // scaled fp16 activations, per token
+    p.xinv = o; o = align_up(o + (size_t)T * 4, 256);        // their inverse scales
+    p.xg = o; o = align_up(o + tk * H * 2, 256);             // gathered by bucket slot
+    p.sxinv = o; o = align_up(o + tk * 4, 256);
+    p.h = o; o = align_up(o + tk * I * 2, 256);              // SwiGLU output, scaled fp16
+    p.hexp = o; o = align_up(o + tk * (I / 32), 256);        // exponents of its 32-row blocks
+    p.wh = o; o = align_up(o + tk * 4, 256);                 // routing weights times the h scales
+    p.dp = o; o = align_up(o + tk * L->down.rows * 4, 256);  // per-slot down outputs
     p.total = o;
     return p;
+}
+
+// The tensor maps and shared-memory layout of one GEMM launch: nmod modules
+// (same geometry and shape) against the fp16 activations act [slots, K].
+vq_status setup_gemm(PrefillArgs &a, const vq_module *m0, const vq_module *m1, const void *act, long slots, int E,
+                     SmemPlan &sp)
+{
+    a.mod[0] = make_moddev(*m0);
+    a.mod[1] = make_moddev(m1 ? *m1 : *m0);
+    a.nmod = m1 ? 2 : 1;
+    sp = smem_plan(a.nmod, a.mod[0].d, a.mod[0].bits, E);
+    if (sp.total == 0)
+        return VQ_ERR_UNSUPPORTED;   // the geometry's stages and codebooks do not fit shared memory
+    if (!map_act(&a.tmap_b, act, slots, a.mod[0].cols, bn_of(a.nmod)) || !map_codes(&a.tmap_c[0], a.mod[0]) ||
+        !map_codes(&a.tmap_c[1], a.mod[1]))
+        return VQ_ERR_CUDA;
+    a.scale_tma = a.mod[0].ngroups % 8 == 0;
+    if (a.scale_tma && (!map_scales(&a.tmap_s[0], a.mod[0]) || !map_scales(&a.tmap_s[1], a.mod[1])))
+        return VQ_ERR_CUDA;
+    a.K = a.mod[0].cols;
+    a.rows = a.mod[0].rows;
+    a.sa = sp.sa;
+    a.sc = sp.sc;
+    a.off_a = sp.off_a;
+    a.off_b = sp.off_b;
+    a.off_c = sp.off_c;
+    a.off_cb = sp.off_cb;
+    a.off_tiles = sp.off_tiles;
+    a.off_bar = sp.off_bar;
+    a.wait_limit = current_wait_limit();
+    return VQ_OK;
 }
 
 bool module_prefill_ok(const vq_module &m)
@@ -714,6 +837,9 @@ vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const flo
         return VQ_ERR_UNSUPPORTED;
     if (L->gate.d != L->up.d || L->gate.bits != L->up.bits)
         return VQ_ERR_UNSUPPORTED;   // gate and up share one fused tile
+    if (smem_plan(2, L->gate.d, L->gate.bits, L->gate.E).total == 0 ||
+        smem_plan(1, L->down.d, L->down.bits, L->gate.E).total == 0)
+        return VQ_ERR_UNSUPPORTED;   // stages and codebooks do not fit shared memory (checked before any launch)
     if (!tma_available())
         return VQ_ERR_CUDA;
     const int E = L->gate.E, H = L->gate.cols, I = L->gate.rows;
@@ -730,8 +856,13 @@ vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const flo
     int32_t *active = ws_at<int32_t>(ws, p.r.active);
     int32_t *nact = ws_at<int32_t>(ws, p.r.nact);
     int *err = ws_at<int>(ws, p.r.err);
+    __half *x16 = ws_at<__half>(ws, p.x16);
+    float *xinv = ws_at<float>(ws, p.xinv);
     __half *xg = ws_at<__half>(ws, p.xg);
+    float *sxinv = ws_at<float>(ws, p.sxinv);
     __half *hh = ws_at<__half>(ws, p.h);
+    int8_t *hexp = ws_at<int8_t>(ws, p.hexp);
+    float *wh = ws_at<float>(ws, p.wh);
     float *dp = ws_at<float>(ws, p.dp);
     const long tk = (long)T * k;
     // the kernels count work items in 32 bits
@@ -743,7 +874,7 @@ vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const flo
 
     trace_point(0, s);
     cudaError_t e = launch_route(logits, T, E, k, renorm, ids, w, offsets, perm, pos, active, nact, nullptr, nullptr,
-                                 nullptr, nullptr, 0, err, s, true);
+                                 x, x16, xinv, H, err, s, true);
     if (e != cudaSuccess)
         return VQ_ERR_CUDA;
     trace_point(1, s);
@@ -753,7 +884,8 @@ vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const flo
         cfg.gridDim = dim3((unsigned)std::min<long>((n + 255) / 256, 8192));
         cfg.blockDim = dim3(256);
         cfg.stream = s;
-        e = cudaLaunchKernelEx(&cfg, vq_gather_kernel, x, (const int32_t *)perm, k, tk, H, xg);
+        e = cudaLaunchKernelEx(&cfg, vq_gather_kernel, (const __half *)x16, (const float *)xinv, (const int32_t *)perm,
+                               k, tk, H, xg, sxinv);
         if (e != cudaSuccess)
             return VQ_ERR_CUDA;
     }
@@ -763,67 +895,43 @@ vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const flo
     // gate/up with the SwiGLU epilogue -> h fp16 [slots, inter]
     {
         PrefillArgs a{};
-        a.mod[0] = make_moddev(L->gate);
-        a.mod[1] = make_moddev(L->up);
-        a.nmod = 2;
-        if (!map_act(&a.tmap_b, xg, tk, H, bn_of(2)) || !map_codes(&a.tmap_c[0], a.mod[0]) || !map_codes(&a.tmap_c[1], a.mod[1]))
-            return VQ_ERR_CUDA;
-        if (a.mod[0].ngroups % 8 == 0 && (!map_scales(&a.tmap_s[0], a.mod[0]) || !map_scales(&a.tmap_s[1], a.mod[1])))
-            return VQ_ERR_CUDA;
+        SmemPlan sp;
+        if (const vq_status st = setup_gemm(a, &L->gate, &L->up, xg, tk, E, sp); st != VQ_OK)
+            return st;
         a.offsets = offsets;
         a.active = active;
         a.n_active = nact;
-        a.K = H;
-        a.rows = I;
-        const SmemPlan sp = smem_plan(2, a.mod[0].d, a.mod[0].bits, E);
-        if (sp.total == 0)
-            return VQ_ERR_UNSUPPORTED;
-        a.sa = sp.sa;
-        a.sc = sp.sc;
-        a.off_a = sp.off_a;
-        a.off_b = sp.off_b;
-        a.off_c = sp.off_c;
-        a.off_cb = sp.off_cb;
-        a.off_tiles = sp.off_tiles;
-        a.off_bar = sp.off_bar;
-        a.scale_tma = a.mod[0].ngroups % 8 == 0;
         a.out = hh;
         a.swiglu = 1;
+        a.sxinv = sxinv;
+        a.hexp = hexp;
+        a.nblk32 = I / 32;
         a.err = err;
         e = dispatch_gemm(a, a.mod[0].d, a.mod[0].bits, sms, sp.total, s);
         if (e != cudaSuccess)
             return VQ_ERR_CUDA;
     }
     trace_point(3, s);
-    // down -> fp32 per-slot outputs [slots, hidden]
+    // the slots' h blocks to one exponent per slot
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)std::max<long>(1, std::min<long>((tk + 7) / 8, 4096)));
+        cfg.blockDim = dim3(256);
+        cfg.stream = s;
+        e = cudaLaunchKernelEx(&cfg, vq_hnorm_kernel, hh, (const int8_t *)hexp, tk, I / 32, (const int32_t *)perm,
+                               (const float *)w, wh);
+        if (e != cudaSuccess)
+            return VQ_ERR_CUDA;
+    }
+    // down -> fp32 per-slot outputs [slots, hidden], still times the slot's h scale (the combine undoes it)
     {
         PrefillArgs a{};
-        a.mod[0] = make_moddev(L->down);
-        a.mod[1] = a.mod[0];
-        a.nmod = 1;
-        if (!map_act(&a.tmap_b, hh, tk, I, bn_of(1)) || !map_codes(&a.tmap_c[0], a.mod[0]))
-            return VQ_ERR_CUDA;
-        if (a.mod[0].ngroups % 8 == 0 && !map_scales(&a.tmap_s[0], a.mod[0]))
-            return VQ_ERR_CUDA;
-        a.tmap_c[1] = a.tmap_c[0];
-        a.tmap_s[1] = a.tmap_s[0];
+        SmemPlan sp;
+        if (const vq_status st = setup_gemm(a, &L->down, nullptr, hh, tk, E, sp); st != VQ_OK)
+            return st;
         a.offsets = offsets;
         a.active = active;
         a.n_active = nact;
-        a.K = I;
-        a.rows = H;
-        const SmemPlan sp = smem_plan(1, a.mod[0].d, a.mod[0].bits, E);
-        if (sp.total == 0)
-            return VQ_ERR_UNSUPPORTED;
-        a.sa = sp.sa;
-        a.sc = sp.sc;
-        a.off_a = sp.off_a;
-        a.off_b = sp.off_b;
-        a.off_c = sp.off_c;
-        a.off_cb = sp.off_cb;
-        a.off_tiles = sp.off_tiles;
-        a.off_bar = sp.off_bar;
-        a.scale_tma = a.mod[0].ngroups % 8 == 0;
         a.out = dp;
         a.swiglu = 0;
         a.err = err;
@@ -832,8 +940,92 @@ vq_status run_prefill(const vq_moe_layer *L, const uint16_t *x, int T, const flo
             return VQ_ERR_CUDA;
     }
     trace_point(4, s);
-    e = launch_combine(dp, 1, 0, w, pos, T, k, H, y, y_dtype, s, true);
+    e = launch_combine(dp, 1, 0, wh, pos, T, k, H, y, y_dtype, s, true);
     trace_point(5, s);
+    return e == cudaSuccess ? VQ_OK : VQ_ERR_CUDA;
+}
+
+namespace {
+
+__global__ void vq_gemm_tables_kernel(int E, int expert, int T, int32_t *offsets, int32_t *active, int32_t *nact,
+                                      int *err)
+{
+    grid_dep_launch();
+    grid_dep_wait();
+    for (int i = threadIdx.x; i <= E; i += blockDim.x)
+        offsets[i] = i <= expert ? 0 : T;
+    if (threadIdx.x == 0) {
+        active[0] = expert;
+        *nact = 1;
+        *err = 0;
+    }
+}
+
+struct GemmPlan {
+    size_t err, offsets, active, nact, x16, xinv, total;
+};
+
+GemmPlan plan_gemm(const vq_module *m, int T)
+{
+    GemmPlan p{};
+    size_t o = 0;
+    p.err = o; o = align_up(o + 4, 256);
+    p.offsets = o; o = align_up(o + (size_t)(m->E + 1) * 4, 256);
+    p.active = o; o = align_up(o + 4, 256);
+    p.nact = o; o = align_up(o + 4, 256);
+    p.x16 = o; o = align_up(o + (size_t)T * m->cols * 2, 256);
+    p.xinv = o; o = align_up(o + (size_t)T * 4, 256);
+    p.total = o;
+    return p;
+}
+
+}  // namespace
+
+size_t gemm_workspace_size(const vq_module *m, int T) { return plan_gemm(m, T).total; }
+
+vq_status run_gemm(const vq_module *m0, const vq_module *m1, int expert, const uint16_t *x, int T, float *y0, float *y1,
+                   void *ws, size_t ws_bytes, cudaStream_t s)
+{
+    if (!module_prefill_ok(*m0) || (m1 && !module_prefill_ok(*m1)) ||
+        smem_plan(m1 ? 2 : 1, m0->d, m0->bits, m0->E).total == 0)
+        return VQ_ERR_UNSUPPORTED;
+    if (!tma_available())
+        return VQ_ERR_CUDA;
+    if (T == 0)
+        return VQ_OK;
+    const GemmPlan p = plan_gemm(m0, T);
+    if (ws_bytes < p.total)
+        return VQ_ERR_WORKSPACE;
+    // the kernels count work items in 32 bits
+    if (((long)(T + bn_of(m1 ? 2 : 1) - 1) / bn_of(m1 ? 2 : 1) + 1) * ((m0->rows + BM - 1) / BM) >= INT_MAX)
+        return VQ_ERR_UNSUPPORTED;
+    int32_t *offsets = ws_at<int32_t>(ws, p.offsets), *active = ws_at<int32_t>(ws, p.active);
+    int32_t *nact = ws_at<int32_t>(ws, p.nact);
+    int *err = ws_at<int>(ws, p.err);
+    __half *x16 = ws_at<__half>(ws, p.x16);
+    float *xinv = ws_at<float>(ws, p.xinv);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, vq_gemm_tables_kernel, m0->E, expert, T, offsets, active, nact, err);
+    if (e == cudaSuccess)
+        e = launch_convert(x, x16, xinv, T, m0->cols, s, false);
+    if (e != cudaSuccess)
+        return VQ_ERR_CUDA;
+    PrefillArgs a{};
+    SmemPlan sp;
+    if (const vq_status st = setup_gemm(a, m0, m1, x16, T, m0->E, sp); st != VQ_OK)
+        return st;
+    a.offsets = offsets;
+    a.active = active;
+    a.n_active = nact;
+    a.out = y0;
+    a.out2 = y1;
+    a.swiglu = 0;
+    a.sxinv = xinv;
+    a.err = err;
+    e = dispatch_gemm(a, a.mod[0].d, a.mod[0].bits, num_sms(), sp.total, s);
     return e == cudaSuccess ? VQ_OK : VQ_ERR_CUDA;
 }
 

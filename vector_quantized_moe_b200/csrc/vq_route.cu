@@ -284,34 +284,54 @@ __device__ __noinline__ void bucket(const int32_t *ids, int npairs, int E, int32
     }
 }
 
-// x16[t, c] = fp16(x[t, c]) for the tokens [t0, t1) (the tensor-core kernels
-// read fp16 activations; bf16 -> fp16 is exact for magnitudes in [2^-14, 65504]).
-// Rows of H % 8 == 0 elements are 16-byte aligned: four 16-byte loads per
-// thread are in flight before the first store.
-__device__ void convert_rows(const uint16_t *x, __half *x16, int t0, int t1, int H, int tid, int nthr)
+// x16[t, :] = fp16(x[t, :] * 2^k_t) and xinv[t] = 2^-k_t for the tokens
+// [t0, t1), one token per warp over the warps [w0, w0 + nw) of the CTA. k_t
+// brings the token's largest |x| into [2^14, 2^15) (scale_exp), so every bf16
+// value keeps its full precision in fp16 (down to 2^-28 of the largest) and no
+// value overflows; the consumers undo the scale exactly in fp32. Rows of
+// H % 8 == 0 elements are 16-byte aligned; the row is read twice (the second
+// time from L1).
+__device__ void convert_rows(const uint16_t *x, __half *x16, float *xinv, int t0, int t1, int H, int w0, int nw)
 {
     if (!x)
         return;
-    const long n8 = (long)(t1 - t0) * H / 8;
-    const uint4 *src = reinterpret_cast<const uint4 *>(x + (long)t0 * H);
-    uint4 *dst = reinterpret_cast<uint4 *>(x16 + (long)t0 * H);
-    const long step = nthr;
-    for (long i0 = tid; i0 < n8; i0 += 4 * step) {
-        uint4 v[4];
+    const int lane = threadIdx.x & 31;
+    const int n8 = H / 8;
+    for (int t = t0 + (int)(threadIdx.x >> 5) - w0; t < t1; t += nw) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (long)t * H);
+        uint4 *dst = reinterpret_cast<uint4 *>(x16 + (long)t * H);
+        uint32_t m = 0;
+        for (int i0 = lane; i0 < n8; i0 += 8 * 32) {
+            uint4 v[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (i0 + u * step < n8)
-                v[u] = ldg_u128(src + i0 + u * step);
+            for (int u = 0; u < 8; ++u)
+                v[u] = i0 + 32 * u < n8 ? ldg_u128(src + i0 + 32 * u) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (i0 + u * step < n8) {
-                uint4 o;
-                o.x = bf16x2_to_f16x2(v[u].x);
-                o.y = bf16x2_to_f16x2(v[u].y);
-                o.z = bf16x2_to_f16x2(v[u].z);
-                o.w = bf16x2_to_f16x2(v[u].w);
-                dst[i0 + u * step] = o;
-            }
+            for (int u = 0; u < 8; ++u)
+                m = max(m, bf16x8_max_mag(v[u]));
+        }
+        m = __reduce_max_sync(0xFFFFFFFFu, m);
+        const int k = scale_exp(m << 16);
+        const float s = pow2f_normal(k);
+        if (lane == 0 && xinv)
+            xinv[t] = pow2f(-k);
+        for (int i0 = lane; i0 < n8; i0 += 8 * 32) {
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (i0 + 32 * u < n8)
+                    v[u] = ldg_u128(src + i0 + 32 * u);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (i0 + 32 * u < n8) {
+                    uint4 o;
+                    o.x = bf16x2_to_f16x2_scaled(v[u].x, s);
+                    o.y = bf16x2_to_f16x2_scaled(v[u].y, s);
+                    o.z = bf16x2_to_f16x2_scaled(v[u].z, s);
+                    o.w = bf16x2_to_f16x2_scaled(v[u].w, s);
+                    dst[i0 + 32 * u] = o;
+                }
+        }
     }
 }
 
@@ -352,8 +372,8 @@ __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_fused_kernel(const flo
                                                                       int32_t *offsets, int32_t *perm, int32_t *pos,
                                                                       int32_t *active, int32_t *n_active,
                                                                       int2 *passes, int32_t *n_passes,
-                                                                      const uint16_t *x, __half *x16, int H, int *err,
-                                                                      const ZeroSpans zero)
+                                                                      const uint16_t *x, __half *x16, float *xinv, int H,
+                                                                      int *err, const ZeroSpans zero)
 {
     if (blockIdx.x > 0) {
         grid_dep_launch();
@@ -399,10 +419,10 @@ __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_fused_kernel(const flo
         if (warp < T)
             route_range(logits, 0, T, E, k, renorm, ids, w, 0, T);
         else
-            convert_rows(x, x16, 0, T, H, threadIdx.x - 32 * T, blockDim.x - 32 * T);
+            convert_rows(x, x16, xinv, 0, T, H, T, nw - T);
     } else {
         route_range(logits, 0, T, E, k, renorm, ids, w, 0, nw);
-        convert_rows(x, x16, 0, T, H, threadIdx.x, blockDim.x);
+        convert_rows(x, x16, xinv, 0, T, H, 0, nw);
     }
     __syncthreads();
     for (int p = threadIdx.x; p < npairs; p += blockDim.x)
@@ -416,8 +436,8 @@ constexpr int ROUTE_TOKENS_PER_CTA = 256;
 
 __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_topk_kernel(const float *logits, int T, int E, int k,
                                                                      int renorm, int32_t *ids, float *w,
-                                                                     const uint16_t *x, __half *x16, int H, int *err,
-                                                                     const ZeroSpans zero)
+                                                                     const uint16_t *x, __half *x16, float *xinv, int H,
+                                                                     int *err, const ZeroSpans zero)
 {
     grid_dep_launch();   // the next kernel may start its prologue; it waits for this one's results
     grid_dep_wait();
@@ -425,7 +445,7 @@ __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_topk_kernel(const floa
         *err = 0;
     zero_spans(zero, blockIdx.x, gridDim.x);
     const int t0 = blockIdx.x * ROUTE_TOKENS_PER_CTA;
-    convert_rows(x, x16, t0, min(T, t0 + ROUTE_TOKENS_PER_CTA), H, threadIdx.x, blockDim.x);
+    convert_rows(x, x16, xinv, t0, min(T, t0 + ROUTE_TOKENS_PER_CTA), H, 0, blockDim.x >> 5);
     route_range(logits, t0, min(T, t0 + ROUTE_TOKENS_PER_CTA), E, k, renorm, ids, w, 0, blockDim.x >> 5);
 }
 
@@ -440,6 +460,15 @@ __global__ void __launch_bounds__(BUCKET_THREADS) vq_bucket_kernel(const int32_t
     grid_dep_wait();
     bucket(ids, npairs, E, offsets, perm, pos, active, n_active, passes, n_passes, sm, sm + (size_t)chunks * E,
            chunks);
+}
+
+// The activation conversion alone: warps over the tokens.
+__global__ void __launch_bounds__(256) vq_convert_kernel(const uint16_t *x, __half *x16, float *xinv, int T, int H)
+{
+    grid_dep_launch();   // the next kernel may start its prologue; it waits for this one's results
+    grid_dep_wait();
+    const int wpc = blockDim.x >> 5;
+    convert_rows(x, x16, xinv, blockIdx.x * wpc, T, H, 0, gridDim.x * wpc);
 }
 
 template <typename K, typename... Args>
@@ -462,8 +491,8 @@ cudaError_t launch_ex(K kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t
 
 cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, int32_t *ids, float *w,
                          int32_t *offsets, int32_t *perm, int32_t *pos, int32_t *active, int32_t *n_active,
-                         int2 *passes, int32_t *n_passes, const uint16_t *x, __half *x16, int H, int *errw,
-                         cudaStream_t s, bool pdl, const ZeroSpans *zero)
+                         int2 *passes, int32_t *n_passes, const uint16_t *x, __half *x16, float *xinv, int H,
+                         int *errw, cudaStream_t s, bool pdl, const ZeroSpans *zero)
 {
     ZeroSpans z{};
     if (zero)
@@ -476,16 +505,12 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
     // + 8192 pair ids + the warm-up scratch (the fused CTA, 112 KB); the kernels'
     // static tables come on top
     constexpr size_t ROUTE_SMEM_MAX = 170 * 1024;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t err = cudaFuncSetAttribute(vq_route_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)ROUTE_SMEM_MAX);
+    {
+        cudaError_t err = set_smem_limit_once((const void *)vq_route_fused_kernel, (int)ROUTE_SMEM_MAX);
         if (err == cudaSuccess)
-            err = cudaFuncSetAttribute(vq_bucket_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)ROUTE_SMEM_MAX);
+            err = set_smem_limit_once((const void *)vq_bucket_kernel, (int)ROUTE_SMEM_MAX);
         if (err != cudaSuccess)
             return err;
-        attr_set = true;
     }
     const bool fused = T <= ROUTE_TOKENS_PER_CTA;
     const size_t smem = bucket_smem_ints(E, T * k, fused, fused ? ROUTE_THREADS : BUCKET_THREADS, k) * sizeof(int32_t);
@@ -493,14 +518,29 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
         return cudaErrorInvalidValue;
     if (fused)
         return launch_ex(vq_route_fused_kernel, dim3(1 + zctas), dim3(ROUTE_THREADS), smem, s, pdl, logits, T, E, k,
-                         renorm, ids, w, offsets, perm, pos, active, n_active, passes, n_passes, x, x16, H, errw, z);
+                         renorm, ids, w, offsets, perm, pos, active, n_active, passes, n_passes, x, x16, xinv, H, errw, z);
     const int ctas = (T + ROUTE_TOKENS_PER_CTA - 1) / ROUTE_TOKENS_PER_CTA;
+    // many tokens: the activations are converted by a launch of their own, over the whole GPU
     cudaError_t err = launch_ex(vq_route_topk_kernel, dim3(ctas), dim3(ROUTE_THREADS), 0, s, pdl, logits, T, E, k,
-                                renorm, ids, w, x, x16, H, errw, z);
+                                renorm, ids, w, (const uint16_t *)nullptr, (__half *)nullptr, (float *)nullptr, H, errw,
+                                z);
+    if (err == cudaSuccess && x)
+        err = launch_ex(vq_convert_kernel, dim3(std::max(1, std::min((T + 7) / 8, 4096))), dim3(256), 0, s, pdl, x,
+                        x16, xinv, T, H);
     if (err != cudaSuccess)
         return err;
     return launch_ex(vq_bucket_kernel, dim3(1), dim3(BUCKET_THREADS), smem, s, pdl, (const int32_t *)ids, T * k, E,
                      offsets, perm, pos, active, n_active, passes, n_passes);
+}
+
+}  // namespace vq
+
+namespace vq {
+
+cudaError_t launch_convert(const uint16_t *x, __half *x16, float *xinv, int T, int H, cudaStream_t s, bool pdl)
+{
+    const int blocks = std::max(1, std::min((T + 7) / 8, 2048));
+    return launch_ex(vq_convert_kernel, dim3(blocks), dim3(256), 0, s, pdl, x, x16, xinv, T, H);
 }
 
 }  // namespace vq

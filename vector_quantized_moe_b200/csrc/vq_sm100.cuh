@@ -7,8 +7,10 @@
 
 namespace vq {
 
-// Upper bound on the polls of one mbarrier wait (each poll may suspend
-// briefly); a wait that reaches it gives up and reports an error.
+// Default bound on the polls of one mbarrier wait (each poll may suspend
+// briefly); a wait that reaches its bound gives up and reports an error. The
+// kernels take the bound as an argument (vq_set_wait_limit), and the drains
+// after a give-up use this one.
 constexpr uint32_t WAIT_LIMIT = 1u << 22;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -41,20 +43,41 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
-// Bounded wait on a phase; false when it gave up (limit reached or the CTA aborted).
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *err,
-                                          int code)
+// The cold end of a bounded wait that ran out: sets the CTA's abort flag and
+// records `code` in *err. Kept out of line so that the wait sites stay small.
+static __device__ __noinline__ bool mbar_give_up(volatile int *abort_flag, int *err, int code)
 {
-    for (uint32_t i = 0; i < WAIT_LIMIT; ++i) {
+    *abort_flag = 1;
+    if (err)
+        atomicExch(err, code);
+    return false;
+}
+
+// Bounded wait on a phase: at most `limit` polls (limit 0: none). False when
+// it gave up: at the bound it sets the CTA's abort flag and records `code` in
+// *err; it also returns false (within 64 polls) once another thread of the
+// CTA has aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *err,
+                                          int code, uint32_t limit)
+{
+    for (uint32_t i = 0; i < limit; ++i) {
         if (mbar_try_wait(bar, parity))
             return true;
         if ((i & 63) == 63 && *abort_flag)
             return false;
     }
-    *abort_flag = 1;
-    if (err)
-        atomicExch(err, code);
-    return false;
+    return mbar_give_up(abort_flag, err, code);
+}
+
+// After a give-up: waits for a phase that work already issued by this thread
+// (TMA copies, MMAs) completes by itself, so that the CTA leaves no copy or
+// MMA in flight when it frees its tensor memory and exits. Ignores the abort
+// flag; bounded by WAIT_LIMIT polls.
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity)
+{
+    for (uint32_t i = 0; i < WAIT_LIMIT; ++i)
+        if (mbar_try_wait(bar, parity))
+            return;
 }
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar)
