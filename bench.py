@@ -1,16 +1,21 @@
 """Benchmark of the VQ-MoE hot path on B200 (one JSON line on rank 0).
 
-Default workload: the MoE decode layer with d=2/K=256 experts (512 experts,
-top-10, hidden 4096, inter 1024, 8 tokens per step). A step is one
-vq_moe_decode call: routing, bucketing, the gate/up grouped VQ GEMV, SwiGLU,
-the down grouped VQ GEMV and the weighted combine, over one batch of seeded
-synthetic inputs rotated among 16 routing draws (3.4 GB of expert weights, far
-beyond L2, so a step's experts are not L2-resident from the previous step).
+Default workload (the headline): the MoE decode layer with d=4/K=512 (9-bit
+codes) in all three projections, 256 experts top-8, hidden 6144, inter 2048, 16
+tokens per step. A step is one vq_moe_decode call: routing and bucketing, the
+gate/up grouped VQ GEMV, SwiGLU, the down grouped VQ GEMV and the weighted
+combine, over one batch of seeded synthetic inputs rotated among 16 routing
+draws (3.0 GB of expert weights, far beyond L2, so a step's experts are not
+L2-resident from the previous step).
 
 metric: decode HBM GB/s = algorithmic bytes of a step (live codes and group
 scales of the experts the step touches, codebooks, activations, logits and
 outputs) / step time. The roofline object reports the gate/up grouped GEMV
-(the dominant kernel) against the measured HBM copy bandwidth.
+(the dominant kernel) against the measured HBM copy bandwidth. The other
+workloads of the configuration list (the single GEMV, the d=2/K=256 decode
+layer at 1 and 8 tokens, the d=4/K=2048 layer, the skipzero layer, the
+prefill layers) are reported under "extra", and a compact per-workload summary
+closes the line.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -37,12 +42,13 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 from synth import workloads as wl  # noqa: E402
 
-METRIC = "VQ expert decode HBM GB/s"
+METRIC = "VQ expert decode HBM GB/s (% of B200 peak); prefill TFLOP/s; MoE-layer tokens/s"
 UNIT = "GB/s"
 N_DRAWS = 16
+MAIN_SPEC, MAIN_T = wl.DECODE_D4K512, 16
 # the other decode workloads, reported under "extra": (layer, tokens)
-OTHER_DECODE = {"decode_d4k512_T16": (wl.DECODE_D4K512, 16), "decode_d4k2048_T16": (wl.DECODE_D4K2048, 16),
-                "decode_skipzero_T1": (wl.SKIPZERO_MIXED, 1)}
+OTHER_DECODE = {"decode_d2k256_T8": (wl.DECODE_D2K256, 8), "decode_d2k256_T1": (wl.DECODE_D2K256, 1),
+                "decode_d4k2048_T16": (wl.DECODE_D4K2048, 16), "decode_skipzero_T1": (wl.SKIPZERO_MIXED, 1)}
 
 
 def _peaks():
@@ -54,11 +60,14 @@ def _peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def _row_words(cols, geo):
+    """uint32 words of one packed row (the format's closed form, computed without either library)."""
+    return (cols // geo.d // 32) * geo.bits
+
+
 def _module_bytes(md):
     """Bytes of one expert's live codes + scales, per expert, for a module."""
-    import vector_quantized_moe_b200 as vq
-    rw = vq.packed_words(1, md.cols // md.d, md.bits)
-    per_row = rw * 4 + (md.cols // 64) * 2
+    per_row = _row_words(md.cols, wl.Geometry(md.d, md.bits)) * 4 + (md.cols // 64) * 2
     if md.bitmap is None:
         live = np.full(md.E, md.rows)
     else:
@@ -67,7 +76,8 @@ def _module_bytes(md):
 
 
 KERNEL_SOURCES = {
-    "grouped_gemv_gate_up": ("vq_decode.cu", "vq_device.cuh", "vq_sm100.cuh"),
+    "grouped_gemv_gate_up_d4k512": ("vq_decode.cu", "vq_device.cuh", "vq_sm100.cuh"),
+    "grouped_gemv_gate_up_d2k256": ("vq_decode.cu", "vq_device.cuh", "vq_sm100.cuh"),
     "prefill_gemm_gate_up": ("vq_prefill.cu", "vq_device.cuh", "vq_sm100.cuh"),
 }
 
@@ -171,20 +181,36 @@ def dist_sum(v, device, ws):
     return float(t.item())
 
 
+def _main_config(spec, T, per_expert, n_gpus):
+    """The workload's config, the same in both arms."""
+    return {"workload": spec.name, "T": T, "top_k": spec.top_k, "E": spec.E, "hidden": spec.hidden,
+            "inter": spec.inter, "geometry": f"d{spec.gate.d}K{1 << spec.gate.bits} ({spec.gate.bits}-bit codes) x3",
+            "l2": f"inputs larger than L2: {N_DRAWS} rotating routing draws over "
+                  f"{sum(float(p.sum()) for p in per_expert) / 1e9:.2f} GB of expert weights",
+            "parallelism": "replicas" if n_gpus > 1 else "single-gpu"}
+
+
+def _token_bytes(spec, per_expert, cb_bytes, ids):
+    """Algorithmic bytes of a set of routed tokens: the live codes and scales of the experts they
+    touch, the codebooks, and each token's activations (bf16), logits (fp32) and output (fp32)."""
+    n = ids.shape[0]
+    return float(sum(p[np.unique(ids)].sum() for p in per_expert) + cb_bytes
+                 + n * (spec.hidden * 2 + spec.E * 4 + spec.hidden * 4))
+
+
 def run_reference(args):
-    """The oracle (CPU, float64) on bounded samples of the same workload."""
+    """The reference arm: the oracle (CPU, float64) on bounded samples of the headline workload,
+    timed on the host's cores; rank 0 only. It loads nothing but the oracle."""
     ws, rank, _ = _dist()
     if rank != 0:
         return
     import oracle
-    oracle.build()
-    spec = wl.DECODE_D2K256
-    T = spec.batches[1]
-    import vector_quantized_moe_b200 as vq
-    mds = wl.layer_modules(spec, raw=False, row_words=lambda c, g: vq.packed_words(1, c // g.d, g.bits))
     from tests.helpers import oracle_module
+    oracle.build()
+    spec, T = MAIN_SPEC, MAIN_T
+    mds = wl.layer_modules(spec, raw=False, row_words=_row_words)
     oms = [oracle_module(m) for m in mds]
-    per_expert = sum(_module_bytes(m) for m in mds)
+    per_expert = [_module_bytes(m) for m in mds]
     cb_bytes = sum(m.codebook.nbytes for m in mds)
     draws = [wl.layer_inputs(spec, T, i) for i in range(N_DRAWS)]
     total_b, total_t = 0.0, 0.0
@@ -192,20 +218,21 @@ def run_reference(args):
         x, lg = draws[step % N_DRAWS]
         tok = np.array([step % T])
         ids, *_ = oracle.route(lg[tok], spec.top_k)
-        nbytes = float(per_expert[np.unique(ids)].sum() + cb_bytes + spec.hidden * 2 + spec.E * 4 + spec.hidden * 4)
         t0 = time.perf_counter()
         oracle.moe(*oms, x, lg, spec.top_k, tokens=tok)
         dt = time.perf_counter() - t0
         if step >= args.warmup:
-            total_b += nbytes
+            total_b += _token_bytes(spec, per_expert, cb_bytes, ids)
             total_t += dt
     value = total_b / total_t / 1e9
+    sample = f"one token of the {T}-token batch per step (its {spec.top_k} experts, all three projections), float64"
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_t / args.steps * 1e3,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": spec.name, "T": T, "sample": "1 token of the batch per step"},
+           "config": _main_config(spec, T, per_expert, args.gpus),
+           "tokens_per_s": args.steps / total_t,
            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-                            "sample": "one token per step (its 10 experts), float64 oracle"},
+                            "sample": sample},
            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
@@ -239,31 +266,16 @@ def run_ours(args):
             vq.fit(w, 4, 512, st, itx, 10)
         torch.cuda.synchronize()
         return
-    if args.only in OTHER_DECODE:
-        # profiler runs of another decode workload: warm-up, then the steps
-        import dataclasses
-        spec_x, T_x = OTHER_DECODE[args.only]
-        if args.small:
-            spec_x = dataclasses.replace(spec_x, E=64, name=spec_x.name.replace(f"e{spec_x.E}", "e64"))
-        mds = wl.layer_modules(spec_x, raw=False, row_words=lambda c, g: vq.packed_words(1, c // g.d, g.bits))
-        layer = vq.MoELayer(*[lib_module(m, device=dev) for m in mds])
-        x, lg = wl.layer_inputs(spec_x, T_x, 200)
-        xt, lt = torch.from_numpy(x.view(np.int16)).to(dev), torch.from_numpy(lg).to(dev)
-        y = torch.empty((T_x, spec_x.hidden), dtype=torch.float32, device=dev)
-        wsp = layer.workspace(T_x, spec_x.top_k, vq.VQ_MODE_DECODE, dev)
-        for i in range(args.warmup + args.steps):
-            layer.decode(xt, lt, spec_x.top_k, out=y, workspace=wsp)
-        torch.cuda.synchronize()
-        return
 
-    spec = wl.DECODE_D2K256
+    spec, T = MAIN_SPEC, MAIN_T
+    if args.only in OTHER_DECODE:
+        spec, T = OTHER_DECODE[args.only]
     if args.small:
-        # same per-expert shapes with 64 experts (430 MB of weights): the case for full ncu captures
+        # same per-expert shapes with 64 experts: the case for full ncu captures
         import dataclasses
-        spec = dataclasses.replace(spec, E=64, name=spec.name.replace("e512", "e64"))
-    T = spec.batches[1]
+        spec = dataclasses.replace(spec, E=64, name=spec.name.replace(f"e{spec.E}", "e64"))
     k = spec.top_k
-    mds = wl.layer_modules(spec, raw=False, row_words=lambda c, g: vq.packed_words(1, c // g.d, g.bits))
+    mds = wl.layer_modules(spec, raw=False, row_words=_row_words)
     mods = [lib_module(m, device=dev) for m in mds]
     layer = vq.MoELayer(*mods)
     per_expert = [_module_bytes(m) for m in mds]
@@ -304,7 +316,7 @@ def run_ours(args):
 
     if args.ncu:
         # minimal launch sequence for profiler captures: 16 route calls above,
-        # warmup * 5 launches, then steps * 5 launches
+        # the warm-up steps, then the timed steps (5 launches per step)
         for i in range(args.steps):
             step(i)
         torch.cuda.synchronize()
@@ -337,14 +349,7 @@ def run_ours(args):
     value = sum_over_ranks(my_bytes) / (ms_total * 1e-3) / 1e9
 
     # trace pass: per-stage durations from events recorded at stage boundaries
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
-    for i in range(args.steps):
-        vq.set_trace_events(evs[i])
-        step(i)
-    vq.set_trace_events(None)
-    torch.cuda.synchronize()
-    stage = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(5)] for i in range(args.steps)])
-    stage_ms = stage.mean(axis=0)
+    stage_ms = _traced(torch, vq, step, args.steps).mean(axis=0)
     gu_ms = float(stage_ms[1])
     gu_avg_bytes = float(np.mean([gu_bytes[i % N_DRAWS] for i in range(args.steps)]))
     hbm, tf_burst, tf_sust, src = _peaks()
@@ -403,50 +408,77 @@ def run_ours(args):
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(mds, draws, spec, T, per_expert, cb_bytes)
+    del layer, mods, xs, lgs, y, wsp, hx, hl, hy, dx, dl, dy
+    torch.cuda.empty_cache()
 
     extra = {}
     if not args.no_extra:
-        extra["decode_T1"] = measure_decode_t1(torch, vq, layer, spec, per_expert, cb_bytes, dev, args.steps,
-                                               args.warmup)
-        del layer, mods
-        torch.cuda.empty_cache()
-        extra["prefill"] = measure_prefill(torch, vq, dev, min(args.steps, 20), args.warmup)
         for key, (spec_x, T_x) in OTHER_DECODE.items():
-            extra[key] = measure_decode_layer(torch, vq, spec_x, T_x, dev, min(args.steps, 100), args.warmup)
+            extra[key] = measure_decode_layer(torch, vq, spec_x, T_x, dev, min(args.steps, 100), args.warmup,
+                                              traffic_tag="grouped_gemv_gate_up_d2k256" if key == "decode_d2k256_T8"
+                                              else None)
+        extra["gemv_d2k256_512x1024"] = measure_gemv_single(torch, vq, dev, min(args.steps, 20), args.warmup)
+        extra["prefill"] = measure_prefill(torch, vq, dev, min(args.steps, 20), args.warmup)
         extra["prefill_skipzero_T2048"] = measure_prefill(torch, vq, dev, min(args.steps, 20), args.warmup,
                                                           spec=wl.SKIPZERO_MIXED, T=2048)
         extra["prefill_chunked_T8192"] = measure_prefill_chunked(torch, vq, dev, min(args.steps, 5), args.warmup)
         extra["fit_d4k512"] = measure_fit(torch, vq, dev, min(args.steps, 5), args.warmup)
 
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": _traffic_per_launch("grouped_gemv_gate_up_d4k512") if not args.small else None,
+                "kernel": f"vq_gemv_tma_kernel<{spec.gate.d},{spec.gate.bits},fp16,dense> (gate+up)",
+                "peak_source": f"{src} hbm_gbs", "bytes_per_launch": gu_avg_bytes, "ms_per_launch": gu_ms}
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f16xf16->f32", "data": "synthetic",
-        "config": {"workload": spec.name, "T": T, "top_k": k, "E": spec.E, "hidden": spec.hidden,
-                   "inter": spec.inter, "geometry": "d2K256 (8-bit codes) x3",
-                   "l2": f"inputs larger than L2: {N_DRAWS} rotating routing draws over "
-                         f"{sum(float(p.sum()) for p in per_expert) / 1e9:.2f} GB of expert weights",
-                   "parallelism": "replicas" if ws > 1 else "single-gpu",
-                   "tokens_per_s": T * args.steps * ws / (ms_total * 1e-3)},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                     "traffic": _traffic_per_launch("grouped_gemv_gate_up"),
-                     "kernel": "vq_gemv_tma_kernel<2,8,fp16,dense> (gate+up)", "peak_source": f"{src} hbm_gbs",
-                     "bytes_per_launch": gu_avg_bytes, "ms_per_launch": gu_ms},
-        "stage_ms": {"route": float(stage_ms[0]), "gate_up_gemv": gu_ms, "swiglu": float(stage_ms[2]),
-                     "down_gemv": float(stage_ms[3]), "combine": float(stage_ms[4])},
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(xs[0].numel() * 2 + lgs[0].numel() * 4),
-                "d2h_bytes_per_step": int(y.numel() * 4),
+        "config": _main_config(spec, T, per_expert, ws),
+        "tokens_per_s": T * args.steps * ws / (ms_total * 1e-3),
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(draws[0][0].nbytes + draws[0][1].nbytes),
+                "d2h_bytes_per_step": int(T * spec.hidden * 4),
                 "pipeline": "pinned host buffers; inputs copied in on a copy stream one step ahead "
                             "(double-buffered), outputs copied out on another while the next step runs"},
         "gpu_launches": 5 * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,
+        "stage_ms": {"route": float(stage_ms[0]), "gate_up_gemv": gu_ms, "swiglu": float(stage_ms[2]),
+                     "down_gemv": float(stage_ms[3]), "combine": float(stage_ms[4])},
         "extra": extra,
+        "roofline": roofline,
     }
+    out["summary"] = _summary(out)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if ws > 1:
         torch.distributed.destroy_process_group()
+
+
+def _summary(out):
+    """A compact line per workload (value, unit, roofline fraction, ms per step), last in the JSON line so
+    that a truncated tail still holds every workload."""
+    def frac(d):
+        r = d.get("roofline") or d.get("gate_up_stage") or {}
+        return None if r.get("frac") is None else round(float(r["frac"]), 4)
+    s = {out["config"]["workload"] + f"_T{out['config']['T']}": {
+        "value": round(out["value"], 1), "unit": out["unit"], "gate_up_frac_of_hbm": frac(out),
+        "ms_per_step": round(out["ms_per_step"], 4), "e2e": round(out["e2e"]["value"], 1)}}
+    for k, d in out.get("extra", {}).items():
+        e = {"value": round(float(d["value"]), 3 if d.get("unit") == "ms" else 1), "unit": d.get("unit")}
+        f = frac(d)
+        if f is not None:
+            e["frac"] = f
+            e["of"] = ((d.get("roofline") or {}).get("peak_source")
+                       or (d.get("gate_up_stage") or {}).get("peak_source") or "")
+        if "ms_per_step" in d:
+            e["ms_per_step"] = round(float(d["ms_per_step"]), 4)
+        if "gate_up_hbm" in d:
+            e["gate_up_frac_of_hbm"] = round(float(d["gate_up_hbm"]["frac"]), 4)
+        s[k] = e
+    if out.get("cpu_baseline"):
+        c = out["cpu_baseline"]
+        s["cpu_oracle"] = {"value": round(c["value"], 3), "cores": c["cores"],
+                           "single_thread": round(c.get("single_thread", {}).get("value", 0.0), 4)}
+    return s
 
 
 def _time_steps(torch, fn, steps):
@@ -471,11 +503,11 @@ def _traced(torch, vq, fn, steps, n_events=6):
     return np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(n_events - 1)] for i in range(steps)])
 
 
-def measure_decode_layer(torch, vq, spec, T, dev, steps, warmup):
+def measure_decode_layer(torch, vq, spec, T, dev, steps, warmup, traffic_tag=None):
     """Another decode workload (its own layer, 16 rotating routing draws): step GB/s and the gate+up
     launch's fraction of the measured HBM bandwidth."""
     from tests.helpers import lib_module
-    mds = wl.layer_modules(spec, raw=False, row_words=lambda c, g: vq.packed_words(1, c // g.d, g.bits))
+    mds = wl.layer_modules(spec, raw=False, row_words=_row_words)
     per_expert = [_module_bytes(m) for m in mds]
     cb_bytes = sum(m.codebook.nbytes for m in mds)
     gu_cb = mds[0].codebook.nbytes + mds[1].codebook.nbytes
@@ -500,39 +532,56 @@ def measure_decode_layer(torch, vq, spec, T, dev, steps, warmup):
     ms = _time_steps(torch, fn, steps)
     stage = _traced(torch, vq, fn, steps).mean(axis=0)
     hbm, _, _, src = _peaks()
-    gu_ach = float(np.mean([gu_bytes[i % N_DRAWS] for i in range(steps)])) / (stage[1] * 1e-3) / 1e9
+    gu_avg = float(np.mean([gu_bytes[i % N_DRAWS] for i in range(steps)]))
+    gu_ach = gu_avg / (stage[1] * 1e-3) / 1e9
     out = {"workload": spec.name, "T": T, "value": sum(step_bytes[i % N_DRAWS] for i in range(steps)) / (ms * 1e-3) / 1e9,
            "unit": UNIT, "ms_per_step": ms / steps, "tokens_per_s": T * steps / (ms * 1e-3),
            "stage_ms": {"route": float(stage[0]), "gate_up_gemv": float(stage[1]), "swiglu": float(stage[2]),
                         "down_gemv": float(stage[3]), "combine": float(stage[4])},
            "gate_up_stage": {"achieved": gu_ach, "peak": hbm, "unit": "GB/s", "frac": gu_ach / hbm,
-                       "peak_source": f"{src} hbm_gbs"},
+                             "peak_source": f"{src} hbm_gbs", "bytes_per_launch": gu_avg,
+                             "traffic": _traffic_per_launch(traffic_tag) if traffic_tag else None},
            "geometry": f"gate {spec.gate.d}/{spec.gate.bits}b, up {spec.up.d}/{spec.up.bits}b, "
-                       f"down {spec.down.d}/{spec.down.bits}b (d / code bits)"}
+                       f"down {spec.down.d}/{spec.down.bits}b (d / code bits)", "launches_per_step": 5}
     del layer, xs, lgs, y, ws
     torch.cuda.empty_cache()
     return out
 
 
-def measure_decode_t1(torch, vq, layer, spec, per_expert, cb_bytes, dev, steps, warmup):
-    """Same layer, one token per step (latency-bound case), 16 rotating routing draws."""
-    draws = [wl.layer_inputs(spec, 1, 100 + i) for i in range(N_DRAWS)]
-    xs = [torch.from_numpy(x.view(np.int16)).to(dev) for x, _ in draws]
-    lgs = [torch.from_numpy(lg).to(dev) for _, lg in draws]
-    y = torch.empty((1, spec.hidden), dtype=torch.float32, device=dev)
-    ws = layer.workspace(1, spec.top_k, vq.VQ_MODE_DECODE, dev)
-    nbytes = []
-    for lg in lgs:
-        _, _, off, _ = vq.route(lg, spec.top_k)
-        touched = np.nonzero(np.diff(off.cpu().numpy()) > 0)[0]
-        nbytes.append(sum(float(p[touched].sum()) for p in per_expert) + cb_bytes + spec.hidden * 6 + spec.E * 4)
-    fn = lambda i: layer.decode(xs[i % N_DRAWS], lgs[i % N_DRAWS], spec.top_k, out=y, workspace=ws)
-    for i in range(warmup):
-        fn(i)
-    ms = _time_steps(torch, fn, steps)
-    tot = sum(nbytes[i % N_DRAWS] for i in range(steps))
-    return {"workload": spec.name, "T": 1, "value": tot / (ms * 1e-3) / 1e9, "unit": UNIT, "ms_per_step": ms / steps,
-            "tokens_per_s": steps / (ms * 1e-3), "launches_per_step": 5}
+def measure_gemv_single(torch, vq, dev, steps, warmup, copies=512):
+    """The single VQ GEMV (512 x 1024, d=2/K=256, one token). One call streams 276 KB, far less than the
+    launch latency covers, so it is measured in throughput mode: `copies` seeded modules (141 MB, more
+    than L2) called round-robin from one CUDA graph, bytes of the calls / device time."""
+    from tests.helpers import lib_module
+    s = wl.GEMV_D2K256
+    mods = []
+    for c in range(copies):
+        md = wl.module_data(1, s.rows, s.cols, s.geo, 0, (s.seed, 5000 + c), raw=False,
+                            row_words=_row_words(s.cols, s.geo))
+        mods.append(lib_module(md, device=dev))
+    x = torch.from_numpy(synth.activations(s.T, s.cols, synth.rng(s.seed, 1)).view(np.int16)).to(dev)
+    ys = [torch.empty((s.T, s.rows), dtype=torch.float32, device=dev) for _ in range(copies)]
+    nbytes = (s.rows * _row_words(s.cols, s.geo) * 4 + s.rows * (s.cols // 64) * 2 + (1 << s.geo.bits) * s.geo.d * 2
+              + s.T * s.cols * 2 + s.T * s.rows * 4)
+    stream = torch.cuda.Stream()
+    for c in range(min(copies, warmup * 8)):
+        vq.gemv(mods[c], 0, x, out=ys[c], stream=stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for c in range(copies):
+            vq.gemv(mods[c], 0, x, out=ys[c], stream=stream)
+    graph.replay()
+    torch.cuda.synchronize()
+    ms = _time_steps(torch, lambda i: graph.replay(), steps)
+    per_call_ms = ms / steps / copies
+    out = {"workload": s.name, "T": s.T, "value": nbytes / (per_call_ms * 1e-3) / 1e9, "unit": UNIT,
+           "ms_per_call": per_call_ms, "bytes_per_call": nbytes,
+           "mode": f"{copies} modules round-robin in one CUDA graph (141 MB > L2)",
+           "note": "launch-latency bound: one call streams 276 KB", "launches_per_step": copies}
+    del graph, mods, ys
+    torch.cuda.empty_cache()
+    return out
 
 
 def measure_prefill(torch, vq, dev, steps, warmup, small=False, ncu_mode=False, spec=None, T=None):
@@ -547,7 +596,7 @@ def measure_prefill(torch, vq, dev, steps, warmup, small=False, ncu_mode=False, 
     if small:
         spec = dataclasses.replace(spec, E=64, name=spec.name.replace("e256", "e64"))
         T = 1024
-    mds = wl.layer_modules(spec, raw=False, row_words=lambda c, g: vq.packed_words(1, c // g.d, g.bits))
+    mds = wl.layer_modules(spec, raw=False, row_words=_row_words)
     layer = vq.MoELayer(*[lib_module(m, device=dev) for m in mds])
     per_expert = [_module_bytes(m) for m in mds]
     draws = [wl.layer_inputs(spec, T, i) for i in range(2)]
@@ -603,7 +652,7 @@ def measure_prefill_chunked(torch, vq, dev, steps, warmup, T=8192, chunk=2048):
     workspace (vq_moe_prefill_chunked): TFLOP/s and the workspace it needs against one call's."""
     from tests.helpers import lib_module
     spec = wl.PREFILL_D4K512
-    mds = wl.layer_modules(spec, raw=False, row_words=lambda c, g: vq.packed_words(1, c // g.d, g.bits))
+    mds = wl.layer_modules(spec, raw=False, row_words=_row_words)
     layer = vq.MoELayer(*[lib_module(m, device=dev) for m in mds])
     del mds
     x, lg = wl.layer_inputs(spec, T, 300)
@@ -653,25 +702,39 @@ def measure_fit(torch, vq, dev, steps, warmup, rows=2048, cols=6144, d=4, K=512,
 
 
 def cpu_baseline(mds, draws, spec, T, per_expert, cb_bytes, budget_s=10.0):
-    """The oracle as it stands on a bounded sample: tokens of the first draw
-    until about budget_s seconds of CPU work."""
+    """The oracle as it stands on a bounded sample of the headline workload: tokens of the first draw
+    until about budget_s seconds of CPU work on all the host's cores, then one token on one core."""
     import oracle
     from tests.helpers import oracle_module
     oracle.build()
     oms = [oracle_module(m) for m in mds]
     x, lg = draws[0]
-    done, nbytes, t_used = 0, 0.0, 0.0
-    while done < T and t_used < budget_s:
-        tok = np.array([done])
-        ids, *_ = oracle.route(lg[tok], spec.top_k)
-        t0 = time.perf_counter()
-        oracle.moe(*oms, x, lg, spec.top_k, tokens=tok)
-        t_used += time.perf_counter() - t0
-        nbytes += float(sum(p[np.unique(ids)].sum() for p in per_expert) + cb_bytes + spec.hidden * 10 + spec.E * 4)
-        done += 1
-    return {"value": nbytes / t_used / 1e9, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{done} token(s) of the 8-token batch ({done * spec.top_k} expert passes), float64",
-            "seconds": t_used}
+    cores = oracle.num_threads()
+
+    def run(n_max, budget):
+        done, nbytes, t_used = 0, 0.0, 0.0
+        while done < n_max and t_used < budget:
+            tok = np.array([done % T])
+            ids, *_ = oracle.route(lg[tok], spec.top_k)
+            t0 = time.perf_counter()
+            oracle.moe(*oms, x, lg, spec.top_k, tokens=tok)
+            t_used += time.perf_counter() - t0
+            nbytes += _token_bytes(spec, per_expert, cb_bytes, ids)
+            done += 1
+        return done, nbytes, t_used
+
+    done, nbytes, t_used = run(T, budget_s)
+    oracle.set_num_threads(1)
+    try:
+        d1, b1, t1 = run(1, float("inf"))
+    finally:
+        oracle.set_num_threads(cores)
+    return {"value": nbytes / t_used / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{done} token(s) of the {T}-token batch ({done * spec.top_k} expert passes of all three "
+                      f"projections), float64, OpenMP over {cores} threads",
+            "seconds": t_used,
+            "single_thread": {"value": b1 / t1 / 1e9, "unit": UNIT, "cores": 1, "seconds": t1,
+                              "sample": "1 token (its experts, all three projections), float64, one thread"}}
 
 
 def main():

@@ -80,6 +80,8 @@ def _L():
         lib.vqo_moe.restype = I
         lib.vqo_moe.argtypes = [ctypes.POINTER(_Module)] * 3 + [I, I, P, P, I, I, I, P, I, P]
         lib.vqo_num_threads.restype = I
+        lib.vqo_set_num_threads.argtypes = [I]
+        lib.vqo_set_num_threads.restype = None
         _lib = lib
     return _lib
 
@@ -95,6 +97,11 @@ def _c(a, dtype):
 def num_threads() -> int:
     """OpenMP threads the oracle uses."""
     return _L().vqo_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    """OpenMP threads for the oracle's loops (the CPU baseline times one and all)."""
+    _L().vqo_set_num_threads(int(n))
 
 
 def f16_to_f64(bits) -> np.ndarray:

@@ -425,3 +425,15 @@ int vqo_num_threads(void)
     return 1;
 #endif
 }
+
+/* Sets the OpenMP threads of the oracle's loops (n >= 1); a timing knob for
+ * the CPU baseline, which reports the oracle on one thread and on all. */
+void vqo_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n >= 1)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

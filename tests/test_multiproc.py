@@ -57,3 +57,27 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     monkeypatch.setenv("WORLD_SIZE", "2")
     bench.run_reference(argparse.Namespace(steps=1, warmup=3, gpus=2))
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_loads_only_the_oracle():
+    # rank 0 of the reference arm on a small layer: one JSON line with the workload's config, and no
+    # product module or library in the process
+    import json
+    import subprocess
+    code = (
+        "import sys, argparse, dataclasses, json; sys.path.insert(0, %r)\n"
+        "import bench\n"
+        "from synth import workloads as wl\n"
+        "bench.MAIN_SPEC = dataclasses.replace(wl.DECODE_D2K256, E=16, hidden=512, inter=256, name='small')\n"
+        "bench.MAIN_T = 4\n"
+        "bench.run_reference(argparse.Namespace(steps=2, warmup=3, gpus=1))\n"
+        "assert 'vector_quantized_moe_b200' not in sys.modules\n"
+        "maps = open('/proc/self/maps').read()\n"
+        "assert 'libvqmoe' not in maps and 'libvqoracle' in maps\n" % ROOT)
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["config"]["workload"] == "small" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle"
+
