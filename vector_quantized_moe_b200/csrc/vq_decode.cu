@@ -29,13 +29,25 @@
 namespace vq {
 namespace {
 
+// Words that hold QB bits starting at bit (j * QB) % 32 of a word, for the
+// worst j (every lane quarter j of a row starts at bit j * QB).
+__host__ __device__ constexpr int words_spanned(int qb)
+{
+    int w = 0;
+    for (int j = 0; j < 32; ++j) {
+        const int n = ((j * qb) % 32 + qb + 31) / 32;
+        w = n > w ? n : w;
+    }
+    return w;
+}
+
 template <int D, int BITS>
 struct Geo {
     static constexpr int CODES = 16 / D;               // codes of one lane in one group
     static constexpr int QB = CODES * BITS;            // their bits
     static constexpr bool ALIGNED = (QB % 32) == 0;    // their bit range starts on a word
     static constexpr int NW = (QB + 31) / 32;          // words once shifted down to bit 0
-    static constexpr int LW = ALIGNED ? NW : NW + 1;   // words loaded from the row
+    static constexpr int LW = words_spanned(QB);       // words loaded from the row (at most NW + 1)
     static constexpr int EW = D <= 2 ? 1 : D / 2;      // shared-memory words per codebook entry
     static constexpr uint32_t MASK = (1u << BITS) - 1u;
     static constexpr int LOG_REP = codebook_log_rep(D, BITS);   // replicas per entry (log2)
@@ -79,7 +91,7 @@ __device__ __forceinline__ void extract_codes(const uint32_t (&w)[Geo<D, BITS>::
     uint32_t n[G::NW];
 #pragma unroll
     for (int i = 0; i < G::NW; ++i)
-        n[i] = G::ALIGNED ? w[i] : __funnelshift_r(w[i], w[i + (G::ALIGNED ? 0 : 1)], o);
+        n[i] = G::ALIGNED ? w[i] : __funnelshift_r(w[i], (!G::ALIGNED && i + 1 < G::LW) ? w[i + 1] : 0u, o);
 #pragma unroll
     for (int k = 0; k < G::CODES; ++k) {
         const int p = k * BITS, wi = p >> 5, sh = p & 31;
@@ -103,7 +115,7 @@ __device__ __forceinline__ void code_offsets(const uint32_t (&w)[Geo<D, BITS>::L
     uint32_t n[G::NW];
 #pragma unroll
     for (int i = 0; i < G::NW; ++i)
-        n[i] = G::ALIGNED ? w[i] : __funnelshift_r(w[i], w[i + (G::ALIGNED ? 0 : 1)], o);
+        n[i] = G::ALIGNED ? w[i] : __funnelshift_r(w[i], (!G::ALIGNED && i + 1 < G::LW) ? w[i + 1] : 0u, o);
 #pragma unroll
     for (int k = 0; k < G::CODES; ++k) {
         const int p = k * BITS, wi = p >> 5, sh = p & 31;
