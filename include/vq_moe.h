@@ -61,7 +61,13 @@ enum { VQ_F32 = 0, VQ_BF16 = 1 };
  *
  * Expert e's weight matrix is W_e [rows, cols] with
  *   W_e[r, c] = fp32(codebook[code_e(r, c / d)][c % d]) * fp32(scale_e[r, c / 64])
- * where code_e(r, j) is the j-th b-bit code of row r.
+ *               (+ fp32(bias_e[r, c / 64]) for a module with biases)
+ * where code_e(r, j) is the j-th b-bit code of row r. The bias is the
+ * optional affine arm: the cards' fallback format "affine 3-bit, group 64"
+ * (Qwen3.5-397B-A17B-VQ-2.4bpw card, Changelog 2026-09-20) is stated without
+ * its formula; this library reads it as the group-wise affine form
+ * w = s * q + b with an fp16 scale and an fp16 bias per (row, 64 weights),
+ * which is d = 1 with the codebook C[q] = q plus the bias.
  *
  * Requirements: d in {1, 2, 4, 8}; cols a multiple of 64 and of 32*d (whole
  * 32-code blocks and whole scale groups); (d, bits) one of the implemented
@@ -93,6 +99,9 @@ typedef struct vq_module {
      * may read); required when live_bitmap is set, ignored (E * rows)
      * otherwise. */
     int64_t live_rows;
+    /* device, 2-byte aligned, or NULL (no bias): fp16 biases [live rows,
+     * cols / 64], the same layout as `scales`. */
+    const uint16_t *biases;
 } vq_module;
 
 /* A SwiGLU MoE layer: y = sum_j w_j * down_e( silu(gate_e x) * up_e x ).

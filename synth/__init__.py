@@ -23,7 +23,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = [
-    "rng", "bf16_bits", "f16_bits", "codebook", "scales", "raw_codes",
+    "rng", "bf16_bits", "f16_bits", "codebook", "scales", "biases", "raw_codes",
     "live_bitmap", "random_words", "activations", "activations_scaled", "logits_normal", "logits_zipf",
     "weights", "fit_draw",
 ]
@@ -58,6 +58,11 @@ def codebook(K: int, d: int, g: np.random.Generator, sigma: float = 0.02) -> np.
 def scales(n_rows: int, n_groups: int, g: np.random.Generator, lo: float = 0.5, hi: float = 2.0) -> np.ndarray:
     """fp16 group scales [n_rows, n_groups] drawn U(lo, hi)."""
     return f16_bits(g.uniform(lo, hi, size=(n_rows, n_groups)).astype(np.float32))
+
+
+def biases(n_rows: int, n_groups: int, g: np.random.Generator, sigma: float = 0.02) -> np.ndarray:
+    """fp16 group biases [n_rows, n_groups] drawn N(0, sigma) (the affine arm's offsets)."""
+    return f16_bits(g.normal(0.0, sigma, size=(n_rows, n_groups)).astype(np.float32))
 
 
 def raw_codes(shape, bits: int, g: np.random.Generator) -> np.ndarray:

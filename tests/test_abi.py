@@ -81,12 +81,12 @@ def _null_module(**kw):
              live_rank=None)
     m.update(kw)
     return vq.vq_module(m["E"], m["rows"], m["cols"], m["d"], m["bits"], m["codes"], m["scales"], m["codebook"],
-                        m["live_bitmap"], m["live_rank"], m.get("live_rows", 0))
+                        m["live_bitmap"], m["live_rank"], m.get("live_rows", 0), m.get("biases"))
 
 
 @pytest.mark.parametrize("kw,status", [
     (dict(codes=None), 1), (dict(cols=100), 1), (dict(d=3), 1), (dict(bits=7), 3), (dict(codes=264), 2),
-    (dict(live_bitmap=4096), 1), (dict(E=0), 1),
+    (dict(live_bitmap=4096), 1), (dict(E=0), 1), (dict(biases=4097), 2),
 ])
 def test_argument_errors_before_launch(kw, status):
     # fake (never dereferenced) pointers: validation fails before any CUDA call

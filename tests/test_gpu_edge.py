@@ -9,6 +9,7 @@ import torch
 import oracle
 import synth
 from helpers import assert_close, lib_module, oracle_module, small_module
+from synth import workloads as wl
 
 import vector_quantized_moe_b200 as vq
 
@@ -106,3 +107,20 @@ def test_decode_step_replays_from_a_cuda_graph():
         torch.cuda.synchronize()
         assert torch.equal(outs[i], want)
     del graph
+
+
+@pytest.mark.parametrize("T", [256, 2048])
+def test_skipzero_layer_decode_bitwise_repeatable_from_the_first_call(T):
+    # the full-size skipzero + mixed-geometry layer (live bitmaps, d=2/10-bit gate/up, d=8/12-bit down): the
+    # first call on a fresh workspace and the calls after it give the same bits
+    from helpers import row_words_fn
+    mds = wl.layer_modules(wl.SKIPZERO_MIXED, raw=False, row_words=row_words_fn())
+    layer = vq.MoELayer(*[lib_module(m) for m in mds])
+    del mds
+    x, lg = wl.layer_inputs(wl.SKIPZERO_MIXED, T)
+    xt, lt = torch.from_numpy(x.view(np.int16)).cuda(), torch.from_numpy(lg).cuda()
+    outs = [layer.decode(xt, lt, wl.SKIPZERO_MIXED.top_k).cpu().numpy().view(np.uint32).copy() for _ in range(4)]
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0])
+    del layer
+    torch.cuda.empty_cache()

@@ -36,7 +36,8 @@ class vq_module(ctypes.Structure):
     _fields_ = [("E", ctypes.c_int32), ("rows", ctypes.c_int32), ("cols", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("bits", ctypes.c_int32),
                 ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("codebook", ctypes.c_void_p),
-                ("live_bitmap", ctypes.c_void_p), ("live_rank", ctypes.c_void_p), ("live_rows", ctypes.c_int64)]
+                ("live_bitmap", ctypes.c_void_p), ("live_rank", ctypes.c_void_p), ("live_rows", ctypes.c_int64),
+                ("biases", ctypes.c_void_p)]
 
 
 class vq_moe_layer(ctypes.Structure):
@@ -173,15 +174,19 @@ def _ptr(t) -> Optional[int]:
 class Module:
     """One VQ module on the device (vq_module). Tensors are kept alive here."""
 
-    def __init__(self, E, rows, cols, d, bits, codes, scales, codebook, live_bitmap=None, live_rank_t=None):
+    def __init__(self, E, rows, cols, d, bits, codes, scales, codebook, live_bitmap=None, live_rank_t=None,
+                 biases=None):
         self.E, self.rows, self.cols, self.d, self.bits = E, rows, cols, d, bits
         self.codes, self.scales, self.codebook = codes, scales, codebook
         self.live_bitmap, self.live_rank = live_bitmap, live_rank_t
+        self.biases = biases
 
     @classmethod
-    def from_host(cls, E, rows, cols, d, bits, words, scales, codebook, live_bitmap=None, device="cuda"):
+    def from_host(cls, E, rows, cols, d, bits, words, scales, codebook, live_bitmap=None, device="cuda",
+                  biases=None):
         """Upload packed words [live rows, row_words], fp16 scale bits [live rows, cols/64],
-        fp16 codebook bits [2^bits, d] and an optional live bitmap [E, ceil(rows/32)]."""
+        fp16 codebook bits [2^bits, d], an optional live bitmap [E, ceil(rows/32)] and optional
+        fp16 bias bits [live rows, cols/64] (the affine arm)."""
         torch = _torch()
         up = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a).view(dt)).to(device)
         bm = rk = None
@@ -189,12 +194,12 @@ class Module:
             bm = up(live_bitmap.astype(np.uint32), np.int32)
             rk = up(live_rank(live_bitmap, rows), np.int32)
         return cls(E, rows, cols, d, bits, up(words.astype(np.uint32), np.int32), up(scales, np.int16),
-                   up(codebook, np.int16), bm, rk)
+                   up(codebook, np.int16), bm, rk, None if biases is None else up(biases, np.int16))
 
     def struct(self) -> vq_module:
         return vq_module(self.E, self.rows, self.cols, self.d, self.bits, _ptr(self.codes), _ptr(self.scales),
                          _ptr(self.codebook), _ptr(self.live_bitmap), _ptr(self.live_rank),
-                         int(self.scales.shape[0]))
+                         int(self.scales.shape[0]), _ptr(self.biases))
 
 
 def unpack(m: Module, expert: int, stream=None):

@@ -55,7 +55,7 @@ vq_status check_module(const vq_module *m)
         return VQ_ERR_ARG;
     if (!geometry_ok(m->d, m->bits))
         return VQ_ERR_UNSUPPORTED;
-    if (!aligned(m->codes, 16) || !aligned(m->codebook, 16) || !aligned(m->scales, 2))
+    if (!aligned(m->codes, 16) || !aligned(m->codebook, 16) || !aligned(m->scales, 2) || !aligned(m->biases, 2))
         return VQ_ERR_ALIGN;
     if ((m->live_bitmap && !aligned(m->live_bitmap, 4)) || (m->live_rank && !aligned(m->live_rank, 4)))
         return VQ_ERR_ALIGN;
@@ -107,7 +107,8 @@ DecodePlan plan_decode(const vq_moe_layer *L, int T, int k)
     const double n_exp = p.E * (1.0 - std::pow(1.0 - (double)k / p.E, (double)T));
     const ModDev gu[2] = {make_moddev(L->gate), make_moddev(L->up)};
     const ModDev dn = make_moddev(L->down);
-    p.gu_shared = gu[0].d == gu[1].d && gu[0].bits == gu[1].bits && gu[0].rep == gu[1].rep;
+    p.gu_shared = gu[0].d == gu[1].d && gu[0].bits == gu[1].bits && gu[0].rep == gu[1].rep &&
+                  (gu[0].biases == nullptr) == (gu[1].biases == nullptr);
     if (p.gu_shared) {
         p.pg = p.pu = gemv_plan(gu, 2, n_exp);
     } else {
@@ -139,6 +140,7 @@ ModDev make_moddev(const vq_module &m)
     ModDev d{};
     d.codes = m.codes;
     d.scales = m.scales;
+    d.biases = m.biases;
     d.codebook = m.codebook;
     d.bitmap = m.live_bitmap;
     d.rank = m.live_rank;

@@ -265,6 +265,9 @@ struct GroupLoads {
     uint16_t sv[4];
 };
 
+// fp16 1.0 in both halves: an A fragment of ones makes the MMA sum a group's activations.
+constexpr uint32_t F16X2_ONES = 0x3C003C00u;
+
 template <int D, int BITS, int PD>
 __global__ void __launch_bounds__(GEMV_THREADS, 2) vq_grouped_gemv_kernel(const __grid_constant__ GemvArgs a)
 {
@@ -396,6 +399,27 @@ __global__ void __launch_bounds__(GEMV_THREADS, 2) vq_grouped_gemv_kernel(const 
                         }
                     }
                 }
+                // affine arm: b * (the group's activation sum), the sum from one MMA against ones
+                float xs[4] = {0.f, 0.f, 0.f, 0.f};
+                if (m.biases) {
+                    const uint32_t ones[4] = {F16X2_ONES, F16X2_ONES, F16X2_ONES, F16X2_ONES};
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        mma_16816(xs, ones, bw[2 * s], bw[2 * s + 1]);
+                    // (not prefetched with the codes: only biased modules pay for these loads)
+                    float bv[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        bv[i] = prow[i] >= 0 ? f16_to_f32(ldg_u16(m.biases + (long)prow[i] * m.ngroups + grp)) : 0.f;
+#pragma unroll
+                    for (int rt = 0; rt < 2; ++rt) {
+                        const float blo = bv[2 * rt], bhi = bv[2 * rt + 1];
+                        acc[rt][0] = fmaf(blo * xs[0], f0, acc[rt][0]);
+                        acc[rt][1] = fmaf(blo * xs[1], f1, acc[rt][1]);
+                        acc[rt][2] = fmaf(bhi * xs[0], f0, acc[rt][2]);
+                        acc[rt][3] = fmaf(bhi * xs[1], f1, acc[rt][3]);
+                    }
+                }
 #pragma unroll
                 for (int rt = 0; rt < 2; ++rt) {
                     const float slo = f16_to_f32(L.sv[2 * rt]);
@@ -516,10 +540,11 @@ struct TGeo {
 struct GemvTmaArgs {
     CUtensorMap tmap[2];      // codes: u32 [live rows, row_words], box {SRB/4, 256}
     CUtensorMap tmap_sc[2];   // scales: fp16 [live rows, ngroups], box {8, 256}
+    CUtensorMap tmap_bi[2];   // biases (affine arm), as the scales
     CUtensorMap tmap_act;     // activations: 16-bit [act rows, cols], box {ACW, 1}
     GemvArgs g;
     int ns;
-    uint32_t stage_bytes, off_sc, off_act;   // stage layout: codes | scales | activations
+    uint32_t stage_bytes, off_sc, off_bi, off_act;   // stage layout: codes | scales | [biases] | activations
     uint32_t off_stage, off_xchg, off_bar;
     int *err;
 };
@@ -594,8 +619,10 @@ __device__ __forceinline__ TgItem tg_item(const GemvArgs &a, long item, int nrb,
 }
 
 // ABF16: activations in bf16 (else fp16). DENSE: no module of the launch has a
-// live bitmap.
-template <int D, int BITS, bool ABF16, bool DENSE>
+// live bitmap. BIAS: the modules carry per-group biases (the affine arm): each
+// group adds b * (its activation sum), the sum from one more MMA per k16 step
+// against an A fragment of ones.
+template <int D, int BITS, bool ABF16, bool DENSE, bool BIAS>
 __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid_constant__ GemvTmaArgs A)
 {
     using G = Geo<D, BITS>;
@@ -679,7 +706,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                         const int q = it.q0 + i;
                         arow[i] = a.act_by_slot ? q : (a.perm ? a.perm[q] / a.top_k : q);
                     }
-                    tx = stage_bytes_codes + (uint32_t)TG_ROWS * 16 + (uint32_t)it.n * TG::ACOLS * 2;
+                    tx = stage_bytes_codes + (uint32_t)TG_ROWS * 16 * (BIAS ? 2 : 1) + (uint32_t)it.n * TG::ACOLS * 2;
                 }
                 if (!(ok = mbar_wait(&empty[slot], ph ^ 1, abort_flag, A.err, 11, a.wait_limit)))
                     break;
@@ -688,6 +715,8 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                 const int g0 = j * TG::CG;
                 tma_load_2d(sb, &A.tmap[mi], g0 * TG::GB / 32, prow0, &full[slot]);
                 tma_load_2d(sb + A.off_sc, &A.tmap_sc[mi], g0 & ~7, prow0, &full[slot]);
+                if constexpr (BIAS)
+                    tma_load_2d(sb + A.off_bi, &A.tmap_bi[mi], g0 & ~7, prow0, &full[slot]);
                 for (int i = 0; i < it.n; ++i)
                     for (int c = 0; c < TG::ACOLS; c += TG::ACW)
                         tma_load_2d(sb + A.off_act + (size_t)i * TG::ACOLS * 2 + c * 2, &A.tmap_act, g0 * 64 + c,
@@ -698,11 +727,13 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                     ph ^= 1;
                 }
             }
-            // the copies issued have landed before this thread leaves (the last use of each slot):
-            // after a give-up the consumers may have left without waiting for them
-            for (uint32_t s = 0; s < (uint32_t)A.ns && s < k; ++s) {
-                const uint32_t kk = k - 1 - s;
-                mbar_drain(&full[kk % A.ns], (kk / A.ns) & 1);
+            // after a give-up, the copies issued land before this thread leaves (the last use of each
+            // slot). A normal end needs no wait: the consumers wait for every stage they read.
+            if (!ok) {
+                for (uint32_t s = 0; s < (uint32_t)A.ns && s < k; ++s) {
+                    const uint32_t kk = k - 1 - s;
+                    mbar_drain(&full[kk % A.ns], (kk / A.ns) & 1);
+                }
             }
         }
         return;
@@ -741,7 +772,8 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
     float acc[TG_RT][4];
     long item = u0 / spp;
     int j = (int)(u0 % spp);
-    for (long u = u0; u < u1 && ok; ++u, j = (j + 1 == spp) ? 0 : j + 1, item += (j == 0)) {
+    long u = u0;
+    for (; u < u1 && ok; ++u, j = (j + 1 == spp) ? 0 : j + 1, item += (j == 0)) {
         if (u == u0 || j == 0) {
             it = tg_item(a, item, nrb, cta_mods, FAST);
             const ModDev &m = it.mi == 0 ? a.mod[0] : a.mod[1];
@@ -800,6 +832,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
             float sv[GP][TG_RL];
             uint32_t bw[GP][8];
             float fa[GP][2];   // bf16 activations: inverse scales of the fragment's token columns
+            float bvv[BIAS ? TG_RL : 1];   // biases of the lane's rows (GP == 1 with them)
 #pragma unroll
             for (int uu = 0; uu < GP; ++uu) {
                 const int gq = half * TG::HG + gh + uu;   // group within the stage
@@ -859,6 +892,13 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
 #pragma unroll
                     for (int i = 0; i < TG_RL; ++i)
                         sv[uu][i] = f16_to_f32(*reinterpret_cast<const uint16_t *>(ssc + soff[i] + 2 * gq));
+                }
+                if constexpr (BIAS) {
+                    const uint8_t *bb = sb + (A.off_bi - A.off_sc) + 2 * ((j * TG::CG) & 7) + 2 * gq;
+#pragma unroll
+                    for (int i = 0; i < TG_RL; ++i)
+                        bvv[i] = f16_to_f32(*reinterpret_cast<const uint16_t *>(
+                            bb + (DENSE ? soff[0] + i * 8 * 16 : soff[i])));
                 }
                 const uint4 v0 = *reinterpret_cast<const uint4 *>(sb + aoff + gq * 128);
                 const uint4 v1 = *reinterpret_cast<const uint4 *>(sb + aoff + gq * 128 + 16);
@@ -920,6 +960,23 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                         }
                         mma_16816(tmp[uu][rt], Aw, bw[uu][2 * s], bw[uu][2 * s + 1]);
                     }
+                }
+            }
+            if constexpr (BIAS) {
+                // b * (the group's activation sum of tokens 2t, 2t + 1), the sums from an MMA against ones
+                static_assert(GP == 1, "biases with one group per warp step");
+                float xs[4] = {0.f, 0.f, 0.f, 0.f};
+                const uint32_t ones[4] = {F16X2_ONES, F16X2_ONES, F16X2_ONES, F16X2_ONES};
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_16816(xs, ones, bw[0][2 * s], bw[0][2 * s + 1]);
+                const float x0 = ABF16 ? xs[0] * fa[0][0] : xs[0], x1 = ABF16 ? xs[1] * fa[0][1] : xs[1];
+#pragma unroll
+                for (int rt = 0; rt < TG_RT; ++rt) {
+                    acc[rt][0] = fmaf(bvv[2 * rt], x0, acc[rt][0]);
+                    acc[rt][1] = fmaf(bvv[2 * rt], x1, acc[rt][1]);
+                    acc[rt][2] = fmaf(bvv[2 * rt + 1], x0, acc[rt][2]);
+                    acc[rt][3] = fmaf(bvv[2 * rt + 1], x1, acc[rt][3]);
                 }
             }
 #pragma unroll
@@ -998,6 +1055,18 @@ __global__ void __launch_bounds__(TG_THREADS, 1) vq_gemv_tma_kernel(const __grid
                         store_out(out, a.out_dtype, (long)sl * a.out_slice_stride + o, 0.f);
                 }
             }
+    }
+    if (!ok) {
+        // a give-up: the producer may have copied up to ns stages past the one this warp stopped at and
+        // left already; they land before the CTA can exit. A stage never issued gives up after a short
+        // bound (the producer, if still running, drains its own copies when it sees the abort).
+        for (int s = 0; s < A.ns && u + s < u1; ++s) {
+            const uint32_t sl = (slot + (uint32_t)s) % (uint32_t)A.ns;
+            const uint32_t p = (slot + (uint32_t)s) >= (uint32_t)A.ns ? (ph ^ 1u) : ph;
+            for (uint32_t i = 0; i < (1u << 14); ++i)
+                if (mbar_try_wait(&full[sl], p))
+                    break;
+        }
     }
 }
 
@@ -1253,9 +1322,11 @@ cudaError_t gemv_dispatch(const GemvArgs &a, cudaStream_t s, bool pdl)
 
 struct TgPlan {
     int ns;
-    uint32_t stage, off_sc, off_act, off_stage, off_xchg, off_bar, total;
+    uint32_t stage, off_sc, off_bi, off_act, off_stage, off_xchg, off_bar, total;
 };
 
+// Shared-memory layout of the TMA kernel for a module's geometry (with the bias
+// box in each stage when the module has biases).
 TgPlan tg_plan(const ModDev &m)
 {
     TgPlan p{};
@@ -1263,7 +1334,8 @@ TgPlan tg_plan(const ModDev &m)
     const int cg = tg_stage_groups(m.d, m.bits);
     const uint32_t codes = (uint32_t)TG_ROWS * (uint32_t)(cg * (64 / m.d) * m.bits / 8);
     p.off_sc = codes;
-    p.off_act = codes + (uint32_t)TG_ROWS * 16;
+    p.off_bi = codes + (uint32_t)TG_ROWS * 16;
+    p.off_act = p.off_bi + (m.biases ? (uint32_t)TG_ROWS * 16 : 0u);
     p.stage = (uint32_t)align_up(p.off_act + (uint32_t)VQ_PASS_TOKENS * cg * 64 * 2, 1024);
     const uint32_t limit = 227 * 1024 - 1024;   // opt-in maximum less the alignment slack
     const uint32_t fixed = cb + TG_XCHG_BYTES + TG_BAR_BYTES;
@@ -1297,10 +1369,14 @@ cudaError_t gemv_tma_dispatch(const GemvArgs &a, cudaStream_t s, bool pdl)
                         TG::SWZ ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
     }
+    const bool bias = a.mod[0].biases != nullptr;   // the modules of a launch agree (plan_decode)
     for (int i = 0; i < a.nmod; ++i) {
         const ModDev &m = a.mod[i];
         if (!tma_map_2d(&A.tmap_sc[i], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, m.scales, (uint64_t)m.ngroups,
                         (uint64_t)m.live_rows, 8, (uint32_t)TG_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
+        if (bias && !tma_map_2d(&A.tmap_bi[i], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, m.biases, (uint64_t)m.ngroups,
+                                (uint64_t)m.live_rows, 8, (uint32_t)TG_ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
             return cudaErrorInvalidValue;
     }
     if (!tma_map_2d(&A.tmap_act, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.act, (uint64_t)a.mod[0].cols,
@@ -1309,11 +1385,13 @@ cudaError_t gemv_tma_dispatch(const GemvArgs &a, cudaStream_t s, bool pdl)
     if (a.nmod == 1) {
         A.tmap[1] = A.tmap[0];
         A.tmap_sc[1] = A.tmap_sc[0];
+        A.tmap_bi[1] = A.tmap_bi[0];
     }
     const TgPlan p = tg_plan(a.mod[0]);
     A.ns = p.ns;
     A.stage_bytes = p.stage;
     A.off_sc = p.off_sc;
+    A.off_bi = p.off_bi;
     A.off_act = p.off_act;
     A.off_stage = p.off_stage;
     A.off_xchg = p.off_xchg;
@@ -1322,8 +1400,13 @@ cudaError_t gemv_tma_dispatch(const GemvArgs &a, cudaStream_t s, bool pdl)
     bool dense = true;
     for (int i = 0; i < a.nmod; ++i)
         dense = dense && !a.mod[i].bitmap;
-    auto k = a.act_bf16 ? (dense ? vq_gemv_tma_kernel<D, BITS, true, true> : vq_gemv_tma_kernel<D, BITS, true, false>)
-                        : (dense ? vq_gemv_tma_kernel<D, BITS, false, true> : vq_gemv_tma_kernel<D, BITS, false, false>);
+    using KFn = void (*)(const GemvTmaArgs);
+    const KFn kernels[2][2][2] = {
+        {{vq_gemv_tma_kernel<D, BITS, false, false, false>, vq_gemv_tma_kernel<D, BITS, false, false, true>},
+         {vq_gemv_tma_kernel<D, BITS, false, true, false>, vq_gemv_tma_kernel<D, BITS, false, true, true>}},
+        {{vq_gemv_tma_kernel<D, BITS, true, false, false>, vq_gemv_tma_kernel<D, BITS, true, false, true>},
+         {vq_gemv_tma_kernel<D, BITS, true, true, false>, vq_gemv_tma_kernel<D, BITS, true, true, true>}}};
+    const KFn k = kernels[a.act_bf16 ? 1 : 0][dense ? 1 : 0][bias ? 1 : 0];
     // the layout of every module of a geometry is the same, so its size is fixed per kernel
     cudaError_t err = set_smem_limit_once((const void *)k, (int)p.total);
     if (err != cudaSuccess)

@@ -38,6 +38,7 @@ __host__ __device__ constexpr int codebook_log_rep(int d, int bits)
 struct ModDev {
     const uint32_t *codes;
     const uint16_t *scales;
+    const uint16_t *biases;   // NULL: none
     const uint16_t *codebook;
     const uint32_t *bitmap;
     const uint32_t *rank;

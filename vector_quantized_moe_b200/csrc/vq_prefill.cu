@@ -118,9 +118,12 @@ struct PrefillArgs {
     uint32_t wait_limit;      // polls of a bounded wait before it gives up
 };
 
-__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b)
+// a * b + c on fp16 pairs, one rounding to nearest even: the weight pair
+// C[q] * s + bias (bias 0 without the affine arm).
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c)
 {
-    __half2 r = __hmul2(*reinterpret_cast<__half2 *>(&a), *reinterpret_cast<__half2 *>(&b));
+    __half2 r = __hfma2(*reinterpret_cast<__half2 *>(&a), *reinterpret_cast<__half2 *>(&b),
+                        *reinterpret_cast<__half2 *>(&c));
     return *reinterpret_cast<uint32_t *>(&r);
 }
 
@@ -166,12 +169,13 @@ __device__ __forceinline__ uint32_t entry_off(const uint32_t (&w)[NW], int pos, 
 
 // One row of the 128 x 64 fp16 weight tile for k-step JJ of a code chunk:
 // 64 weights = 64/D codes read from the chunk row `crow` in shared memory,
-// each a codebook entry (the lane's replica) times the row's scale (fp16
-// product, rounded to nearest), as 32 words o[c] = weights (2c, 2c+1), the
-// layout of one tensor-memory lane of the MMA's A operand.
+// each a codebook entry (the lane's replica) times the row's scale plus the
+// row's bias (one fp16 fused multiply-add, rounded to nearest; the bias is 0
+// without the affine arm), as 32 words o[c] = weights (2c, 2c+1), the layout
+// of one tensor-memory lane of the MMA's A operand.
 template <int D, int BITS, int L, int JJ>
 __device__ __forceinline__ void dequant_step(const uint8_t *crow, const char *cb, uint32_t rep_off, uint32_t s2,
-                                             bool live, uint32_t (&o)[32])
+                                             uint32_t b2, bool live, uint32_t (&o)[32])
 {
     using W = Win<D, BITS, JJ>;
     constexpr int NC = 64 / D;
@@ -192,28 +196,28 @@ __device__ __forceinline__ void dequant_step(const uint8_t *crow, const char *cb
                                ((uint32_t)*reinterpret_cast<const uint16_t *>(
                                     cb + entry_off<BITS, L>(w, W::BASE + (c + 1) * BITS, rep_off))
                                 << 16);
-            o[c >> 1] = hmul2(v, s2);
+            o[c >> 1] = hfma2(v, s2, b2);
         }
     } else if constexpr (D == 2) {
 #pragma unroll
         for (int c = 0; c < NC; ++c)
-            o[c] = hmul2(*reinterpret_cast<const uint32_t *>(cb + entry_off<BITS, L>(w, W::BASE + c * BITS, rep_off)),
-                         s2);
+            o[c] = hfma2(*reinterpret_cast<const uint32_t *>(cb + entry_off<BITS, L>(w, W::BASE + c * BITS, rep_off)),
+                         s2, b2);
     } else if constexpr (D == 4) {
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
             const uint2 v = *reinterpret_cast<const uint2 *>(cb + entry_off<BITS, L>(w, W::BASE + c * BITS, rep_off));
-            o[2 * c] = hmul2(v.x, s2);
-            o[2 * c + 1] = hmul2(v.y, s2);
+            o[2 * c] = hfma2(v.x, s2, b2);
+            o[2 * c + 1] = hfma2(v.y, s2, b2);
         }
     } else {
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
             const uint4 v = *reinterpret_cast<const uint4 *>(cb + entry_off<BITS, L>(w, W::BASE + c * BITS, rep_off));
-            o[4 * c] = hmul2(v.x, s2);
-            o[4 * c + 1] = hmul2(v.y, s2);
-            o[4 * c + 2] = hmul2(v.z, s2);
-            o[4 * c + 3] = hmul2(v.w, s2);
+            o[4 * c] = hfma2(v.x, s2, b2);
+            o[4 * c + 1] = hfma2(v.y, s2, b2);
+            o[4 * c + 2] = hfma2(v.z, s2, b2);
+            o[4 * c + 3] = hfma2(v.w, s2, b2);
         }
     }
     if (!live) {
@@ -493,6 +497,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                         sc = prow[m] >= 0 ? ldg_u16(a.mod[m].scales + prow[m] * a.mod[m].ngroups + c * P::CH + j) : 0u;
                     return sc | (sc << 16);
                 };
+                // the row's fp16 bias of k-step j (the affine arm), as a half2 pair; 0 without
+                auto bfetch = [&](int m, int j) {
+                    const uint16_t *bi = a.mod[m].biases;
+                    const uint32_t b = (bi && prow[m] >= 0) ? ldg_u16(bi + prow[m] * a.mod[m].ngroups + c * P::CH + j) : 0u;
+                    return b | (b << 16);
+                };
                 auto step = [&](auto jj_c) {
                     constexpr int JJ = decltype(jj_c)::value;
                     if (!ok)
@@ -503,11 +513,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                         // stage, stored with one instruction); the wait for the stage's previous
                         // MMA overlaps the decode
                         uint32_t o[32 * NMOD];
-                        dequant_step<D, BITS, P::L, JJ>(crow[0], sm_cb, rep_off, sfetch(0, JJ), lrow[0] >= 0,
-                                                        *reinterpret_cast<uint32_t(*)[32]>(o));
+                        dequant_step<D, BITS, P::L, JJ>(crow[0], sm_cb, rep_off, sfetch(0, JJ), bfetch(0, JJ),
+                                                        lrow[0] >= 0, *reinterpret_cast<uint32_t(*)[32]>(o));
                         if constexpr (NMOD == 2)
                             dequant_step<D, BITS, P::L, JJ>(crow[1], sm_cb + cb_bytes, rep_off, sfetch(1, JJ),
-                                                            lrow[1] >= 0, *reinterpret_cast<uint32_t(*)[32]>(o + 32));
+                                                            bfetch(1, JJ), lrow[1] >= 0,
+                                                            *reinterpret_cast<uint32_t(*)[32]>(o + 32));
                         if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag, a.err, 7, a.wait_limit)))
                             return;
                         tc_fence_after();   // the stage's previous MMA has read it
