@@ -222,9 +222,13 @@ static void live_rows(const vqo_module *m, int e, long *idx)
 }
 
 /* Dequantise expert e of a module: W[r, c] = C[code(r, c/d)][c % d] * s[r, c/64]
- * (+ b[r, c/64] for a module with biases: the affine form s * q + b of the
- * "affine 3-bit, group 64" modules, Qwen3.5-397B-A17B-VQ-2.4bpw "2026-09-20
- * correction", with the identity codebook C[q] = q); dead rows are all zero.
+ * (+ b[r, c/64] for a module with biases); dead rows are all zero. The biases
+ * carry a reading, not a formula from the pages: the Qwen3.5-397B-A17B-VQ-2.4bpw
+ * card's "2026-09-20 correction" names a fallback format "affine 3-bit, group
+ * 64" (three layers had fallen through to it before they were refitted as VQ)
+ * and prints no formula; the reading is the group-wise affine form
+ * w = s * q + b, an fp16 scale and an fp16 bias per (row, 64 weights), which
+ * is d = 1 with the identity codebook C[q] = q plus the bias.
  * W is [rows, cols] row-major. */
 void vqo_dequant(const vqo_module *m, int e, double *W)
 {

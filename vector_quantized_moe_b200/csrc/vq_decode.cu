@@ -535,6 +535,11 @@ struct TGeo {
     static constexpr int SRB = CG * GB / 8;         // bytes per row per stage
     static constexpr int ACOLS = CG * 64;           // activation columns per stage
     static constexpr int ACW = ACOLS < 256 ? ACOLS : 256;   // columns per activation box
+    // a stage holds one 16-byte scale (and bias) box row per weight row: at most 8 groups
+    static_assert(CG <= 8, "a stage's groups fit one 8-group scale box row");
+    // the paired scale loads of a half read 2 * HG bytes at byte offsets that are multiples of their size
+    static_assert(HG != 2 || CG % 2 == 0, "4-byte scale pairs stay aligned");
+    static_assert(HG != 4 || CG % 8 == 0, "8-byte scale quads stay aligned");
 };
 
 struct GemvTmaArgs {
