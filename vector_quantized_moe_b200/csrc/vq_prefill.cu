@@ -9,8 +9,8 @@
 // The gemma-4 card ("Faster prefill") describes its Apple-GPU prefill only as
 // decoding weights in chunks before the matmul; this kernel is a new design.
 //
-// One CTA per SM, persistent over (expert, 128-row weight tile, 128-token
-// tile) work items. Warp roles:
+// One CTA per SM, persistent over (expert, 128-row weight tile, token tile)
+// work items. Warp roles:
 //   warp 0     TMA: activation tiles (fp16, 128B-swizzled, one 64-column
 //              k-step per stage) and packed-code tiles (a chunk of CH k-steps)
 //   warp 1     owns the tensor memory; one thread issues tcgen05.mma
@@ -23,9 +23,10 @@
 //              32-column blocks
 // D[row, token] = sum_k W[row, k] X[token, k]: the weight tile is the
 // M=128 operand (in tensor memory), the tokens of the bucket the N operand
-// (16..128, shared memory), so small buckets waste no M rows. Tensor memory
-// holds the accumulators (nmod x 128 columns) and 4 stages of A tiles; the MMAs of a
-// tile start once both warpgroups have read the previous tile's accumulators.
+// (16..BN, shared memory), so small buckets waste no M rows. Tensor memory
+// holds the accumulators (nmod x BN columns) and the A stages left beside
+// them; the MMAs of a tile start once both warpgroups have read the previous
+// tile's accumulators.
 // Every mbarrier wait is bounded; on a timeout the CTA records an error word,
 // stops, and frees its tensor memory.
 #include <cuda.h>
@@ -43,12 +44,23 @@ namespace vq {
 namespace {
 
 constexpr int BM = 128;             // weight rows per tile = TMEM lanes
-// tokens per tile: the accumulators of nmod modules (nmod x BN fp32 columns)
-// and 4 A stages (nmod x 32 columns each) share the 512 tensor-memory columns
-__host__ __device__ constexpr int bn_of(int nmod) { return nmod == 2 ? 128 : 256; }
 constexpr int NWG = 2;              // dequant/epilogue warpgroups (take k-steps in turn)
 constexpr int NTHREADS = 64 + 128 * NWG;   // TMA warp, MMA warp, the warpgroups
 constexpr int A_COLS = 32;          // tensor-memory columns of one 128 x 64 fp16 weight tile
+constexpr int TMEM_COLS = 512;
+// Tokens per tile. One M = 128, K = 16 instruction costs the same for any
+// N <= 192, so gate/up takes 192-token tiles: its two fp32 accumulators
+// (2 x 192 columns) leave 128 tensor-memory columns, two A stages of both
+// modules' weight tiles. down (one module) takes 256-token tiles.
+__host__ __device__ constexpr int bn_of(int nmod) { return nmod == 2 ? 192 : 256; }
+// A stages (decoded weight tiles of the nmod modules) in tensor memory: what
+// the accumulators leave, at most 4
+__host__ __device__ constexpr int a_stages_of(int nmod)
+{
+    return (TMEM_COLS - nmod * bn_of(nmod)) / (nmod * A_COLS) < 4 ? (TMEM_COLS - nmod * bn_of(nmod)) / (nmod * A_COLS)
+                                                                    : 4;
+}
+static_assert(a_stages_of(2) >= NWG && a_stages_of(1) >= NWG, "each warpgroup needs an A stage of its own");
 
 __host__ __device__ constexpr int chunk_steps(int kb)
 {
@@ -60,10 +72,14 @@ __host__ __device__ constexpr int chunk_steps(int kb)
 
 __host__ __device__ constexpr int log2i(int v) { return v <= 1 ? 0 : 1 + log2i(v / 2); }
 
-constexpr int B_STAGES = 4;           // activation tiles in shared memory (= A stages in tensor memory)
+constexpr int B_STAGES = 4;           // at most this many activation tiles in shared memory
 constexpr int CODE_STAGES = 2;
 constexpr long SMEM_LIMIT = 227L * 1024;
-constexpr long SMEM_RESERVE = 1024 + 17L * 1024;   // alignment slack, tile table (E <= 4096), barriers
+// the codebook replica count is sized for this many activation stages, the
+// alignment slack, barriers and a tile table of up to 1024 experts (more
+// experts take activation stages instead)
+__host__ __device__ constexpr int design_b_stages(int nmod) { return nmod == 2 ? 3 : 4; }
+constexpr long SMEM_RESERVE = 1024 + 1024 + 4L * 1024;
 
 // bytes of one code stage of one module: the chunk's packed codes of BM rows,
 // then the scales of an 8-group block
@@ -76,7 +92,7 @@ __host__ __device__ constexpr long code_stage_bytes(int d, int bits)
 // fit next to the operand and code stages
 __host__ __device__ constexpr int prefill_log_rep(int d, int bits, int nmod)
 {
-    const long left = SMEM_LIMIT - SMEM_RESERVE - (long)B_STAGES * bn_of(nmod) * 128 -
+    const long left = SMEM_LIMIT - SMEM_RESERVE - (long)design_b_stages(nmod) * bn_of(nmod) * 128 -
                       (long)CODE_STAGES * nmod * code_stage_bytes(d, bits);
     int lr = 0;
     while (lr < 4 && (long)nmod * (1L << bits) * d * 2 * (2L << lr) <= left)
@@ -285,8 +301,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
     char *sm_cb = reinterpret_cast<char *>(smem + a.off_cb);
     int *tiles = reinterpret_cast<int *>(smem + a.off_tiles);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + a.off_bar);
-    uint64_t *full_a = bars, *full_b = bars + a.sa, *empty = bars + 2 * a.sa;
-    uint64_t *full_c = bars + 3 * a.sa, *empty_c = full_c + a.sc;
+    constexpr int SAT = a_stages_of(NMOD);
+    uint64_t *full_a = bars;                                      // A stages (tensor memory)
+    uint64_t *full_b = bars + 2 * SAT, *empty_b = full_b + a.sa;  // activation stages
+    uint64_t *full_c = empty_b + a.sa, *empty_c = full_c + a.sc;  // code stages
+    // with as many A stages as activation stages, k-step k uses stage k % sa of both, and one
+    // commit per k-step frees both
+    const bool a_alias = SAT == a.sa;
+    uint64_t *empty_a = a_alias ? empty_b : bars + SAT;
     uint64_t *acc_full = empty_c + a.sc, *acc_empty = acc_full + 1, *drain_bar = acc_empty + 1;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(drain_bar + 1);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 2);
@@ -304,10 +326,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
             (m == 0 ? a.mod[0].codebook : a.mod[1].codebook)[(slot >> log_rep) * D + comp];
     }
     if (threadIdx.x == 0) {
-        for (int s = 0; s < a.sa; ++s) {
+        for (int s = 0; s < SAT; ++s) {
             mbar_init(&full_a[s], 128);
+            mbar_init(&bars[SAT + s], 1);
+        }
+        for (int s = 0; s < a.sa; ++s) {
             mbar_init(&full_b[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty_b[s], 1);
         }
         for (int s = 0; s < a.sc; ++s) {
             mbar_init(&full_c[s], 1);
@@ -319,9 +344,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    // accumulators: nmod x BN columns; then sa stages of nmod A tiles
+    // accumulators: nmod x BN columns; then SAT stages of nmod A tiles
     const uint32_t acc_cols = (uint32_t)nmod * BN;
-    const uint32_t tmem_cols = 512;
+    const uint32_t tmem_cols = TMEM_COLS;
+    static_assert(NMOD * BN + SAT * NMOD * A_COLS <= TMEM_COLS, "tensor memory");
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(tmem_cols));
@@ -368,17 +394,27 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
 
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
+        // Two independent streams in work-item order: code chunks (into sc stages) and activation
+        // tiles (into sa stages). One thread tests both (without blocking) and issues whichever has
+        // a free stage, so a code chunk never waits behind activation stages that only the MMAs
+        // free. A wait gives up after wait_limit idle polls.
         if (lane == 0) {
             uint32_t ks = 0, st = 0, ph = 0, cks = 0, cst = 0, cph = 0;   // operand / code stage counters
-            bool ok = true;
-            for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-                const Item itm = item_of<BN>(it, MT, tiles, n_act, a.active, a.offsets);
-                int prow0[2];
+            long itc = blockIdx.x, itb = blockIdx.x;   // the streams' current work items
+            int c = 0, kb = 0;                         // next chunk / k-step within them
+            int prow0[2] = {0, 0};
+            int q0 = 0;
+            if (itc < n_items) {
+                const Item itm = item_of<BN>(itc, MT, tiles, n_act, a.active, a.offsets);
                 for (int m = 0; m < nmod; ++m)
                     prow0[m] = tile_prow0(a.mod[m], itm.e, itm.m0);
-                for (int c = 0; c < nchunks && ok; ++c) {
-                    if (!(ok = mbar_wait(&empty_c[cst], cph ^ 1, abort_flag, a.err, 1, a.wait_limit)))
-                        break;
+                q0 = itm.q0;
+            }
+            bool ok = a.wait_limit != 0 || n_items <= blockIdx.x || mbar_give_up(abort_flag, a.err, 1);
+            uint32_t idle = 0;   // polls since the last issue
+            while (ok && (itc < n_items || itb < n_items)) {
+                bool did = false;
+                if (itc < n_items && mbar_test_wait(&empty_c[cst], cph ^ 1)) {
                     mbar_expect_tx(&full_c[cst], (uint32_t)(nmod * (a.scale_tma ? CODE_STAGE : BM * P::CHW * 4)));
                     for (int m = 0; m < nmod; ++m) {
                         uint8_t *stg = sm_c + ((size_t)cst * nmod + m) * CODE_STAGE;
@@ -392,17 +428,41 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                         cst = 0;
                         cph ^= 1;
                     }
-                    for (int j = 0; j < P::CH; ++j) {
-                        if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag, a.err, 2, a.wait_limit)))
-                            break;
-                        mbar_expect_tx(&full_b[st], (uint32_t)B_TILE);
-                        tma_load_2d(sm_b + (size_t)st * B_TILE, &a.tmap_b, (c * P::CH + j) * 64, itm.q0, &full_b[st]);
-                        ++ks;
-                        if (++st == (uint32_t)a.sa) {
-                            st = 0;
-                            ph ^= 1;
+                    if (++c == nchunks) {
+                        c = 0;
+                        itc += gridDim.x;
+                        if (itc < n_items) {
+                            const Item itm = item_of<BN>(itc, MT, tiles, n_act, a.active, a.offsets);
+                            for (int m = 0; m < nmod; ++m)
+                                prow0[m] = tile_prow0(a.mod[m], itm.e, itm.m0);
                         }
                     }
+                    did = true;
+                }
+                if (itb < n_items && mbar_test_wait(&empty_b[st], ph ^ 1)) {
+                    if (kb == 0)
+                        q0 = item_of<BN>(itb, MT, tiles, n_act, a.active, a.offsets).q0;
+                    mbar_expect_tx(&full_b[st], (uint32_t)B_TILE);
+                    tma_load_2d(sm_b + (size_t)st * B_TILE, &a.tmap_b, kb * 64, q0, &full_b[st]);
+                    ++ks;
+                    if (++st == (uint32_t)a.sa) {
+                        st = 0;
+                        ph ^= 1;
+                    }
+                    if (++kb == ksteps) {
+                        kb = 0;
+                        itb += gridDim.x;
+                    }
+                    did = true;
+                }
+                if (did) {
+                    idle = 0;
+                } else if (++idle >= a.wait_limit) {
+                    ok = mbar_give_up(abort_flag, a.err, 2);
+                } else {
+                    if ((idle & 63) == 63 && *abort_flag)
+                        ok = false;
+                    __nanosleep(32);   // leave the issue slots to the dequant warps of this sub-partition
                 }
             }
             // the loads issued have landed before the CTA leaves (the last use of each stage): after
@@ -415,7 +475,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            uint32_t st = 0, ph = 0, nacc = 0;
+            uint32_t ast = 0, aph = 0, st = 0, ph = 0, nacc = 0;   // A stage / activation stage counters
             bool ok = true, issued = false;
             for (long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
                 const Item itm = item_of<BN>(it, MT, tiles, n_act, a.active, a.offsets);
@@ -427,7 +487,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                 ++nacc;
                 tc_fence_after();
                 for (int k = 0; k < ksteps; ++k) {
-                    if (!(ok = mbar_wait(&full_a[st], ph, abort_flag, a.err, 4, a.wait_limit)))
+                    if (!(ok = mbar_wait(&full_a[ast], aph, abort_flag, a.err, 4, a.wait_limit)))
                         break;
                     if (!(ok = mbar_wait(&full_b[st], ph, abort_flag, a.err, 5, a.wait_limit)))
                         break;
@@ -438,14 +498,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
 #pragma unroll
                     for (int k16 = 0; k16 < 4; ++k16)
                         for (int m = 0; m < nmod; ++m) {
-                            const uint32_t a_tmem = tmem + acc_cols + (st * nmod + m) * A_COLS;
+                            const uint32_t a_tmem = tmem + acc_cols + (ast * nmod + m) * A_COLS;
                             umma_ts(tmem + m * BN, a_tmem + 8 * k16, bdesc + 2 * k16, idesc, (k | k16) != 0);
                         }
-                    umma_commit(&empty[st]);
+                    umma_commit(&empty_b[st]);
+                    if (!a_alias)
+                        umma_commit(&empty_a[ast]);
                     issued = true;
                     if (++st == (uint32_t)a.sa) {
                         st = 0;
                         ph ^= 1;
+                    }
+                    if (++ast == (uint32_t)SAT) {
+                        ast = 0;
+                        aph ^= 1;
                     }
                 }
                 if (ok)
@@ -519,7 +585,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                             dequant_step<D, BITS, P::L, JJ>(crow[1], sm_cb + cb_bytes, rep_off, sfetch(1, JJ),
                                                             bfetch(1, JJ), lrow[1] >= 0,
                                                             *reinterpret_cast<uint32_t(*)[32]>(o + 32));
-                        if (!(ok = mbar_wait(&empty[st], ph ^ 1, abort_flag, a.err, 7, a.wait_limit)))
+                        if (!(ok = mbar_wait(&empty_a[st], ph ^ 1, abort_flag, a.err, 7, a.wait_limit)))
                             return;
                         tc_fence_after();   // the stage's previous MMA has read it
                         if constexpr (NMOD == 2)
@@ -530,7 +596,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                         tc_fence_before();
                         mbar_arrive(&full_a[st]);
                     }
-                    if (++st == (uint32_t)a.sa) {
+                    if (++st == (uint32_t)SAT) {
                         st = 0;
                         ph ^= 1;
                     }
@@ -726,7 +792,7 @@ SmemPlan smem_plan(int nmod, int d, int bits, int E)
         (uint32_t)align_up((size_t)nmod * ((size_t)1 << bits) * d * 2 << prefill_log_rep(d, bits, nmod), 128);
     const uint32_t tiles = (uint32_t)align_up((size_t)(E + 1) * 4, 128);
     SmemPlan p{};
-    for (int sa = B_STAGES; sa >= 2; --sa) {   // tensor memory holds up to B_STAGES A stages
+    for (int sa = B_STAGES; sa >= 2; --sa) {
         p.sa = sa;
         p.sc = CODE_STAGES;
         p.off_a = 0;
@@ -735,7 +801,7 @@ SmemPlan smem_plan(int nmod, int d, int bits, int E)
         p.off_cb = p.off_c + p.sc * code_stage;
         p.off_tiles = p.off_cb + cb;
         p.off_bar = (uint32_t)align_up(p.off_tiles + tiles, 8);
-        p.total = p.off_bar + (3 * sa + 2 * p.sc + 3) * 8 + 16 + 1024;
+        p.total = p.off_bar + (2 * sa + 2 * a_stages_of(nmod) + 2 * p.sc + 3) * 8 + 16 + 1024;
         if (p.total <= limit + 1024)
             return p;
     }
