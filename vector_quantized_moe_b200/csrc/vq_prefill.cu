@@ -62,12 +62,34 @@ __host__ __device__ constexpr int a_stages_of(int nmod)
 }
 static_assert(a_stages_of(2) >= NWG && a_stages_of(1) >= NWG, "each warpgroup needs an A stage of its own");
 
-__host__ __device__ constexpr int chunk_steps(int kb)
+// k-steps whose code bits fill whole 16-byte units (a TMA box of code words
+// starts on a 16-byte boundary)
+__host__ __device__ constexpr int chunk_steps_aligned(int kb)
 {
     int ch = 1;
     while ((ch * kb) % 128)
         ++ch;
     return ch;
+}
+
+// Steps per code chunk. Where whole 16-byte units take 4 or more steps (e.g.
+// d = 4 with an odd code width: 144, 176 or 208 bits a step), a chunk is half
+// that: its bits are then an odd multiple of 64, and the odd chunks start 64
+// bits into their box, which begins on the 16-byte boundary below them.
+__host__ __device__ constexpr bool chunk_split(int kb) { return chunk_steps_aligned(kb) >= 4; }
+__host__ __device__ constexpr int chunk_steps(int kb)
+{
+    return chunk_split(kb) ? chunk_steps_aligned(kb) / 2 : chunk_steps_aligned(kb);
+}
+// words per row of a chunk's box: its bits, plus the 64-bit lead of odd chunks
+__host__ __device__ constexpr int chunk_words(int kb)
+{
+    return chunk_split(kb) ? (64 + chunk_steps(kb) * kb + 127) / 128 * 4 : chunk_steps(kb) * kb / 32;
+}
+// first word of chunk c's box (a multiple of 4)
+__host__ __device__ constexpr int chunk_x(int kb, int c)
+{
+    return (c * chunk_steps(kb) * kb - (chunk_split(kb) && (c & 1) ? 64 : 0)) / 32;
 }
 
 __host__ __device__ constexpr int log2i(int v) { return v <= 1 ? 0 : 1 + log2i(v / 2); }
@@ -85,7 +107,7 @@ constexpr long SMEM_RESERVE = 1024 + 1024 + 4L * 1024;
 // then the scales of an 8-group block
 __host__ __device__ constexpr long code_stage_bytes(int d, int bits)
 {
-    return (long)128 * (chunk_steps((64 / d) * bits) * ((64 / d) * bits) / 32) * 4 + 128 * 16;
+    return (long)128 * chunk_words((64 / d) * bits) * 4 + 128 * 16;
 }
 
 // codebook replicas in shared memory (log2, at most 16 replicas): as many as
@@ -103,8 +125,9 @@ __host__ __device__ constexpr int prefill_log_rep(int d, int bits, int nmod)
 template <int D, int BITS, int NMOD>
 struct PG {
     static constexpr int KB = (64 / D) * BITS;       // code bits of one row per 64-column step
-    static constexpr int CH = chunk_steps(KB);       // steps per code chunk (whole 16-byte units)
-    static constexpr int CHW = CH * KB / 32;         // words per row per chunk
+    static constexpr int CH = chunk_steps(KB);       // steps per code chunk
+    static constexpr bool SPLIT = chunk_split(KB);   // odd chunks start 64 bits into their box
+    static constexpr int CHW = chunk_words(KB);      // words per row of a chunk's box
     static constexpr uint32_t MASK = (1u << BITS) - 1u;
     static constexpr int LREP = prefill_log_rep(D, BITS, NMOD);
     static constexpr int L = LREP + 1 + log2i(D);    // code -> byte offset of its replica row
@@ -154,14 +177,16 @@ __device__ __forceinline__ uint32_t code_at(const uint32_t (&w)[NW], int pos)
     return __funnelshift_r(w[wi], w[wi + 1], sh) & ((1u << BITS) - 1u);
 }
 
-// The 16-byte-aligned words of a chunk row that hold k-step JJ's code bits.
-template <int D, int BITS, int JJ>
+// The 16-byte-aligned words of a chunk row that hold k-step JJ's code bits,
+// the chunk's first code starting OFF bits into the row.
+template <int D, int BITS, int JJ, int OFF>
 struct Win {
     static constexpr int KB = (64 / D) * BITS;
-    static constexpr int W0 = ((JJ * KB) / 32) & ~3;
-    static constexpr int W1 = (((JJ * KB + KB + 31) / 32) + 3) & ~3;
+    static constexpr int W0 = ((OFF + JJ * KB) / 32) & ~3;
+    static constexpr int W1 = (((OFF + JJ * KB + KB + 31) / 32) + 3) & ~3;
     static constexpr int NV = (W1 - W0) / 4;
-    static constexpr int BASE = JJ * KB - 32 * W0;
+    static constexpr int BASE = OFF + JJ * KB - 32 * W0;
+    static_assert(W1 <= chunk_words(KB), "the window stays inside the chunk's box");
 };
 
 // Byte offset of the lane's replica of the code at bit `pos` of the window:
@@ -189,11 +214,11 @@ __device__ __forceinline__ uint32_t entry_off(const uint32_t (&w)[NW], int pos, 
 // row's bias (one fp16 fused multiply-add, rounded to nearest; the bias is 0
 // without the affine arm), as 32 words o[c] = weights (2c, 2c+1), the layout
 // of one tensor-memory lane of the MMA's A operand.
-template <int D, int BITS, int L, int JJ>
+template <int D, int BITS, int L, int JJ, int OFF>
 __device__ __forceinline__ void dequant_step(const uint8_t *crow, const char *cb, uint32_t rep_off, uint32_t s2,
                                              uint32_t b2, bool live, uint32_t (&o)[32])
 {
-    using W = Win<D, BITS, JJ>;
+    using W = Win<D, BITS, JJ, OFF>;
     constexpr int NC = 64 / D;
     uint32_t w[4 * W::NV];
 #pragma unroll
@@ -418,7 +443,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                     mbar_expect_tx(&full_c[cst], (uint32_t)(nmod * (a.scale_tma ? CODE_STAGE : BM * P::CHW * 4)));
                     for (int m = 0; m < nmod; ++m) {
                         uint8_t *stg = sm_c + ((size_t)cst * nmod + m) * CODE_STAGE;
-                        tma_load_2d(stg, &a.tmap_c[m], c * P::CHW, prow0[m], &full_c[cst]);
+                        tma_load_2d(stg, &a.tmap_c[m], chunk_x(P::KB, c), prow0[m], &full_c[cst]);
                         if (a.scale_tma)
                             tma_load_2d(stg + BM * P::CHW * 4, &a.tmap_s[m], (c * P::CH) & ~7, prow0[m],
                                         &full_c[cst]);
@@ -569,6 +594,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                     const uint32_t b = (bi && prow[m] >= 0) ? ldg_u16(bi + prow[m] * a.mod[m].ngroups + c * P::CH + j) : 0u;
                     return b | (b << 16);
                 };
+                // the chunk's steps, its first code OFF bits into the box row
+                auto chunk = [&](auto off_c) {
+                constexpr int OFF = decltype(off_c)::value;
                 auto step = [&](auto jj_c) {
                     constexpr int JJ = decltype(jj_c)::value;
                     if (!ok)
@@ -579,12 +607,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                         // stage, stored with one instruction); the wait for the stage's previous
                         // MMA overlaps the decode
                         uint32_t o[32 * NMOD];
-                        dequant_step<D, BITS, P::L, JJ>(crow[0], sm_cb, rep_off, sfetch(0, JJ), bfetch(0, JJ),
-                                                        lrow[0] >= 0, *reinterpret_cast<uint32_t(*)[32]>(o));
+                        dequant_step<D, BITS, P::L, JJ, OFF>(crow[0], sm_cb, rep_off, sfetch(0, JJ), bfetch(0, JJ),
+                                                             lrow[0] >= 0, *reinterpret_cast<uint32_t(*)[32]>(o));
                         if constexpr (NMOD == 2)
-                            dequant_step<D, BITS, P::L, JJ>(crow[1], sm_cb + cb_bytes, rep_off, sfetch(1, JJ),
-                                                            bfetch(1, JJ), lrow[1] >= 0,
-                                                            *reinterpret_cast<uint32_t(*)[32]>(o + 32));
+                            dequant_step<D, BITS, P::L, JJ, OFF>(crow[1], sm_cb + cb_bytes, rep_off, sfetch(1, JJ),
+                                                                 bfetch(1, JJ), lrow[1] >= 0,
+                                                                 *reinterpret_cast<uint32_t(*)[32]>(o + 32));
                         if (!(ok = mbar_wait(&empty_a[st], ph ^ 1, abort_flag, a.err, 7, a.wait_limit)))
                             return;
                         tc_fence_after();   // the stage's previous MMA has read it
@@ -604,6 +632,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                 [&]<int... J>(std::integer_sequence<int, J...>) {
                     (step(std::integral_constant<int, J>{}), ...);
                 }(std::make_integer_sequence<int, P::CH>{});
+                };
+                if constexpr (P::SPLIT) {
+                    if (c & 1)
+                        chunk(std::integral_constant<int, 64>{});
+                    else
+                        chunk(std::integral_constant<int, 0>{});
+                } else {
+                    chunk(std::integral_constant<int, 0>{});
+                }
                 mbar_arrive(&empty_c[cst]);
                 if (++cst == (uint32_t)a.sc) {
                     cst = 0;
@@ -771,13 +808,11 @@ bool map_codes(CUtensorMap *map, const ModDev &m)
                       (uint32_t)chw_of(m.d, m.bits), BM, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-int chw_of(int d, int bits)
-{
-    const int kb = (64 / d) * bits;
-    return chunk_steps(kb) * kb / 32;
-}
+int chw_of(int d, int bits) { return chunk_words((64 / d) * bits); }
 
-int ch_of(int d, int bits) { return chunk_steps((64 / d) * bits); }
+// k-steps a module's columns must be a multiple of (whole 16-byte units; a
+// split geometry then has an even number of chunks)
+int ch_of(int d, int bits) { return chunk_steps_aligned((64 / d) * bits); }
 
 struct SmemPlan {
     int sa, sc;
