@@ -112,14 +112,15 @@ def test_decode_step_replays_from_a_cuda_graph():
 @pytest.mark.parametrize("T", [256, 2048])
 def test_skipzero_layer_decode_bitwise_repeatable_from_the_first_call(T):
     # the full-size skipzero + mixed-geometry layer (live bitmaps, d=2/10-bit gate/up, d=8/12-bit down): the
-    # first call on a fresh workspace and the calls after it give the same bits
+    # first call on a fresh workspace and the calls after it give the same bits (16 calls: a race that
+    # changed a few sums in about one call in eight shows up here)
     from helpers import row_words_fn
     mds = wl.layer_modules(wl.SKIPZERO_MIXED, raw=False, row_words=row_words_fn())
     layer = vq.MoELayer(*[lib_module(m) for m in mds])
     del mds
     x, lg = wl.layer_inputs(wl.SKIPZERO_MIXED, T)
     xt, lt = torch.from_numpy(x.view(np.int16)).cuda(), torch.from_numpy(lg).cuda()
-    outs = [layer.decode(xt, lt, wl.SKIPZERO_MIXED.top_k).cpu().numpy().view(np.uint32).copy() for _ in range(4)]
+    outs = [layer.decode(xt, lt, wl.SKIPZERO_MIXED.top_k).cpu().numpy().view(np.uint32).copy() for _ in range(16)]
     for o in outs[1:]:
         assert np.array_equal(o, outs[0])
     del layer

@@ -661,7 +661,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                 if (nmod == 2)
                     tmem_ld32(tmem + lane_addr + BN + cb0, u);
                 tmem_wait_ld();
-                if (a.swiglu) {
+
+                if (NMOD == 2 && a.swiglu) {
                     // the tile's 32 token columns j: the accumulators carry each token's activation
                     // scale 2^k, undone exactly; h = silu(g) u in fp32. The down GEMM reads h as fp16, so
                     // each (slot, 32-row block) is stored times 2^e, e putting the block's largest |h| in
@@ -672,20 +673,31 @@ __global__ void __launch_bounds__(NTHREADS, 1) vq_prefill_gemm_kernel(const __gr
                     if (wrow0 < a.rows) {
                         // lane j holds the inverse activation scale of column j
                         const float fl = cb0 + lane < itm.n ? a.sxinv[itm.q0 + cb0 + lane] : 0.f;
+                        // eight columns at a time, in three passes (h; the columns' largest |h|;
+                        // scaled stores), so that each pass's eight operations are independent
                         int my_e = 0;   // lane j: the exponent of column j
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int n = cb0 + j;
-                            const float f = __shfl_sync(0xFFFFFFFFu, fl, j);
-                            const float gv = __uint_as_float(g[j]) * f, uv = __uint_as_float(u[j]) * f;
-                            const float hv = __fdividef(gv, 1.f + __expf(-gv)) * uv;
-                            // the column's largest |h| over the warp's 32 rows, in every lane
-                            const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(hv) & 0x7FFFFFFFu);
-                            const int e = scale_exp(m);
-                            my_e = lane == j ? e : my_e;
-                            if (n < itm.n)
-                                reinterpret_cast<__half *>(a.out)[(long)(itm.q0 + n) * a.rows + r] =
-                                    __float2half_rn(hv * pow2f_normal(e));
+                        for (int j0 = 0; j0 < 32; j0 += 8) {
+                            float hv[8];
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const float f = __shfl_sync(0xFFFFFFFFu, fl, j0 + j);
+                                const float gv = __uint_as_float(g[j0 + j]) * f, uv = __uint_as_float(u[j0 + j]) * f;
+                                hv[j] = __fdividef(gv, 1.f + __expf(-gv)) * uv;
+                            }
+                            uint32_t mx[8];   // column j's largest |h| over the warp's 32 rows, in every lane
+#pragma unroll
+                            for (int j = 0; j < 8; ++j)
+                                mx[j] = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(hv[j]) & 0x7FFFFFFFu);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const int n = cb0 + j0 + j;
+                                const int e = scale_exp(mx[j]);
+                                my_e = lane == j0 + j ? e : my_e;
+                                if (n < itm.n)
+                                    reinterpret_cast<__half *>(a.out)[(long)(itm.q0 + n) * a.rows + r] =
+                                        __float2half_rn(hv[j] * pow2f_normal(e));
+                            }
                         }
                         if (cb0 + lane < itm.n)
                             a.hexp[(long)(itm.q0 + cb0 + lane) * a.nblk32 + (wrow0 >> 5)] = (int8_t)my_e;
@@ -851,16 +863,15 @@ cudaError_t launch_gemm(const PrefillArgs &a, int ctas, uint32_t smem, cudaStrea
     cudaError_t err = set_smem_limit_once((const void *)k, (int)smem);
     if (err != cudaSuccess)
         return err;
+    // An ordinary launch, not a programmatic one: launched early, the persistent CTAs (a whole SM's
+    // shared memory and a third of its registers each) crowd the memory-bound kernel before them
+    // off the SMs and slow it more than their own prologue gains (the 4096-token Zipf layer's step
+    // took 5.7 ms with a programmatic launch, 5.0 ms without).
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(ctas);
     cfg.blockDim = dim3(NTHREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, k, a);
 }
 
