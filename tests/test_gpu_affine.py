@@ -52,7 +52,7 @@ GEOS = [(1, 3, True), (2, 8, False), (4, 9, False), (2, 10, False)]
 
 
 @pytest.mark.parametrize("d,bits,affine", GEOS)
-@pytest.mark.parametrize("cols,rows", [(1024, 300), (256, 80)])   # TMA-staged kernel; register kernel
+@pytest.mark.parametrize("cols,rows", [(1024, 300), (256, 80)])   # TMA-staged kernel (d = 8: register); register kernel
 def test_gemv_weights_bit_exact_with_bias(d, bits, affine, cols, rows):
     md = small_module(2, rows, cols, d, bits, n_dead=17, seed=1110 + 16 * d + bits)
     om, lm = _biased(md, d * 100 + bits, affine)

@@ -161,7 +161,7 @@ def test_moe_decode_full_size(spec, T, sample):
 @pytest.mark.parametrize("d,bits", GEOS)
 @pytest.mark.parametrize("T", [1, 9])
 def test_gemv_staged_path(d, bits, T):
-    # 1024 columns (16 groups) and 300 rows with skipzero: the TMA-staged kernel
+    # 1024 columns (16 groups) and 300 rows with skipzero: the TMA-staged kernel (d = 8: the register kernel)
     # path (several 256-row items, a ragged last item, compacted live rows)
     E, rows, cols = 3, 300, 1024
     md = small_module(E, rows, cols, d, bits, n_dead=37, seed=11 * d + bits)

@@ -39,7 +39,7 @@ def _live(md, e):
 
 
 @pytest.mark.parametrize("d,bits", GEOS)
-@pytest.mark.parametrize("cols,rows", [(1024, 300), (256, 80)])   # TMA-staged kernel; register kernel
+@pytest.mark.parametrize("cols,rows", [(1024, 300), (256, 80)])   # TMA-staged kernel (d = 8: register); register kernel
 def test_gemv_weights_bit_exact(d, bits, cols, rows):
     md = small_module(3, rows, cols, d, bits, n_dead=29, seed=600 + 16 * d + bits)
     om, lm = oracle_module(md), lib_module(md)

@@ -40,7 +40,7 @@ def _per_token(got, ref, what):
         assert_close(got[t], ref[t], what=f"{what} token {t}")
 
 
-@pytest.mark.parametrize("cols,rows", [(1024, 300), (256, 80)])   # TMA-staged and register kernels
+@pytest.mark.parametrize("cols,rows", [(1024, 300), (256, 80)])   # TMA-staged (d = 8: register) and register kernels
 @pytest.mark.parametrize("d,bits", [(2, 8), (4, 9), (2, 10), (8, 12), (1, 4)])
 def test_gemv_range(cols, rows, d, bits):
     md = small_module(2, rows, cols, d, bits, n_dead=11, seed=510 + d * bits)
