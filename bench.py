@@ -78,6 +78,7 @@ def _module_bytes(md):
 KERNEL_SOURCES = {
     "grouped_gemv_gate_up_d4k512": ("vq_decode.cu", "vq_device.cuh", "vq_sm100.cuh"),
     "grouped_gemv_gate_up_d2k256": ("vq_decode.cu", "vq_device.cuh", "vq_sm100.cuh"),
+    "grouped_gemv_gate_up_d4k2048": ("vq_decode.cu", "vq_device.cuh", "vq_sm100.cuh"),
     "prefill_gemm_gate_up": ("vq_prefill.cu", "vq_device.cuh", "vq_sm100.cuh"),
 }
 
@@ -415,8 +416,8 @@ def run_ours(args):
     if not args.no_extra:
         for key, (spec_x, T_x) in OTHER_DECODE.items():
             extra[key] = measure_decode_layer(torch, vq, spec_x, T_x, dev, min(args.steps, 100), args.warmup,
-                                              traffic_tag="grouped_gemv_gate_up_d2k256" if key == "decode_d2k256_T8"
-                                              else None)
+                                              traffic_tag={"decode_d2k256_T8": "grouped_gemv_gate_up_d2k256",
+                                                           "decode_d4k2048_T16": "grouped_gemv_gate_up_d4k2048"}.get(key))
         extra["gemv_d2k256_512x1024"] = measure_gemv_single(torch, vq, dev, min(args.steps, 20), args.warmup)
         extra["prefill"] = measure_prefill(torch, vq, dev, min(args.steps, 20), args.warmup)
         extra["prefill_skipzero_T2048"] = measure_prefill(torch, vq, dev, min(args.steps, 20), args.warmup,
