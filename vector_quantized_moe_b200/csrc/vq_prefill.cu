@@ -755,8 +755,9 @@ __global__ void vq_gather_kernel(const __half *__restrict__ x16, const float *__
 // exponent E = min_b e_b (the one of its largest |h|): hs *= 2^(E - e_b), a
 // power of two <= 1, exact unless a value falls into fp16's subnormal range;
 // and the slot's pair p = perm[q] gets wh[p] = w[p] * 2^-E, the routing weight
-// that the combine applies to the down projection. One warp per slot; a lane
-// rescales whole 64-byte blocks.
+// that the combine applies to the down projection. One warp per slot; the
+// lanes take consecutive 16-byte chunks of the row, so each load and store of
+// the warp covers 512 contiguous bytes.
 __global__ void vq_hnorm_kernel(__half *__restrict__ h, const int8_t *__restrict__ hexp, long slots, int nblk,
                                 const int32_t *__restrict__ perm, const float *__restrict__ w, float *__restrict__ wh)
 {
@@ -774,23 +775,20 @@ __global__ void vq_hnorm_kernel(__half *__restrict__ h, const int8_t *__restrict
             const int p = perm[q];
             wh[p] = w[p] * pow2f(-E);
         }
-        for (int b = lane; b < nblk; b += 32) {
-            const int d = max(E - (int)eq[b], -64);   // beyond 2^-64 every fp16 value becomes 0
+        uint4 *row = reinterpret_cast<uint4 *>(h + q * nblk * 32);
+        for (int c = lane; c < nblk * 4; c += 32) {   // chunk c: 8 values of block c / 4
+            const int d = max(E - (int)eq[c >> 2], -64);   // beyond 2^-64 every fp16 value becomes 0
             if (d >= 0)
                 continue;
             const float sc = pow2f(d);
-            uint4 *p = reinterpret_cast<uint4 *>(h + (q * nblk + b) * 32);
+            uint4 x = row[c];
+            __half2 *hw = reinterpret_cast<__half2 *>(&x);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                uint4 x = p[v];
-                __half2 *hw = reinterpret_cast<__half2 *>(&x);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 f = __half22float2(hw[i]);   // exact; the product too, then one rounding
-                    hw[i] = __floats2half2_rn(f.x * sc, f.y * sc);
-                }
-                p[v] = x;
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = __half22float2(hw[i]);   // exact; the product too, then one rounding
+                hw[i] = __floats2half2_rn(f.x * sc, f.y * sc);
             }
+            row[c] = x;
         }
     }
 }
