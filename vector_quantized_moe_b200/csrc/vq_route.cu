@@ -432,7 +432,8 @@ __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_fused_kernel(const flo
 }
 
 // Large T: many CTAs route, then one CTA buckets.
-constexpr int ROUTE_TOKENS_PER_CTA = 256;
+constexpr int ROUTE_TOKENS_PER_CTA = 256;     // up to this many tokens: the fused one-CTA routing
+constexpr int TOPK_TOKENS_PER_CTA = 32;       // more: top-k CTAs of this many tokens (2 per warp), then bucketing
 
 __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_topk_kernel(const float *logits, int T, int E, int k,
                                                                      int renorm, int32_t *ids, float *w,
@@ -444,9 +445,9 @@ __global__ void __launch_bounds__(ROUTE_THREADS) vq_route_topk_kernel(const floa
     if (err && blockIdx.x == 0 && threadIdx.x == 0)
         *err = 0;
     zero_spans(zero, blockIdx.x, gridDim.x);
-    const int t0 = blockIdx.x * ROUTE_TOKENS_PER_CTA;
-    convert_rows(x, x16, xinv, t0, min(T, t0 + ROUTE_TOKENS_PER_CTA), H, 0, blockDim.x >> 5);
-    route_range(logits, t0, min(T, t0 + ROUTE_TOKENS_PER_CTA), E, k, renorm, ids, w, 0, blockDim.x >> 5);
+    const int t0 = blockIdx.x * TOPK_TOKENS_PER_CTA;
+    convert_rows(x, x16, xinv, t0, min(T, t0 + TOPK_TOKENS_PER_CTA), H, 0, blockDim.x >> 5);
+    route_range(logits, t0, min(T, t0 + TOPK_TOKENS_PER_CTA), E, k, renorm, ids, w, 0, blockDim.x >> 5);
 }
 
 __global__ void __launch_bounds__(BUCKET_THREADS) vq_bucket_kernel(const int32_t *ids, int npairs, int E,
@@ -519,7 +520,7 @@ cudaError_t launch_route(const float *logits, int T, int E, int k, int renorm, i
     if (fused)
         return launch_ex(vq_route_fused_kernel, dim3(1 + zctas), dim3(ROUTE_THREADS), smem, s, pdl, logits, T, E, k,
                          renorm, ids, w, offsets, perm, pos, active, n_active, passes, n_passes, x, x16, xinv, H, errw, z);
-    const int ctas = (T + ROUTE_TOKENS_PER_CTA - 1) / ROUTE_TOKENS_PER_CTA;
+    const int ctas = (T + TOPK_TOKENS_PER_CTA - 1) / TOPK_TOKENS_PER_CTA;
     // many tokens: the activations are converted by a launch of their own, over the whole GPU
     cudaError_t err = launch_ex(vq_route_topk_kernel, dim3(ctas), dim3(ROUTE_THREADS), 0, s, pdl, logits, T, E, k,
                                 renorm, ids, w, (const uint16_t *)nullptr, (__half *)nullptr, (float *)nullptr, H, errw,
